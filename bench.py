@@ -1,0 +1,356 @@
+"""Benchmark of the grouped top-k MoE block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = the whole block (router logits, route, permute, expert FFNs with
+the shared MLP, combine) through ``moe_forward`` on one batch of synthetic
+tokens already resident in HBM. Weak scaling: every rank runs its own batch
+against its own weight replica; no data-path collective. Rank 0 prints one
+JSON line.
+
+``--impl reference`` times the CPU oracle (the reference arm: a plain fp64
+program, no GPU work) on bounded token samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from grouped_top_routing_b200 import inputs as G  # noqa: E402
+
+METRIC = "MoE-block tokens/s at 1 B200; HBM GB/s (decode) & TFLOPS (prefill) vs roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "ling26_flash_t512"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of one step (counted from the step's actual routing)
+# ---------------------------------------------------------------------------
+
+def algorithmic(wl, T, n_unique):
+    """Bytes and flops the block must move / perform once, given the number of
+    distinct routed experts the batch touched."""
+    H, E, k, I, Is = (wl["hidden_size"], wl["num_experts"], wl["num_experts_per_tok"],
+                      wl["moe_intermediate_size"], wl["shared_width"])
+    R = T * k
+    w_gate_up = (n_unique * 2 * I + 2 * Is) * H * 2
+    w_down = (n_unique * I + Is) * H * 2
+    gate_up_bytes = w_gate_up + (R + T) * H * 2 + (R * I + T * Is) * 2   # weights + x rows in + h out
+    down_bytes = w_down + (R * I + T * Is) * 2 + (R + T) * H * 2          # weights + h in + rows out
+    step_bytes = (w_gate_up + w_down + E * H * 4 + 2 * T * H * 2)         # weights + router + x in + y out
+    flops = R * 6 * H * I + T * 6 * H * Is + 2 * T * H * E
+    return dict(gate_up_bytes=gate_up_bytes, down_bytes=down_bytes, step_bytes=step_bytes, flops=flops)
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def time_oracle(wl, inp, token_rows):
+    """Seconds the oracle takes for the block on the given token rows."""
+    from oracle import moe_oracle as O
+    sub = dict(inp)
+    sub["x"] = inp["x"][token_rows]
+    t0 = time.perf_counter()
+    O.moe_block(sub, wl)
+    return time.perf_counter() - t0
+
+
+def run_reference(args):
+    rank = _env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    wl = G.workload(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = G.make_inputs(wl, seed=0, device=dev)  # generation is not timed; the oracle pulls rows to the host
+    T = inp["tokens"]
+    per_step = args.ref_sample
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        time_oracle(wl, inp, torch.from_numpy(rng.choice(T, per_step, replace=False)).to(dev))
+    secs = []
+    for _ in range(args.steps):
+        secs.append(time_oracle(wl, inp, torch.from_numpy(rng.choice(T, per_step, replace=False)).to(dev)))
+    total = sum(secs)
+    value = per_step * args.steps / total
+    sample = f"{per_step} random tokens of the {T}-token batch per step, fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch.distributed as dist
+    from grouped_top_routing_b200 import build as B
+    B.build()
+    from grouped_top_routing_b200 import moe as M
+
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local = _env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = G.workload(args.workload)
+    inp = G.make_inputs(wl, seed=0, device=dev)
+    T = inp["tokens"]
+    if rank > 0:  # each rank its own batch (weak scaling), same weights
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + rank)
+        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=dev).to(torch.bfloat16)
+    ws = M.Workspace(wl, T, device=dev)
+    y = torch.empty_like(inp["x"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x=None):
+        return M.moe_forward(wl, inp["x"] if x is None else x, inp["router_w"], inp["expert_bias"],
+                             inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"], inp["ws_down"], ws, y=y)
+
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check()
+
+    # routing of this batch: distinct experts touched (algorithmic bytes)
+    _, idx, _ = M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                              inp["ws_gate_up"], inp["ws_down"], ws, return_routing=True)
+    n_unique = int(torch.unique(idx).numel())
+    work = algorithmic(wl, T, n_unique)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = M.launch_count()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.zero_()  # L2 flush, outside the timed events
+            M.set_kernel_timer(args.kernel, kev[i][0], kev[i][1])
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        M.set_kernel_timer(args.kernel)
+        torch.cuda.synchronize(dev)
+    launches = M.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ws.check()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_ms = [a.elapsed_time(b) for a, b in kev]
+    total_ms = sum(step_ms)
+
+    # e2e: host pinned x in, host y out, through the same public call
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        eev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / K
+    value = T * world / (ms_per_step / 1e3)
+    e2e_value = T * world / (e2e_ms / K / 1e3)
+
+    pk = peaks()
+    kms = statistics.mean(kern_ms)
+    kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
+    achieved = kbytes / (kms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": args.kernel, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
+                "algorithmic_bytes": kbytes, "kernel_ms": kms}
+    step_gbs = work["step_bytes"] / (ms_per_step / 1e3) / 1e9
+    step_tflops = work["flops"] / (ms_per_step / 1e3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = torch.arange(0, T, max(1, T // args.cpu_sample), device=dev)[:args.cpu_sample]
+        secs = time_oracle(wl, inp, rows)
+        cpu = {"value": len(rows) / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{len(rows)} evenly spaced tokens of the {T}-token batch, fp64 numpy oracle, one pass",
+               "seconds": secs}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": T, "hidden_size": wl["hidden_size"],
+                   "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
+                   "n_group": wl["n_group"], "topk_group": wl["topk_group"],
+                   "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
+                   "experts_touched": n_unique, "parallelism": f"replicas x{world} (token batches)",
+                   "l2": "256 MiB L2 flush between timed steps; weights 6.4 GB >> 126 MB L2"},
+        "step_hbm_gbs": step_gbs, "step_tflops": step_tflops,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2)},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(G.WORKLOADS))
+    ap.add_argument("--kernel", default="expert_gate_up", choices=["expert_gate_up", "expert_down"])
+    ap.add_argument("--cpu-sample", type=int, default=64)
+    ap.add_argument("--ref-sample", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -7,8 +7,8 @@ library has not been built: there is no fallback.
 """
 
 _BINDING_NAMES = (
-    "MoeConfig", "MoeError", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
-    "moe_workspace_size", "moe_router_logits", "lib", "library_path", "config_from_workload",
+    "MoeConfig", "MoeError", "Workspace", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+    "moe_forward", "moe_workspace_size", "moe_router_logits", "lib", "library_path", "config_from_workload",
 )
 
 

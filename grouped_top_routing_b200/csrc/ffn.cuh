@@ -1,0 +1,29 @@
+// Arguments of the expert FFN kernels (routed experts + shared MLP).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct FfnArgs {
+  const uint16_t* x;          // [T, H]
+  int64_t T;
+  int H, I, Is, k, E;
+  const int32_t* offsets;     // [E+1]
+  const int32_t* tok_of;      // [T*k]
+  const int32_t* active;      // [num_active]
+  WsHeader* hdr;              // num_active, error word
+  const float* topk_w;        // [T*k] or null
+  const uint16_t* w_gate_up;  // [E, 2I, H]
+  const uint16_t* w_down;     // [E, H, I]
+  const uint16_t* ws_gate_up; // [2Is, H] or null
+  const uint16_t* ws_down;    // [H, Is]
+  uint16_t* h_perm;           // [T*k, I]
+  uint16_t* h_shared;         // [T, Is]
+  uint16_t* y_slots;          // [T*k, H]
+  uint16_t* shared_out;       // [T, H]
+};
+
+cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s);
+
+}  // namespace moe

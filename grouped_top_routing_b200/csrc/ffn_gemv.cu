@@ -1,0 +1,283 @@
+// Decode expert FFN: weight-streaming GEMV over the selected experts only.
+//
+// The page "Ling-3.0-flash-GGUF" (section "Measured performance") bounds
+// decode by memory bandwidth: only the selected experts' weights are read.
+// The expert is the SwiGLU MLP of mlxcel issue #838 ("Architecture notes";
+// "Shared experts are one wide MLP, not N separate experts"):
+//   h = silu(gate x) * (up x),  y = down h.
+//
+// Work items are single weight rows (gate/up pass) or blocks of kDownRows
+// rows (down pass) of the experts in the compacted active list written by the
+// permutation, plus the shared MLP's rows. One warp per item: lanes stride the
+// row in 16-byte chunks (ld.global.nc, no L1 allocation), every token routed
+// to that expert is multiplied against the chunk, and the warp reduces with
+// shuffles. Tokens are taken kTok at a time; an expert with more rows streams
+// its weights again per group of kTok (those re-reads hit L2).
+#include "common.cuh"
+#include "ffn.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kTok = 8;       // tokens per pass
+constexpr int kUnroll = 4;    // 16-byte chunks in flight per lane per row
+constexpr int kDownRows = 4;  // rows per down-projection item
+
+// Resolves the rows [r0, r0 + m) of one active expert, clamped to [0, T*k).
+__device__ __forceinline__ bool expert_rows(const FfnArgs& a, int aidx, int& e, int64_t& r0, int64_t& m) {
+  e = a.active[aidx];
+  if (e < 0 || e >= a.E) {
+    record_error(a.hdr, MOE_ERR_DEVICE_CHECK, aidx);
+    return false;
+  }
+  const int64_t R = a.T * a.k;
+  int64_t lo = a.offsets[e], hi = a.offsets[e + 1];
+  if (lo < 0 || hi > R || hi < lo) {
+    record_error(a.hdr, MOE_ERR_DEVICE_CHECK, e);
+    return false;
+  }
+  r0 = lo;
+  m = hi - lo;
+  return true;
+}
+
+__device__ __forceinline__ int64_t slot_token(const FfnArgs& a, int64_t row, int64_t& slot) {
+  slot = a.tok_of[row];
+  if (slot < 0 || slot >= a.T * a.k) {
+    record_error(a.hdr, MOE_ERR_DEVICE_CHECK, (int)row);
+    return -1;
+  }
+  return slot / a.k;
+}
+
+__global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int n_act = min(max(*(volatile int*)&a.hdr->num_active, 0), a.E);
+  const int64_t routed_items = (int64_t)n_act * a.I;
+  const int64_t total = routed_items + (a.ws_gate_up != nullptr ? a.Is : 0);
+  const int H = a.H, nv = H / 8;
+
+  for (int64_t item = gw; item < total; item += nw) {
+    const bool shared = item >= routed_items;
+    int j;
+    const uint16_t *gate, *up;
+    int64_t r0 = 0, m = 0;
+    if (!shared) {
+      const int aidx = (int)(item / a.I);
+      j = (int)(item - (int64_t)aidx * a.I);
+      int e;
+      if (!expert_rows(a, aidx, e, r0, m)) continue;
+      gate = a.w_gate_up + ((int64_t)e * 2 * a.I + j) * H;
+      up = gate + (int64_t)a.I * H;
+    } else {
+      j = (int)(item - routed_items);
+      gate = a.ws_gate_up + (int64_t)j * H;
+      up = gate + (int64_t)a.Is * H;
+      m = a.T;
+    }
+    for (int64_t c0 = 0; c0 < m; c0 += kTok) {
+      const int mc = (int)min((int64_t)kTok, m - c0);
+      const uint16_t* xr[kTok];
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) {
+        xr[t] = nullptr;
+        if (t < mc) {
+          int64_t tok = c0 + t, slot;
+          if (!shared) tok = slot_token(a, r0 + c0 + t, slot);
+          if (tok >= 0) xr[t] = a.x + tok * H;
+        }
+      }
+      float ag[kTok], au[kTok];
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) ag[t] = au[t] = 0.0f;
+      for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+        uint4 gv[kUnroll], uv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nv) {
+            gv[u] = ld_stream_u4(gate + v * 8);
+            uv[u] = ld_stream_u4(up + v * 8);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nv) {
+#pragma unroll
+            for (int t = 0; t < kTok; ++t) {
+              if (t < mc && xr[t] != nullptr) {
+                float xf[8];
+                unpack8_bf16(ld_nc_u4(xr[t] + v * 8), xf);
+                ag[t] = dot8_bf16(gv[u], xf, ag[t]);
+                au[t] = dot8_bf16(uv[u], xf, au[t]);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) {
+        if (t < mc) {
+          const float g = warp_sum(ag[t]);
+          const float u = warp_sum(au[t]);
+          if (lane == t && xr[t] != nullptr) {
+            const uint16_t h = f32_to_bf16(silu_f32(g) * u);
+            if (!shared) a.h_perm[(r0 + c0 + t) * a.I + j] = h;
+            else a.h_shared[(c0 + t) * a.Is + j] = h;
+          }
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int n_act = min(max(*(volatile int*)&a.hdr->num_active, 0), a.E);
+  const int H = a.H;
+  const int nrb = (H + kDownRows - 1) / kDownRows;
+  const int64_t routed_items = (int64_t)n_act * nrb;
+  const int64_t total = routed_items + (a.ws_down != nullptr ? nrb : 0);
+
+  for (int64_t item = gw; item < total; item += nw) {
+    const bool shared = item >= routed_items;
+    int n0, K;
+    const uint16_t* w0;
+    const uint16_t* hin;
+    int64_t r0 = 0, m = 0;
+    if (!shared) {
+      const int aidx = (int)(item / nrb);
+      n0 = (int)(item - (int64_t)aidx * nrb) * kDownRows;
+      int e;
+      if (!expert_rows(a, aidx, e, r0, m)) continue;
+      K = a.I;
+      w0 = a.w_down + ((int64_t)e * H + n0) * K;
+      hin = a.h_perm;
+    } else {
+      n0 = (int)(item - routed_items) * kDownRows;
+      K = a.Is;
+      w0 = a.ws_down + (int64_t)n0 * K;
+      hin = a.h_shared;
+      m = a.T;
+    }
+    const int nvk = K / 8;
+    const int nrows = min(kDownRows, H - n0);
+    for (int64_t c0 = 0; c0 < m; c0 += kTok) {
+      const int mc = (int)min((int64_t)kTok, m - c0);
+      float acc[kDownRows][kTok];
+#pragma unroll
+      for (int r = 0; r < kDownRows; ++r)
+#pragma unroll
+        for (int t = 0; t < kTok; ++t) acc[r][t] = 0.0f;
+#pragma unroll 2
+      for (int v = lane; v < nvk; v += 32) {
+        uint4 wv[kDownRows];
+#pragma unroll
+        for (int r = 0; r < kDownRows; ++r)
+          if (r < nrows) wv[r] = ld_stream_u4(w0 + (int64_t)r * K + v * 8);
+#pragma unroll
+        for (int t = 0; t < kTok; ++t) {
+          if (t < mc) {
+            float hf[8];
+            unpack8_bf16(ld_nc_u4(hin + (r0 + c0 + t) * K + v * 8), hf);
+#pragma unroll
+            for (int r = 0; r < kDownRows; ++r)
+              if (r < nrows) acc[r][t] = dot8_bf16(wv[r], hf, acc[r][t]);
+          }
+        }
+      }
+      float mine = 0.0f;
+#pragma unroll
+      for (int r = 0; r < kDownRows; ++r)
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+          if (t < mc && r < nrows) {
+            const float s = warp_sum(acc[r][t]);
+            if (lane == r * kTok + t) mine = s;
+          }
+      const int r = lane / kTok, t = lane % kTok;
+      if (r < nrows && t < mc) {
+        if (!shared) {
+          int64_t slot;
+          if (slot_token(a, r0 + c0 + t, slot) >= 0) {
+            const float w = a.topk_w != nullptr ? a.topk_w[slot] : 1.0f;
+            a.y_slots[slot * H + n0 + r] = f32_to_bf16(w * mine);
+          }
+        } else {
+          a.shared_out[(c0 + t) * H + n0 + r] = f32_to_bf16(mine);
+        }
+      }
+    }
+  }
+}
+
+// y[t] = bf16( sum_j float(y_slots[t*k + j]) + float(shared_out[t]) ), in
+// slot order then the shared row; one thread per 8 outputs.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y_slots,
+                                                      const uint16_t* __restrict__ shared_out, int64_t T, int k,
+                                                      int H, uint16_t* __restrict__ y) {
+  const int nv = H / 8;
+  const int64_t n = T * nv;
+  const uint4* ys = reinterpret_cast<const uint4*>(y_slots);
+  const uint4* sh = reinterpret_cast<const uint4*>(shared_out);
+  uint4* out = reinterpret_cast<uint4*>(y);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nv;
+    const int v = (int)(i - t * nv);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      float f[8];
+      unpack8_bf16(__ldg(ys + (t * k + j) * nv + v), f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+    }
+    if (sh != nullptr) {
+      float f[8];
+      unpack8_bf16(__ldg(sh + i), f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    out[i] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s) {
+  const int blocks = sm_count() * 4;
+  before_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
+  gemv_gate_up_kernel<<<blocks, 256, 0, s>>>(a);
+  after_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  before_launch(MOE_KERNEL_EXPERT_DOWN, s);
+  gemv_down_kernel<<<blocks, 256, 0, s>>>(a);
+  after_launch(MOE_KERNEL_EXPERT_DOWN, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* y_slots, const uint16_t* shared_out, int64_t T, int k, int H,
+                           uint16_t* y, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t n = T * (H / 8);
+  int64_t blocks = (n + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  before_launch(MOE_KERNEL_COMBINE, s);
+  combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(y_slots, shared_out, T, k, H, y);
+  after_launch(MOE_KERNEL_COMBINE, s);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

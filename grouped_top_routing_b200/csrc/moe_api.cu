@@ -1,0 +1,466 @@
+// C ABI of libmoe.so: argument validation, workspace layout, launch sequence.
+//
+// Validation follows mlxcel issue #838, section "Defensive requirements":
+// magnitude ceilings on every architecture scalar, zero checks before any
+// divisibility check, 1 <= k <= E, E divisible by n_group, topk_group in
+// [1, n_group], reject rather than terminate. Every rule here runs on the host
+// before the first launch and returns a status with a message naming the field.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "ffn.cuh"
+
+namespace moe {
+
+cudaError_t launch_router_logits(const moe_config& c, const uint16_t* x, int64_t T, const float* w, float* out,
+                                 cudaStream_t s);
+cudaError_t launch_route(const moe_config& c, const float* logits, const float* bias, int64_t T, int32_t* idx,
+                         float* w, cudaStream_t s);
+size_t permute_scratch_ints(int E, int64_t T);
+cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, const uint16_t* x, int32_t* offsets,
+                           int32_t* row_of, int32_t* tok_of, uint16_t* x_perm, int32_t* active, int32_t* tile_cnt,
+                           int32_t* tile_base, WsHeader* hdr, cudaStream_t s);
+cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, WsHeader* hdr,
+                                       cudaStream_t s);
+cudaError_t launch_combine(const uint16_t* y_slots, const uint16_t* shared_out, int64_t T, int k, int H,
+                           uint16_t* y, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// errors, hooks, device cache
+// ---------------------------------------------------------------------------
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<uint64_t> g_launches{0};
+void* g_ev_start[MOE_KERNEL_COUNT] = {};
+void* g_ev_stop[MOE_KERNEL_COUNT] = {};
+int g_sm_count[64] = {};
+
+moe_status fail(moe_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+void before_launch(int id, cudaStream_t s) {
+  if (id >= 0 && id < MOE_KERNEL_COUNT && g_ev_start[id] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_ev_start[id]), s);
+}
+
+void after_launch(int id, cudaStream_t s, int nkernels) {
+  g_launches.fetch_add((uint64_t)nkernels, std::memory_order_relaxed);
+  if (id >= 0 && id < MOE_KERNEL_COUNT && g_ev_stop[id] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_ev_stop[id]), s);
+}
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int32_t kMaxHidden = 32768;
+constexpr int32_t kMaxExperts = 1024;
+constexpr int32_t kMaxGroups = 32;
+constexpr int32_t kMaxIntermediate = 32768;
+constexpr int32_t kMaxShared = 64;
+constexpr int64_t kMaxTokens = int64_t(1) << 22;
+
+int32_t shared_width(const moe_config& c) {
+  if (c.num_shared_experts <= 0) return 0;
+  const int32_t per = c.moe_shared_expert_intermediate_size > 0 ? c.moe_shared_expert_intermediate_size
+                                                                : c.moe_intermediate_size;
+  return per * c.num_shared_experts;
+}
+
+moe_status check_range(const char* name, int64_t v, int64_t lo, int64_t hi) {
+  if (v < lo || v > hi) return fail(MOE_ERR_INVALID_ARG, "%s = %lld outside [%lld, %lld]", name, (long long)v,
+                                    (long long)lo, (long long)hi);
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)              \
+  do {                             \
+    moe_status _st = (expr);       \
+    if (_st != MOE_OK) return _st; \
+  } while (0)
+
+moe_status validate_config(const moe_config* c) {
+  if (c == nullptr) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  MOE_TRY(check_range("hidden_size", c->hidden_size, 1, kMaxHidden));
+  MOE_TRY(check_range("num_experts", c->num_experts, 1, kMaxExperts));
+  MOE_TRY(check_range("num_experts_per_tok", c->num_experts_per_tok, 1, c->num_experts));
+  MOE_TRY(check_range("n_group", c->n_group, 1, kMaxGroups));
+  MOE_TRY(check_range("topk_group", c->topk_group, 1, c->n_group));  // zero rejected before any division
+  if (c->n_group > 1) {
+    if (c->num_experts % c->n_group != 0)
+      return fail(MOE_ERR_INVALID_ARG, "num_experts = %d not divisible by n_group = %d", c->num_experts, c->n_group);
+    const int gsz = c->num_experts / c->n_group;
+    if ((int64_t)c->topk_group * gsz < c->num_experts_per_tok)
+      return fail(MOE_ERR_INVALID_ARG, "topk_group * (num_experts / n_group) = %d < num_experts_per_tok = %d",
+                  c->topk_group * gsz, c->num_experts_per_tok);
+  }
+  if (c->score_function != MOE_SCORE_SOFTMAX && c->score_function != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "score_function = %d is neither softmax (0) nor sigmoid (1)", c->score_function);
+  MOE_TRY(check_range("norm_topk_prob", c->norm_topk_prob, 0, 1));
+  if (!std::isfinite(c->routed_scaling_factor))
+    return fail(MOE_ERR_INVALID_ARG, "routed_scaling_factor is not finite");
+  MOE_TRY(check_range("moe_intermediate_size", c->moe_intermediate_size, 1, kMaxIntermediate));
+  MOE_TRY(check_range("num_shared_experts", c->num_shared_experts, 0, kMaxShared));
+  MOE_TRY(check_range("moe_shared_expert_intermediate_size", c->moe_shared_expert_intermediate_size, 0,
+                      kMaxIntermediate));
+  if (c->hidden_size % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden_size = %d is not a multiple of 8 (16-byte rows)", c->hidden_size);
+  if (c->moe_intermediate_size % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_intermediate_size = %d is not a multiple of 8 (16-byte rows)",
+                c->moe_intermediate_size);
+  if (c->moe_shared_expert_intermediate_size % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_shared_expert_intermediate_size = %d is not a multiple of 8",
+                c->moe_shared_expert_intermediate_size);
+  if (shared_width(*c) > kMaxIntermediate * 4)
+    return fail(MOE_ERR_UNSUPPORTED, "shared MLP width %d exceeds %d", shared_width(*c), kMaxIntermediate * 4);
+  return MOE_OK;
+}
+
+moe_status check_tokens(const moe_config& c, int64_t T) {
+  if (T < 0 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T = %lld outside [0, %lld]", (long long)T,
+                                           (long long)kMaxTokens);
+  if (T * c.num_experts_per_tok > INT32_MAX)
+    return fail(MOE_ERR_UNSUPPORTED, "T * num_experts_per_tok = %lld exceeds int32 row indices",
+                (long long)(T * c.num_experts_per_tok));
+  return MOE_OK;
+}
+
+moe_status check_ptr(const char* name, const void* p, size_t align, bool required) {
+  if (p == nullptr) {
+    if (required) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+    return MOE_OK;
+  }
+  if (reinterpret_cast<uintptr_t>(p) % align != 0)
+    return fail(MOE_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layout
+// ---------------------------------------------------------------------------
+struct Layout {
+  size_t hdr, logits, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
+  size_t x_perm, h_perm, h_shared, y_slots, shared_out, total;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+Layout layout(const moe_config& c, int64_t max_tokens) {
+  const int64_t T = max_tokens > 0 ? max_tokens : 1;
+  const int64_t E = c.num_experts, k = c.num_experts_per_tok, H = c.hidden_size, I = c.moe_intermediate_size;
+  const int64_t Is = shared_width(c);
+  const int64_t R = T * k;
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.hdr = take(sizeof(WsHeader));
+  L.logits = take((size_t)T * E * 4);
+  L.topk_idx = take((size_t)R * 4);
+  L.topk_w = take((size_t)R * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.row_of = take((size_t)R * 4);
+  L.tok_of = take((size_t)R * 4);
+  L.active = take((size_t)E * 4);
+  L.tile_cnt = take(permute_scratch_ints((int)E, T) * 4);
+  L.tile_base = take(permute_scratch_ints((int)E, T) * 4);
+  L.x_perm = take((size_t)R * H * 2);
+  L.h_perm = take((size_t)R * I * 2);
+  L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 2);
+  L.y_slots = take((size_t)R * H * 2);
+  L.shared_out = take((size_t)T * H * 2);
+  L.total = off;
+  return L;
+}
+
+template <class P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+moe_status check_ws(const moe_config& c, int64_t T, void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  const size_t need = layout(c, T).total;
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed for T = %lld", ws_bytes, need, (long long)T);
+  return MOE_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint16_t* x_perm,
+                   const int32_t* offsets, const int32_t* tok_of, const float* topk_w, const uint16_t* wgu,
+                   const uint16_t* wd, const uint16_t* swgu, const uint16_t* swd, uint16_t* y_slots,
+                   uint16_t* shared_out, void* ws, bool active_ready, cudaStream_t s) {
+  const Layout L = layout(c, T);
+  WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  int32_t* active = at<int32_t>(ws, L.active);
+  cudaError_t e;
+  if (!active_ready) {
+    e = launch_active_from_offsets(offsets, c.num_experts, active, hdr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "active list");
+  }
+  FfnArgs a{};
+  a.x = x;
+  a.T = T;
+  a.H = c.hidden_size;
+  a.I = c.moe_intermediate_size;
+  a.Is = shared_width(c);
+  a.k = c.num_experts_per_tok;
+  a.E = c.num_experts;
+  a.offsets = offsets;
+  a.tok_of = tok_of;
+  a.active = active;
+  a.hdr = hdr;
+  a.topk_w = topk_w;
+  a.w_gate_up = wgu;
+  a.w_down = wd;
+  a.ws_gate_up = (swgu != nullptr && a.Is > 0) ? swgu : nullptr;
+  a.ws_down = a.ws_gate_up != nullptr ? swd : nullptr;
+  a.h_perm = at<uint16_t>(ws, L.h_perm);
+  a.h_shared = at<uint16_t>(ws, L.h_shared);
+  a.y_slots = y_slots;
+  a.shared_out = shared_out;
+  (void)x_perm;
+  e = launch_gemv_ffn(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "expert ffn");
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+// ---------------------------------------------------------------------------
+// extern "C" entry points
+// ---------------------------------------------------------------------------
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg, int64_t max_tokens) {
+  if (validate_config(cfg) != MOE_OK) return 0;
+  if (check_tokens(*cfg, max_tokens) != MOE_OK) return 0;
+  g_err[0] = '\0';
+  return layout(*cfg, max_tokens).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "workspace init");
+  return MOE_OK;
+}
+
+moe_status moe_router_logits(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
+                             float* logits, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr("x", x, 16, true));
+  MOE_TRY(check_ptr("router_w", router_w, 16, true));
+  MOE_TRY(check_ptr("logits", logits, 4, true));
+  cudaError_t e = launch_router_logits(*cfg, x, T, router_w, logits, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "router logits");
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const float* logits, const float* expert_bias, int64_t T,
+                     int32_t* topk_idx, float* topk_w, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr("logits", logits, 4, true));
+  MOE_TRY(check_ptr("expert_bias", expert_bias, 4, false));
+  MOE_TRY(check_ptr("topk_idx", topk_idx, 4, true));
+  MOE_TRY(check_ptr("topk_w", topk_w, 4, true));
+  cudaError_t e = launch_route(*cfg, logits, expert_bias, T, topk_idx, topk_w, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "route");
+  return MOE_OK;
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T, const uint16_t* x,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* tok_of, uint16_t* x_perm, void* ws,
+                       size_t ws_bytes, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  MOE_TRY(check_ptr("expert_offsets", expert_offsets, 4, true));
+  if (T > 0) {
+    MOE_TRY(check_ptr("topk_idx", topk_idx, 4, true));
+    MOE_TRY(check_ptr("row_of", row_of, 4, true));
+    MOE_TRY(check_ptr("tok_of", tok_of, 4, true));
+    MOE_TRY(check_ptr("x_perm", x_perm, 16, false));
+    MOE_TRY(check_ptr("x", x, 16, x_perm != nullptr));
+  }
+  const Layout L = layout(*cfg, T);
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(expert_offsets, 0, (size_t)(cfg->num_experts + 1) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "permute");
+    return MOE_OK;
+  }
+  cudaError_t e = launch_permute(*cfg, topk_idx, T, x, expert_offsets, row_of, tok_of, x_perm,
+                                 at<int32_t>(ws, L.active), at<int32_t>(ws, L.tile_cnt), at<int32_t>(ws, L.tile_base),
+                                 at<WsHeader>(ws, L.hdr), s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute");
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, const uint16_t* x_perm,
+                          const int32_t* expert_offsets, const int32_t* tok_of, const float* topk_w,
+                          const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* ws_gate_up,
+                          const uint16_t* ws_down, uint16_t* y_slots, uint16_t* shared_out, void* ws,
+                          size_t ws_bytes, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const bool has_shared = shared_width(*cfg) > 0;
+  MOE_TRY(check_ptr("x", x, 16, true));
+  MOE_TRY(check_ptr("x_perm", x_perm, 16, false));
+  MOE_TRY(check_ptr("expert_offsets", expert_offsets, 4, true));
+  MOE_TRY(check_ptr("tok_of", tok_of, 4, true));
+  MOE_TRY(check_ptr("topk_w", topk_w, 4, false));
+  MOE_TRY(check_ptr("w_gate_up", w_gate_up, 16, true));
+  MOE_TRY(check_ptr("w_down", w_down, 16, true));
+  MOE_TRY(check_ptr("y_slots", y_slots, 16, true));
+  MOE_TRY(check_ptr("ws_gate_up", ws_gate_up, 16, false));
+  MOE_TRY(check_ptr("ws_down", ws_down, 16, ws_gate_up != nullptr));
+  MOE_TRY(check_ptr("shared_out", shared_out, 16, ws_gate_up != nullptr));
+  if (ws_gate_up != nullptr && !has_shared)
+    return fail(MOE_ERR_INVALID_ARG, "ws_gate_up given but the config has no shared MLP");
+  if (ws_gate_up == nullptr) shared_out = nullptr;
+  return run_ffn(*cfg, T, x, x_perm, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws_gate_up, ws_down, y_slots,
+                 shared_out, ws, false, as_stream(stream));
+}
+
+moe_status moe_combine(const moe_config* cfg, int64_t T, const uint16_t* y_slots, const uint16_t* shared_out,
+                       uint16_t* y, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr("y_slots", y_slots, 16, true));
+  MOE_TRY(check_ptr("shared_out", shared_out, 16, false));
+  MOE_TRY(check_ptr("y", y, 16, true));
+  cudaError_t e =
+      launch_combine(y_slots, shared_out, T, cfg->num_experts_per_tok, cfg->hidden_size, y, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
+                       const float* expert_bias, const float* logits_override, const uint16_t* w_gate_up,
+                       const uint16_t* w_down, const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y,
+                       int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const moe_config& c = *cfg;
+  const bool has_shared = shared_width(c) > 0;
+  MOE_TRY(check_ptr("x", x, 16, true));
+  MOE_TRY(check_ptr("logits_override", logits_override, 4, false));
+  MOE_TRY(check_ptr("router_w", router_w, 16, logits_override == nullptr));
+  MOE_TRY(check_ptr("expert_bias", expert_bias, 4, false));
+  MOE_TRY(check_ptr("w_gate_up", w_gate_up, 16, true));
+  MOE_TRY(check_ptr("w_down", w_down, 16, true));
+  MOE_TRY(check_ptr("ws_gate_up", ws_gate_up, 16, has_shared));
+  MOE_TRY(check_ptr("ws_down", ws_down, 16, has_shared));
+  MOE_TRY(check_ptr("y", y, 16, true));
+  MOE_TRY(check_ptr("topk_idx_out", topk_idx_out, 4, false));
+  MOE_TRY(check_ptr("topk_w_out", topk_w_out, 4, false));
+  if (!has_shared && ws_gate_up != nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "ws_gate_up given but the config has no shared MLP");
+
+  const Layout L = layout(c, T);
+  cudaStream_t s = as_stream(stream);
+  WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  const float* logits = logits_override;
+  cudaError_t e;
+  if (logits == nullptr) {
+    float* lg = at<float>(ws, L.logits);
+    e = launch_router_logits(c, x, T, router_w, lg, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router logits");
+    logits = lg;
+  }
+  int32_t* idx = topk_idx_out != nullptr ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+  float* w = topk_w_out != nullptr ? topk_w_out : at<float>(ws, L.topk_w);
+  e = launch_route(c, logits, expert_bias, T, idx, w, s);
+  if (e != cudaSuccess) return cuda_fail(e, "route");
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* tok_of = at<int32_t>(ws, L.tok_of);
+  e = launch_permute(c, idx, T, x, offsets, at<int32_t>(ws, L.row_of), tok_of, nullptr, at<int32_t>(ws, L.active),
+                     at<int32_t>(ws, L.tile_cnt), at<int32_t>(ws, L.tile_base), hdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute");
+  uint16_t* y_slots = at<uint16_t>(ws, L.y_slots);
+  uint16_t* shared_out = has_shared ? at<uint16_t>(ws, L.shared_out) : nullptr;
+  MOE_TRY(run_ffn(c, T, x, nullptr, offsets, tok_of, w, w_gate_up, w_down, has_shared ? ws_gate_up : nullptr,
+                  has_shared ? ws_down : nullptr, y_slots, shared_out, ws, true, s));
+  e = launch_combine(y_slots, shared_out, T, c.num_experts_per_tok, c.hidden_size, y, s);
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
+  return MOE_OK;
+}
+
+moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
+  int32_t word[2] = {0, 0};
+  e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (word[0] == 0) return MOE_OK;
+  e = cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (word[0] == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "device wait timed out (site %d)", word[1]);
+  return fail(MOE_ERR_DEVICE_CHECK, "device index check failed (index %d)", word[1]);
+}
+
+moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop) {
+  if (which < 0 || which >= MOE_KERNEL_COUNT) return fail(MOE_ERR_INVALID_ARG, "which = %d is not a kernel id", which);
+  if ((ev_start == nullptr) != (ev_stop == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "ev_start and ev_stop must both be set or both be NULL");
+  g_ev_start[which] = ev_start;
+  g_ev_stop[which] = ev_stop;
+  return MOE_OK;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* moe_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,234 @@
+"""ctypes binding of libmoe.so (declared in include/moe.h).
+
+Argument marshalling only: every step of the block runs in the library's CUDA
+kernels. torch supplies device memory and the current stream. Importing this
+module raises if libmoe.so is missing; there is no other implementation to
+fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
+SCORE = {"softmax": 0, "sigmoid": 1}
+KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "expert_down": 4, "combine": 5}
+
+# Every entry point include/moe.h declares.
+EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
+           "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
+           "moe_launch_count", "moe_last_error")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [
+        ("hidden_size", ctypes.c_int32),
+        ("num_experts", ctypes.c_int32),
+        ("num_experts_per_tok", ctypes.c_int32),
+        ("n_group", ctypes.c_int32),
+        ("topk_group", ctypes.c_int32),
+        ("score_function", ctypes.c_int32),
+        ("norm_topk_prob", ctypes.c_int32),
+        ("routed_scaling_factor", ctypes.c_float),
+        ("moe_intermediate_size", ctypes.c_int32),
+        ("num_shared_experts", ctypes.c_int32),
+        ("moe_shared_expert_intermediate_size", ctypes.c_int32),
+    ]
+
+
+def config_from_workload(wl: dict) -> MoeConfig:
+    sf = wl["score_function"]
+    return MoeConfig(
+        hidden_size=wl["hidden_size"], num_experts=wl["num_experts"],
+        num_experts_per_tok=wl["num_experts_per_tok"], n_group=wl.get("n_group", 1),
+        topk_group=wl.get("topk_group", 1), score_function=SCORE[sf] if isinstance(sf, str) else int(sf),
+        norm_topk_prob=int(bool(wl["norm_topk_prob"])), routed_scaling_factor=float(wl["routed_scaling_factor"]),
+        moe_intermediate_size=wl["moe_intermediate_size"], num_shared_experts=wl.get("num_shared_experts", 0),
+        moe_shared_expert_intermediate_size=wl.get("moe_shared_expert_intermediate_size", 0),
+    )
+
+
+def _load():
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is not built; run `python -m grouped_top_routing_b200.build`")
+    L = ctypes.CDLL(library_path)
+    vp, i64, sz, cfgp = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.POINTER(MoeConfig)
+    st = ctypes.c_int
+    sig = {
+        "moe_workspace_size": (sz, [cfgp, i64]),
+        "moe_workspace_init": (st, [vp, sz, vp]),
+        "moe_router_logits": (st, [cfgp, vp, i64, vp, vp, vp]),
+        "moe_route": (st, [cfgp, vp, vp, i64, vp, vp, vp]),
+        "moe_permute": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_expert_ffn": (st, [cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_combine": (st, [cfgp, i64, vp, vp, vp, vp]),
+        "moe_forward": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_check_device": (st, [vp, sz, vp]),
+        "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
+        "moe_launch_count": (ctypes.c_uint64, []),
+        "moe_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def last_error() -> str:
+    return lib.moe_last_error().decode()
+
+
+def _check(status: int):
+    if status != MOE_OK:
+        raise MoeError(status, last_error())
+
+
+def _p(t):
+    """Device (or host) address of a tensor, or None."""
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cfg(cfg):
+    return ctypes.byref(cfg if isinstance(cfg, MoeConfig) else config_from_workload(cfg))
+
+
+def _as_cfg(cfg):
+    return cfg if isinstance(cfg, MoeConfig) else config_from_workload(cfg)
+
+
+def moe_workspace_size(cfg, max_tokens: int) -> int:
+    n = lib.moe_workspace_size(_cfg(cfg), int(max_tokens))
+    if n == 0:
+        raise MoeError(1, last_error())
+    return n
+
+
+class Workspace:
+    """A device workspace sized by moe_workspace_size, header zeroed."""
+
+    def __init__(self, cfg, max_tokens: int, device="cuda"):
+        self.nbytes = moe_workspace_size(cfg, max_tokens)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.ptr = (base + 255) & ~255
+        _check(lib.moe_workspace_init(ctypes.c_void_p(self.ptr), self.nbytes, _stream()))
+
+    @property
+    def cptr(self):
+        return ctypes.c_void_p(self.ptr)
+
+    def check(self, stream=None):
+        """Synchronise and raise if a device-side check or wait failed."""
+        _check(lib.moe_check_device(self.cptr, self.nbytes, _stream(stream)))
+
+
+def moe_router_logits(cfg, x, router_w, out=None, stream=None):
+    c = _as_cfg(cfg)
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, c.num_experts), dtype=torch.float32, device=x.device)
+    _check(lib.moe_router_logits(ctypes.byref(c), _p(x), T, _p(router_w), _p(out), _stream(stream)))
+    return out
+
+
+def moe_route(cfg, logits, expert_bias=None, topk_idx=None, topk_w=None, stream=None):
+    c = _as_cfg(cfg)
+    T = logits.shape[0]
+    k = c.num_experts_per_tok
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check(lib.moe_route(ctypes.byref(c), _p(logits), _p(expert_bias), T, _p(topk_idx), _p(topk_w), _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_permute(cfg, topk_idx, ws: Workspace, x=None, want_x_perm=False, stream=None):
+    c = _as_cfg(cfg)
+    T = topk_idx.shape[0]
+    k, E, H = c.num_experts_per_tok, c.num_experts, c.hidden_size
+    dev = topk_idx.device
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tok_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev) if want_x_perm else None
+    _check(lib.moe_permute(ctypes.byref(c), _p(topk_idx), T, _p(x), _p(offsets), _p(row_of), _p(tok_of), _p(x_perm),
+                           ws.cptr, ws.nbytes, _stream(stream)))
+    return offsets, row_of, tok_of, x_perm
+
+
+def moe_expert_ffn(cfg, x, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws: Workspace, ws_gate_up=None,
+                   ws_down=None, x_perm=None, y_slots=None, shared_out=None, stream=None):
+    c = _as_cfg(cfg)
+    T = x.shape[0]
+    k, H = c.num_experts_per_tok, c.hidden_size
+    if y_slots is None:
+        y_slots = torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
+    if ws_gate_up is not None and shared_out is None:
+        shared_out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib.moe_expert_ffn(ctypes.byref(c), T, _p(x), _p(x_perm), _p(expert_offsets), _p(tok_of), _p(topk_w),
+                              _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y_slots), _p(shared_out),
+                              ws.cptr, ws.nbytes, _stream(stream)))
+    return y_slots, shared_out
+
+
+def moe_combine(cfg, y_slots, shared_out, T: int, y=None, stream=None):
+    c = _as_cfg(cfg)
+    if y is None:
+        y = torch.empty((T, c.hidden_size), dtype=torch.bfloat16, device=y_slots.device)
+    _check(lib.moe_combine(ctypes.byref(c), T, _p(y_slots), _p(shared_out), _p(y), _stream(stream)))
+    return y
+
+
+def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws_down, ws: Workspace,
+                logits_override=None, y=None, return_routing=False, stream=None):
+    c = _as_cfg(cfg)
+    T = x.shape[0]
+    k = c.num_experts_per_tok
+    if y is None:
+        y = torch.empty_like(x)
+    idx = w = None
+    if return_routing:
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib.moe_forward(ctypes.byref(c), _p(x), T, _p(router_w), _p(expert_bias), _p(logits_override),
+                           _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y), _p(idx), _p(w),
+                           ws.cptr, ws.nbytes, _stream(stream)))
+    if return_routing:
+        return y, idx, w
+    return y
+
+
+def set_kernel_timer(kernel: str, ev_start=None, ev_stop=None):
+    a = ctypes.c_void_p(ev_start.cuda_event) if ev_start is not None else None
+    b = ctypes.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
+    _check(lib.moe_set_kernel_timer(KERNELS[kernel], a, b))
+
+
+def launch_count() -> int:
+    return int(lib.moe_launch_count())

@@ -1,0 +1,211 @@
+/*
+ * moe.h -- C ABI of libmoe.so, the B200 (sm_100a) grouped top-k MoE block.
+ *
+ * The block is the Bailing/Ling mixture-of-experts feed-forward layer:
+ *   router (softmax or sigmoid scores, selection-only expert bias, optional
+ *   grouped top-k, renormalisation, routed scaling) -> token-to-expert
+ *   permutation -> SwiGLU routed experts + one always-on shared MLP ->
+ *   weighted combine.
+ *
+ * Sources (page title, section):
+ *   [ROUTER]  mlxcel issue #838 "add Ant Group Ling / Bailing MoE (bailing_moe)",
+ *             section "Router: selection uses biased scores, weights come from
+ *             unbiased scores".
+ *   [SCALE]   same issue, "moe_router_enable_routed_scaling is dead code
+ *             upstream" (the scaling factor is applied unconditionally).
+ *   [SHARED]  same issue, "Shared experts are one wide MLP, not N separate
+ *             experts".
+ *   [FIELDS]  same issue, "Config fields the checkpoint does not contain".
+ *   [ARCH]    same issue, "Architecture notes".
+ *   [DEFENSE] same issue, "Defensive requirements" (validate before use, reject
+ *             instead of terminating, take gather bounds from real shapes).
+ *   [LING26]  model card "Ling-2.6-flash-JANGTQ", "Architecture
+ *             (bailing_hybrid)", paragraph "MoE routing".
+ *   [GGUF]    page "Ling-3.0-flash-GGUF", "Measured performance": decode reads
+ *             only the selected experts' weights.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated otherwise. bf16 tensors are
+ *     passed as uint16_t (raw bf16 bits), row-major, densely packed.
+ *   - Every matrix and vector pointer must be 16-byte aligned (vector and TMA
+ *     loads); the workspace 256-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream). They return once the work is enqueued.
+ *   - The caller owns every buffer. The library allocates no device memory and
+ *     keeps no state beyond a per-device attribute cache, per-thread error text
+ *     and the measurement hooks of moe_set_kernel_timer.
+ *   - All arguments are validated on the host BEFORE any launch. A rejected call
+ *     launches nothing and returns a status; the library never aborts or throws
+ *     across this ABI ([DEFENSE]). moe_last_error() names the offending field.
+ *   - Index-driven reads on the device are bounds-checked against the sizes
+ *     passed in; an out-of-range id is skipped and recorded in the workspace
+ *     error word, which moe_check_device() reports as MOE_ERR_DEVICE_CHECK.
+ *   - Device-side waits are bounded; a wait that runs out records
+ *     MOE_ERR_TIMEOUT in the same word and the kernel returns.
+ *
+ * Shapes (T tokens, H hidden_size, E num_experts, k num_experts_per_tok,
+ * I moe_intermediate_size, Is the shared MLP width):
+ *   x          [T, H]      bf16
+ *   router_w   [E, H]      fp32          (router projection, mlp.gate)
+ *   expert_bias[E]         fp32 or NULL  (e_score_correction_bias)
+ *   w_gate_up  [E, 2I, H]  bf16          rows [0,I) gate_proj, rows [I,2I) up_proj
+ *   w_down     [E, H, I]   bf16          down_proj
+ *   ws_gate_up [2Is, H]    bf16          shared MLP, same row split
+ *   ws_down    [H, Is]     bf16
+ *   Is = (moe_shared_expert_intermediate_size ? that : I) * num_shared_experts
+ *   ([SHARED]: one wide MLP, added at weight 1.0, never routed).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* a config field, size or pointer is invalid */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid for the method, outside this build's limits */
+  MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_CHECK = 5, /* a device-side index check failed (see moe_check_device) */
+  MOE_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_function;
+
+/* Block configuration. Field names follow the Bailing config ([FIELDS]). */
+typedef struct {
+  int32_t hidden_size;          /* H: multiple of 8, <= 32768 */
+  int32_t num_experts;          /* E: 1..1024 */
+  int32_t num_experts_per_tok;  /* k: 1..E */
+  int32_t n_group;              /* >= 1; E % n_group == 0 when > 1; <= 32 */
+  int32_t topk_group;           /* 1..n_group; == n_group keeps every group */
+  int32_t score_function;       /* moe_score_function; anything else is rejected ([FIELDS]) */
+  int32_t norm_topk_prob;       /* 0/1: renormalise, only when k > 1, eps 1e-20 ([ROUTER]) */
+  float routed_scaling_factor;  /* finite; always applied ([SCALE]) */
+  int32_t moe_intermediate_size;               /* I: multiple of 8, <= 32768 */
+  int32_t num_shared_experts;                  /* 0..64; 0 = no shared MLP */
+  int32_t moe_shared_expert_intermediate_size; /* 0 = use I ([SHARED]) */
+} moe_config;
+
+/* Kernels that moe_set_kernel_timer can bracket. */
+typedef enum {
+  MOE_KERNEL_ROUTER_LOGITS = 0,
+  MOE_KERNEL_ROUTE = 1,
+  MOE_KERNEL_PERMUTE = 2,
+  MOE_KERNEL_EXPERT_GATE_UP = 3, /* routed + shared gate/up projections with SwiGLU */
+  MOE_KERNEL_EXPERT_DOWN = 4,    /* routed + shared down projections, weighted */
+  MOE_KERNEL_COMBINE = 5,
+  MOE_KERNEL_COUNT = 6
+} moe_kernel_id;
+
+/* Workspace bytes moe_permute, moe_expert_ffn and moe_forward need for up to
+ * max_tokens tokens. Returns 0 (and sets moe_last_error) on an invalid config.
+ * The workspace holds the device error word, routing and permutation scratch
+ * and the intermediate activations. Only its header must be zeroed, once, by
+ * moe_workspace_init; the rest needs no initialisation. */
+size_t moe_workspace_size(const moe_config* cfg, int64_t max_tokens);
+
+/* Zeroes the workspace's 256-byte header (its device error word). Call once
+ * after allocating a workspace and before its first use; moe_check_device
+ * clears the word again after reporting. Asynchronous on `stream`. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Router projection ([ROUTER]; router weight mlp.gate [E, H]):
+ *   logits[t, e] = sum_h float(x[t, h]) * router_w[e, h]   (fp32 accumulate)
+ * x [T,H] bf16, router_w [E,H] fp32, logits [T,E] fp32 out. T may be 0. */
+moe_status moe_router_logits(const moe_config* cfg, const uint16_t* x, int64_t T,
+                             const float* router_w, float* logits, void* stream);
+
+/* Router on fp32 gates ([ROUTER], [ARCH], [LING26]). Per token:
+ *   s    = softmax(logits) or sigmoid(logits), each score the fp32 rounding of
+ *          the value evaluated in fp64;
+ *   sel  = s + expert_bias (fp32; selection only; skipped when bias is NULL);
+ *   if n_group > 1 and topk_group < n_group: group score = top-1 + top-2 of sel
+ *          in each contiguous group of E/n_group experts; keep the topk_group
+ *          best groups (ties: lower group id), sel = -inf elsewhere;
+ *   topk_idx[t, 0..k) = the k largest sel, ordered (sel desc, id asc);
+ *   w_j  = s[idx_j] (UNBIASED); if norm_topk_prob and k > 1:
+ *          w_j /= (((w_0 + w_1) + ...) + 1e-20f); then w_j *= routed_scaling_factor.
+ * logits [T,E] fp32; expert_bias [E] fp32 or NULL; topk_idx [T,k] int32 out;
+ * topk_w [T,k] fp32 out. Indices are always valid and distinct, even for
+ * non-finite logits (whose selection is then unspecified). */
+moe_status moe_route(const moe_config* cfg, const float* logits, const float* expert_bias, int64_t T,
+                     int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Token-to-expert permutation (histogram -> exclusive scan -> stable scatter).
+ * The T*k assignments are ordered by (expert, token):
+ *   expert_offsets [E+1] int32 out: rows of expert e are [off[e], off[e+1]);
+ *   row_of [T*k] int32 out: permuted row of assignment (t, j), index t*k + j;
+ *   tok_of [T*k] int32 out: the slot t*k + j that permuted row r holds;
+ *   x_perm [T*k, H] bf16 out (optional): x_perm[r] = x[tok_of[r] / k];
+ *   x may be NULL when x_perm is NULL.
+ * topk_idx entries outside [0, E) or repeated within a token are skipped and
+ * recorded as MOE_ERR_DEVICE_CHECK in the workspace error word. */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T, const uint16_t* x,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* tok_of, uint16_t* x_perm,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Routed SwiGLU experts and the shared MLP ([ARCH], [SHARED], [GGUF]):
+ *   F_e(v) = down_e( silu(gate_e v) * up_e v ),   silu(z) = z / (1 + exp(-z)),
+ * fp32 accumulation, the SwiGLU product rounded to bf16 before the down
+ * projection. Only experts with rows in expert_offsets are read.
+ *   y_slots[t*k + j] = bf16( topk_w[t*k + j] * F_{e}(x_t) )  for the expert e
+ *                      holding that slot (topk_w NULL: weight 1);
+ *   shared_out[t]    = bf16( F_shared(x_t) )  (when ws_gate_up is not NULL).
+ * x [T,H]; x_perm [T*k,H] from moe_permute, or NULL (rows are then gathered
+ * from x through tok_of); expert_offsets [E+1], tok_of [T*k] from moe_permute;
+ * y_slots [T*k,H] bf16 out; shared_out [T,H] bf16 out or NULL. */
+moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, const uint16_t* x_perm,
+                          const int32_t* expert_offsets, const int32_t* tok_of, const float* topk_w,
+                          const uint16_t* w_gate_up, const uint16_t* w_down,
+                          const uint16_t* ws_gate_up, const uint16_t* ws_down,
+                          uint16_t* y_slots, uint16_t* shared_out,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Weighted combine ([ROUTER], [SHARED]: out = routed mixture + shared(x)):
+ *   y[t] = bf16( sum_{j<k} float(y_slots[t*k + j]) + float(shared_out[t]) ),
+ * summed in fp32 in slot order then the shared row: deterministic.
+ * y_slots [T*k,H] bf16 (already weighted); shared_out [T,H] bf16 or NULL;
+ * y [T,H] bf16 out. */
+moe_status moe_combine(const moe_config* cfg, int64_t T, const uint16_t* y_slots, const uint16_t* shared_out,
+                       uint16_t* y, void* stream);
+
+/* The whole block: router logits -> route -> permute -> experts -> combine.
+ *   logits_override [T,E] fp32 or NULL: when given, replaces the router
+ *   projection (router_w may then be NULL).
+ *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
+ *   routing. y [T,H] bf16 out. ws / ws_bytes >= moe_workspace_size(cfg, T). */
+moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
+                       const float* expert_bias, const float* logits_override,
+                       const uint16_t* w_gate_up, const uint16_t* w_down,
+                       const uint16_t* ws_gate_up, const uint16_t* ws_down,
+                       uint16_t* y, int32_t* topk_idx_out, float* topk_w_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the workspace error word. Returns
+ * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT (first error recorded), or
+ * MOE_ERR_CUDA if the stream itself reports an error. Blocking. */
+moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
+
+/* Measurement aid. While set, every launch of kernel `which` is bracketed by
+ * cudaEventRecord(ev_start) / cudaEventRecord(ev_stop) on its launch stream
+ * (events are cudaEvent_t passed as void*; the caller owns them). Passing NULL
+ * events clears the hook. Not thread-safe with concurrent launches. */
+moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop);
+
+/* Number of this library's kernel launches since load (host-side counter). */
+uint64_t moe_launch_count(void);
+
+/* Per-thread text of the last rejected call ("" when none). Never NULL. */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

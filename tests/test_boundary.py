@@ -1,0 +1,188 @@
+"""The C-ABI boundary on the host: the library loads, exports every symbol
+include/moe.h declares, and rejects each invalid argument with a status
+before any launch (mlxcel issue #838, section "Defensive requirements": one
+rejection test per validation rule). No call here reaches the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_top_routing_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    B.build()
+    from grouped_top_routing_b200 import moe
+    return moe
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points(M):
+    names = _declared()
+    assert set(names) == set(M.EXPORTS), names
+    for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(M):
+    lib = ctypes.CDLL(M.library_path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def _good(**over):
+    c = dict(hidden_size=4096, num_experts=256, num_experts_per_tok=8, n_group=8, topk_group=4,
+             score_function=1, norm_topk_prob=1, routed_scaling_factor=2.5, moe_intermediate_size=1024,
+             num_shared_experts=1, moe_shared_expert_intermediate_size=0)
+    c.update(over)
+    return c
+
+
+def _cfg(M, **over):
+    return M.MoeConfig(**_good(**over))
+
+
+BAD_CONFIGS = [
+    ("hidden_size", dict(hidden_size=0), 1),
+    ("hidden_size", dict(hidden_size=-8), 1),
+    ("hidden_size", dict(hidden_size=1 << 20), 1),
+    ("hidden_size", dict(hidden_size=4100), 2),          # not a multiple of 8
+    ("num_experts", dict(num_experts=0), 1),
+    ("num_experts", dict(num_experts=4096, n_group=1, topk_group=1), 1),
+    ("num_experts_per_tok", dict(num_experts_per_tok=0), 1),
+    ("num_experts_per_tok", dict(num_experts_per_tok=257), 1),  # k > E
+    ("n_group", dict(n_group=0), 1),                     # zero checked before divisibility
+    ("n_group", dict(n_group=64, topk_group=4), 1),
+    ("divisible", dict(n_group=7, topk_group=4), 1),     # 256 % 7 != 0
+    ("topk_group", dict(topk_group=0), 1),
+    ("topk_group", dict(topk_group=9), 1),               # > n_group
+    ("topk_group", dict(n_group=8, topk_group=1, num_experts_per_tok=64), 1),  # too few experts kept
+    ("score_function", dict(score_function=2), 1),
+    ("score_function", dict(score_function=-1), 1),
+    ("norm_topk_prob", dict(norm_topk_prob=2), 1),
+    ("routed_scaling_factor", dict(routed_scaling_factor=float("nan")), 1),
+    ("routed_scaling_factor", dict(routed_scaling_factor=float("inf")), 1),
+    ("moe_intermediate_size", dict(moe_intermediate_size=0), 1),
+    ("moe_intermediate_size", dict(moe_intermediate_size=1030), 2),
+    ("num_shared_experts", dict(num_shared_experts=-1), 1),
+    ("num_shared_experts", dict(num_shared_experts=1000), 1),
+    ("moe_shared_expert_intermediate_size", dict(moe_shared_expert_intermediate_size=-8), 1),
+    ("moe_shared_expert_intermediate_size", dict(moe_shared_expert_intermediate_size=12), 2),
+]
+
+
+@pytest.mark.parametrize("field,over,status", BAD_CONFIGS, ids=[f"{b[0]}-{i}" for i, b in enumerate(BAD_CONFIGS)])
+def test_invalid_config_rejected(M, field, over, status):
+    c = _cfg(M, **over)
+    fake = ctypes.c_void_p(1 << 20)
+    for call in (
+        lambda: M.lib.moe_route(ctypes.byref(c), fake, None, 4, fake, fake, None),
+        lambda: M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None,
+                                  None, fake, 1 << 40, None),
+        lambda: M.lib.moe_combine(ctypes.byref(c), 4, fake, None, fake, None),
+    ):
+        st = call()
+        assert st == status, (field, st, M.last_error())
+        msg = M.last_error()
+        key = "num_experts" if field == "divisible" else field
+        assert key in msg, msg
+    assert M.lib.moe_workspace_size(ctypes.byref(c), 16) == 0
+
+
+def test_null_config_rejected(M):
+    assert M.lib.moe_route(None, None, None, 1, None, None, None) == 1
+    assert "cfg" in M.last_error()
+
+
+def test_valid_config_sizes(M):
+    c = _cfg(M)
+    n1 = M.lib.moe_workspace_size(ctypes.byref(c), 1)
+    n2 = M.lib.moe_workspace_size(ctypes.byref(c), 512)
+    assert 0 < n1 < n2 and n2 % 256 == 0
+    # topk_group == n_group is valid: every group kept
+    c2 = _cfg(M, topk_group=8)
+    assert M.lib.moe_workspace_size(ctypes.byref(c2), 8) > 0
+
+
+def test_token_count_rejected(M):
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    assert M.lib.moe_route(ctypes.byref(c), fake, None, -1, fake, fake, None) == 1
+    assert "T" in M.last_error()
+    assert M.lib.moe_route(ctypes.byref(c), fake, None, 1 << 40, fake, fake, None) == 1
+
+
+def test_zero_tokens_is_a_no_op(M):
+    c = _cfg(M)
+    assert M.lib.moe_route(ctypes.byref(c), None, None, 0, None, None, None) == 0
+    assert M.lib.moe_combine(ctypes.byref(c), 0, None, None, None, None) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(M):
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert M.lib.moe_route(ctypes.byref(c), None, None, 4, fake, fake, None) == 1
+    assert "logits" in M.last_error()
+    assert M.lib.moe_route(ctypes.byref(c), fake, None, 4, None, fake, None) == 1
+    assert "topk_idx" in M.last_error()
+    assert M.lib.moe_combine(ctypes.byref(c), 4, odd, None, fake, None) == 1
+    assert "y_slots" in M.last_error() and "aligned" in M.last_error()
+    ws_need = M.lib.moe_workspace_size(ctypes.byref(c), 4)
+    # forward: router weight required unless logits are given
+    st = M.lib.moe_forward(ctypes.byref(c), fake, 4, None, None, None, fake, fake, fake, fake, fake, None, None, fake,
+                           ws_need, None)
+    assert st == 1 and "router_w" in M.last_error()
+    # shared weights required when the config has a shared MLP
+    st = M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, None, None, fake, None, None, fake,
+                           ws_need, None)
+    assert st == 1 and "ws_gate_up" in M.last_error()
+    # and rejected when it has none
+    c0 = _cfg(M, num_shared_experts=0)
+    ws0 = M.lib.moe_workspace_size(ctypes.byref(c0), 4)
+    st = M.lib.moe_forward(ctypes.byref(c0), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None, None, fake,
+                           ws0, None)
+    assert st == 1 and "shared" in M.last_error()
+
+
+def test_workspace_rejected(M):
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    need = M.lib.moe_workspace_size(ctypes.byref(c), 64)
+    st = M.lib.moe_permute(ctypes.byref(c), fake, 64, None, fake, fake, fake, None, fake, need - 1, None)
+    assert st == 3 and "workspace" in M.last_error()
+    st = M.lib.moe_permute(ctypes.byref(c), fake, 64, None, fake, fake, fake, None, None, need, None)
+    assert st == 3
+    st = M.lib.moe_permute(ctypes.byref(c), fake, 64, None, fake, fake, fake, None, ctypes.c_void_p((1 << 20) + 16),
+                           need, None)
+    assert st == 3 and "aligned" in M.last_error()
+    assert M.lib.moe_workspace_init(None, 0, None) == 3
+
+
+def test_kernel_timer_arguments(M):
+    assert M.lib.moe_set_kernel_timer(99, None, None) == 1
+    assert M.lib.moe_set_kernel_timer(0, ctypes.c_void_p(8), None) == 1
+    assert M.lib.moe_set_kernel_timer(0, None, None) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    # The binding has no fallback: a missing library is an import error.
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "pkgcopy"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "grouped_top_routing_b200", "moe.py"), pkg / "moe.py")
+    spec = importlib.util.spec_from_file_location("moe_nolib", pkg / "moe.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,335 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Routing and permutation are compared bit for bit on identical inputs; the
+expert FFN and the whole block within max-abs 2e-2 / rel-L2 5e-3 against the
+fp64 oracle, near-tie tokens reported separately. Inputs are seeded and
+synthetic (grouped_top_routing_b200.inputs); the oracle never sees a value the
+CUDA path produced except where a test compares them.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import support as S
+from grouped_top_routing_b200 import build as B
+from grouped_top_routing_b200 import inputs as G
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def M():
+    B.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from grouped_top_routing_b200 import moe
+    return moe
+
+
+_CACHE = {}
+
+
+def _inputs(name, device=DEV, **over):
+    """Full-size inputs of a workload family, generated once on the device."""
+    key = (name, device, tuple(sorted(over.items())))
+    if key not in _CACHE:
+        _CACHE.clear()
+        torch.cuda.empty_cache()
+        wl = G.workload(name, **over)
+        _CACHE[key] = (wl, G.make_inputs(wl, seed=0, device=device))
+    return _CACHE[key]
+
+
+def _np_bias(inp):
+    b = inp["expert_bias"]
+    return None if b is None else b.detach().cpu().numpy().astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# routing workloads: (name, overrides)
+# ---------------------------------------------------------------------------
+ROUTE_CASES = [
+    ("ling_lite_t64", {}),
+    ("ling_lite_t64", dict(norm_topk_prob=True, routed_scaling_factor=2.5)),
+    ("ling26_flash_t512", {}),
+    ("ling30_flash_decode_t1", {}),
+    ("ling30_flash_decode_t8", {}),
+    ("ling30_flash_decode_t32", {}),
+    ("ling30_flash_decode_t64", {}),
+    ("ling30_flash_decode_t64", dict(norm_topk_prob=False, routed_scaling_factor=1.0)),
+    ("ling26_flash_prefill_t8192", {}),
+    ("ling26_flash_prefill_t32768", {}),
+    ("ling30_flash_skew_t16384", {}),
+    ("ling30_flash_skew_t16384", dict(norm_topk_prob=False, routed_scaling_factor=1.0)),
+    # edge shapes: E not a multiple of 32, k == E, one expert per group, k = 1
+    ("edge_e48_g4", dict(tokens=77, hidden_size=64, num_experts=48, num_experts_per_tok=5, n_group=4, topk_group=2,
+                         score_function="softmax", bias="normal")),
+    ("edge_k_eq_e", dict(tokens=33, hidden_size=64, num_experts=8, num_experts_per_tok=8, n_group=2, topk_group=2,
+                         score_function="softmax", bias="none")),
+    ("edge_group_of_one", dict(tokens=40, hidden_size=64, num_experts=16, num_experts_per_tok=2, n_group=16,
+                               topk_group=4, score_function="sigmoid", bias="normal")),
+    ("edge_k1", dict(tokens=50, hidden_size=64, num_experts=64, num_experts_per_tok=1, score_function="sigmoid",
+                     bias="normal", norm_topk_prob=True, routed_scaling_factor=2.5)),
+    ("edge_e1024", dict(tokens=20, hidden_size=64, num_experts=1024, num_experts_per_tok=16, n_group=32,
+                        topk_group=8, score_function="sigmoid", bias="normal")),
+]
+
+
+def _route_wl(name, over):
+    if name.startswith("edge_"):
+        return G.tiny_workload(**over)
+    return G.workload(name, **over)
+
+
+@pytest.mark.parametrize("name,over", ROUTE_CASES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(ROUTE_CASES)])
+def test_route_bit_exact(M, name, over):
+    wl = _route_wl(name, over)
+    T, E, k = wl["tokens"], wl["num_experts"], wl["num_experts_per_tok"]
+    inp = G.make_inputs(wl, seed=0, device="cpu", weights=False, tokens=1)
+    bias = _np_bias(inp)
+    L = G.random_logits(T, E, S.logit_std(wl), seed=1).numpy()
+    ties = None
+    if wl["bias"] == "zipf":
+        toks, pairs = S.add_exact_ties(L, bias, k)
+        S.check_ties_constructed(L, bias, wl, toks, pairs)
+        ties = (toks, pairs)
+    ref_idx, ref_w = O.route(L, bias, wl)
+    Ld = torch.from_numpy(L).to(DEV)
+    bd = None if bias is None else torch.from_numpy(bias).to(DEV)
+    idx, w = M.moe_route(wl, Ld, bd)
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    bad = np.nonzero((idx != ref_idx).any(1))[0]
+    assert bad.size == 0, f"{bad.size} tokens differ, first {bad[:5]}: gpu {idx[bad[:2]]} oracle {ref_idx[bad[:2]]}"
+    assert np.array_equal(w.view(np.uint32), ref_w.view(np.uint32)), np.abs(w - ref_w).max()
+    if ties is not None:
+        toks, pairs = ties
+        assert np.all(idx[toks, k - 1] == pairs), "exact ties must go to the lower expert id"
+        print(f"{len(toks)} exact-tie tokens resolved to the lower id")
+    near, _ = S.near_tie_tokens(L, bias, wl)
+    print(f"{name}: {T} tokens bit-exact; {int(near.sum())} near-tie tokens (gap < 1e-6) included")
+
+
+@pytest.mark.parametrize("name,T", [("ling_lite_t64", 64), ("ling26_flash_t512", 512), ("ling30_flash_decode_t1", 1),
+                                    ("ling30_flash_decode_t8", 8), ("ling30_flash_decode_t32", 32),
+                                    ("ling26_flash_t512", 77)])
+def test_router_logits(M, name, T):
+    wl = G.workload(name)
+    inp = G.make_inputs(wl, seed=0, device="cpu", weights=False, tokens=T)
+    ref = O.router_logits(inp["x"], inp["router_w"]).astype(np.float64)
+    got = M.moe_router_logits(wl, inp["x"].to(DEV), inp["router_w"].to(DEV)).cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref).max()
+    print(f"{name} T={T}: max |logit - oracle| = {err:.3e}")
+    # fp32 accumulation over H terms of size ~0.02: a few 1e-6 typical
+    assert err < 5e-5
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 512, 8), (5, 64, 6), (128, 256, 8), (129, 256, 8), (300, 48, 5),
+                                   (4096, 512, 8), (32768, 256, 8), (1000, 1024, 16)])
+def test_permute_bit_exact(M, T, E, k):
+    wl = G.tiny_workload(tokens=T, num_experts=E, num_experts_per_tok=k, hidden_size=64, score_function="sigmoid")
+    L = G.random_logits(T, E, 1.0, seed=T).numpy()
+    idx, _ = O.route(L, None, wl)
+    off, row_of, tok_of = O.permutation(idx, E)
+    x = G.make_inputs(wl, seed=0, device="cpu", weights=False)["x"]
+    ws = M.Workspace(wl, T)
+    d_off, d_row, d_tok, d_xp = M.moe_permute(wl, torch.from_numpy(idx).to(DEV), ws, x=x.to(DEV), want_x_perm=True)
+    ws.check()
+    assert np.array_equal(d_off.cpu().numpy(), off)
+    assert np.array_equal(d_row.cpu().numpy(), row_of)
+    assert np.array_equal(d_tok.cpu().numpy(), tok_of)
+    xp = d_xp.cpu().view(torch.int16).numpy()
+    assert np.array_equal(xp, x.view(torch.int16).numpy()[tok_of // k])
+
+
+def test_permute_rejects_bad_ids_on_device(M):
+    wl = G.tiny_workload(tokens=200, num_experts=16, num_experts_per_tok=2, hidden_size=64)
+    idx = torch.zeros((200, 2), dtype=torch.int32)
+    idx[:, 0] = torch.arange(200) % 16
+    idx[:, 1] = (torch.arange(200) + 1) % 16
+    idx[17, 1] = 16       # out of range
+    idx[30, 1] = idx[30, 0]  # repeated within a token
+    ws = M.Workspace(wl, 200)
+    M.moe_permute(wl, idx.to(DEV), ws)
+    with pytest.raises(M.MoeError) as ei:
+        ws.check()
+    assert ei.value.status == 5
+    ws.check()  # the word was cleared; the workspace is usable again
+    idx[17, 1] = 3
+    idx[30, 1] = 4
+    off, _, _, _ = M.moe_permute(wl, idx.to(DEV), ws)
+    ws.check()
+    assert int(off[-1]) == 400
+
+
+def test_combine_definition(M):
+    # y[t] = bf16(sum_j float(y_slots[t*k+j]) + float(shared[t])), fp32, slot order
+    T, k, H = 37, 6, 256
+    g = torch.Generator().manual_seed(3)
+    ys = torch.randn((T * k, H), generator=g).to(torch.bfloat16)
+    sh = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    wl = G.tiny_workload(hidden_size=H, num_experts=8, num_experts_per_tok=k)
+    y = M.moe_combine(wl, ys.to(DEV), sh.to(DEV), T).cpu()
+    acc = np.zeros((T, H), np.float32)
+    f = ys.float().numpy().reshape(T, k, H)
+    for j in range(k):
+        acc = (acc + f[:, j]).astype(np.float32)
+    acc = (acc + sh.float().numpy()).astype(np.float32)
+    ref = torch.from_numpy(acc).to(torch.bfloat16)
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    y0 = M.moe_combine(wl, ys.to(DEV), None, T).cpu()
+    acc0 = np.zeros((T, H), np.float32)
+    for j in range(k):
+        acc0 = (acc0 + f[:, j]).astype(np.float32)
+    assert torch.equal(y0.view(torch.int16), torch.from_numpy(acc0).to(torch.bfloat16).view(torch.int16))
+
+
+FFN_CASES = [
+    ("ling_lite_t64", {}),
+    ("ling30_flash_decode_t8", {}),
+    ("tiny_no_shared", dict(tokens=40, hidden_size=256, num_experts=16, num_experts_per_tok=4,
+                            moe_intermediate_size=128, num_shared_experts=0, shared_width=0)),
+    ("tiny_ragged", dict(tokens=13, hidden_size=136, num_experts=12, num_experts_per_tok=3,
+                         moe_intermediate_size=72, shared_width=144, num_shared_experts=2)),
+]
+
+
+@pytest.mark.parametrize("name,over", FFN_CASES, ids=[c[0] for c in FFN_CASES])
+def test_expert_ffn(M, name, over):
+    if name.startswith("tiny"):
+        wl = G.tiny_workload(**over)
+        inp = S.inputs_to(G.make_inputs(wl, seed=0, device="cpu"), DEV)
+    else:
+        wl, inp = _inputs(name)
+    T, E, k, H = inp["tokens"], wl["num_experts"], wl["num_experts_per_tok"], wl["hidden_size"]
+    L = G.random_logits(T, E, S.logit_std(wl), seed=5).numpy()
+    idx, w = O.route(L, _np_bias(inp), wl)
+    ws = M.Workspace(wl, T)
+    d_idx = torch.from_numpy(idx).to(DEV)
+    d_w = torch.from_numpy(w).to(DEV)
+    off, _, tok_of, _ = M.moe_permute(wl, d_idx, ws)
+    has_shared = inp["ws_gate_up"] is not None
+    y_slots, shared = M.moe_expert_ffn(wl, inp["x"], off, tok_of, d_w.reshape(-1), inp["w_gate_up"], inp["w_down"],
+                                       ws, ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"])
+    ws.check()
+    X = O.as_f64(inp["x"])
+    I = wl["moe_intermediate_size"]
+    ref = np.zeros((T * k, H))
+    for e in np.unique(idx):
+        t_sel, j_sel = np.nonzero(idx == e)
+        Wg, Wu, Wd = O.expert_weights_f64(inp["w_gate_up"], inp["w_down"], int(e), I)
+        ref[t_sel * k + j_sel] = w[t_sel, j_sel][:, None].astype(np.float64) * O.swiglu_mlp(X[t_sel], Wg, Wu, Wd)
+    S.compare(O.as_f64(y_slots), ref, f"{name} y_slots")
+    if has_shared:
+        Wg, Wu, Wd = O.shared_weights_f64(inp["ws_gate_up"], inp["ws_down"])
+        S.compare(O.as_f64(shared), O.swiglu_mlp(X, Wg, Wu, Wd), f"{name} shared")
+
+
+# ---------------------------------------------------------------------------
+# whole block
+# ---------------------------------------------------------------------------
+
+def _forward_and_compare(M, wl, inp, tokens=None, logits=None):
+    """Run moe_forward on all tokens; compare (all or sampled) tokens with the
+    oracle run on its own router logits (or on the given logits)."""
+    T = inp["tokens"]
+    ws = M.Workspace(wl, T)
+    Ld = None if logits is None else torch.from_numpy(logits).to(DEV)
+    y, idx, w = M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                              inp["ws_gate_up"], inp["ws_down"], ws, logits_override=Ld, return_routing=True)
+    ws.check()
+    rows = np.arange(T) if tokens is None else np.asarray(tokens)
+    bias = _np_bias(inp)
+    if logits is None:
+        L = O.router_logits(inp["x"][torch.from_numpy(rows).to(DEV)], inp["router_w"])
+    else:
+        L = logits[rows]
+    ref_idx, ref_w = O.route(L, bias, wl)
+    g_idx = idx.cpu().numpy()[rows]
+    g_w = w.cpu().numpy()[rows]
+    near, gap = S.near_tie_tokens(L, bias, wl)
+    differ = (np.sort(g_idx, 1) != np.sort(ref_idx, 1)).any(1)
+    if logits is not None:
+        assert not differ.any(), "identical logits must give identical routing"
+        assert np.array_equal(g_idx, ref_idx) and np.array_equal(g_w.view(np.uint32), ref_w.view(np.uint32))
+    # With the router projection on both sides, fp32 accumulation order can flip
+    # only tokens whose selection gap is within the logits' rounding (<< 1e-5).
+    assert np.all(gap[differ] < 1e-5), f"routing differs off the tie band: gaps {gap[differ]}"
+    keep = ~(differ | near)
+    sub = {k2: v for k2, v in inp.items()}
+    sub["x"] = inp["x"][torch.from_numpy(rows[keep]).to(DEV)]
+    ref = O.moe_block(sub, wl, logits=L[keep])["y"]
+    got = O.as_f64(y[torch.from_numpy(rows[keep]).to(DEV)])
+    ma, rl = S.compare(got, ref, f"{wl.get('name', '')} T={T} y ({keep.sum()} tokens)")
+    print(f"near-tie tokens reported separately: {int(near.sum())}; routing flips inside 1e-5: {int(differ.sum())}")
+    return y
+
+
+FORWARD_CASES = [
+    ("ling_lite_t64", {}),
+    ("ling_lite_t64", dict(norm_topk_prob=True, routed_scaling_factor=2.5)),
+    ("ling26_flash_t512", {}),
+    ("ling30_flash_decode_t64", {}),
+    ("ling30_flash_decode_t64", dict(norm_topk_prob=False, routed_scaling_factor=1.0)),
+]
+
+
+@pytest.mark.parametrize("name,over", FORWARD_CASES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(FORWARD_CASES)])
+def test_forward_matches_oracle(M, name, over):
+    wl, inp = _inputs(name)
+    wl = dict(wl, **over, name=name)
+    _forward_and_compare(M, wl, inp)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32])
+def test_forward_decode_batches(M, T):
+    wl, inp = _inputs("ling30_flash_decode_t64")
+    sub = dict(inp, x=inp["x"][:T].contiguous(), tokens=T)
+    _forward_and_compare(M, dict(wl, name=f"decode_t{T}"), sub)
+
+
+@pytest.mark.parametrize("name", ["ling26_flash_prefill_t8192", "ling26_flash_prefill_t32768"])
+def test_forward_prefill_sampled(M, name):
+    wl, inp = _inputs(name)
+    T = inp["tokens"]
+    rows = np.unique(np.concatenate([np.linspace(0, T - 1, 40).astype(int), [0, 1, T - 1]]))
+    _forward_and_compare(M, dict(wl, name=name), inp, tokens=rows)
+
+
+def test_forward_skew_ties_sampled(M):
+    wl, inp = _inputs("ling30_flash_skew_t16384")
+    T, E, k = inp["tokens"], wl["num_experts"], wl["num_experts_per_tok"]
+    bias = _np_bias(inp)
+    L = O.router_logits(inp["x"], inp["router_w"]) if False else G.random_logits(T, E, S.logit_std(wl), seed=2).numpy()
+    toks, pairs = S.add_exact_ties(L, bias, k)
+    S.check_ties_constructed(L, bias, wl, toks, pairs)
+    rows = np.unique(np.concatenate([toks[:12], np.linspace(0, T - 1, 36).astype(int)]))
+    _forward_and_compare(M, dict(wl, name="skew"), inp, tokens=rows, logits=L)
+
+
+def test_forward_deterministic(M):
+    wl, inp = _inputs("ling26_flash_t512")
+    ws = M.Workspace(wl, inp["tokens"])
+    args = (wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"],
+            inp["ws_down"], ws)
+    a = M.moe_forward(*args).clone()
+    b = M.moe_forward(*args).clone()
+    ws.check()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_forward_zero_tokens_and_launch_count(M):
+    wl, inp = _inputs("ling26_flash_t512")
+    ws = M.Workspace(wl, 1)
+    n0 = M.launch_count()
+    x0 = inp["x"][:0]
+    y = M.moe_forward(wl, x0, inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                      inp["ws_gate_up"], inp["ws_down"], ws)
+    assert y.shape == (0, wl["hidden_size"]) and M.launch_count() == n0
+    x1 = inp["x"][:1].contiguous()
+    M.moe_forward(wl, x1, inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"],
+                  inp["ws_down"], ws)
+    ws.check()
+    assert M.launch_count() > n0
