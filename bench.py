@@ -163,11 +163,21 @@ def time_oracle(wl, inp, token_rows):
     return time.perf_counter() - t0
 
 
+def workload_from_args(args):
+    wl = G.workload(args.workload)
+    for kv in args.set:
+        key, val = kv.split("=", 1)
+        if key not in wl:
+            raise SystemExit(f"unknown workload field {key}")
+        wl[key] = type(wl[key])(val) if not isinstance(wl[key], bool) else val.lower() in ("1", "true")
+    return wl
+
+
 def run_reference(args):
     rank = _env_int("RANK", 0)
     if rank != 0:
         return 0
-    wl = G.workload(args.workload)
+    wl = workload_from_args(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = G.make_inputs(wl, seed=0, device=dev)  # generation is not timed; the oracle pulls rows to the host
     T = inp["tokens"]
@@ -211,7 +221,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = G.workload(args.workload)
+    wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
     if rank > 0:  # each rank its own batch (weak scaling), same weights
@@ -242,6 +252,9 @@ def run_ours(args):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in kev:  # torch creates the CUDA event on first record; the library needs the handles
+        a.record(stream)
+        b.record(stream)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -317,7 +330,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "tokens": T, "hidden_size": wl["hidden_size"],
+        "config": {"workload": args.workload, "overrides": args.set, "tokens": T, "hidden_size": wl["hidden_size"],
                    "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
@@ -346,6 +359,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=64)
     ap.add_argument("--ref-sample", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a workload field (e.g. num_experts=64 for a small profiling case)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

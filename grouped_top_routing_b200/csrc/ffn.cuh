@@ -18,12 +18,14 @@ struct FfnArgs {
   const uint16_t* w_down;     // [E, H, I]
   const uint16_t* ws_gate_up; // [2Is, H] or null
   const uint16_t* ws_down;    // [H, Is]
-  uint16_t* h_perm;           // [T*k, I]
-  uint16_t* h_shared;         // [T, Is]
-  uint16_t* y_slots;          // [T*k, H]
-  uint16_t* shared_out;       // [T, H]
+  void* h_perm;               // [T*k, I]: fp32 (streaming path) or bf16 (tensor-core path)
+  void* h_shared;             // [T, Is]: same element type as h_perm
+  float* y_slots;             // [T*k, H]
+  float* shared_out;          // [T, H]
 };
 
 cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s);
+int umma_pick_bn(int64_t T, int k, int E);
+cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cudaStream_t s);
 
 }  // namespace moe

@@ -125,9 +125,9 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
           const float g = warp_sum(ag[t]);
           const float u = warp_sum(au[t]);
           if (lane == t && xr[t] != nullptr) {
-            const uint16_t h = f32_to_bf16(silu_f32(g) * u);
-            if (!shared) a.h_perm[(r0 + c0 + t) * a.I + j] = h;
-            else a.h_shared[(c0 + t) * a.Is + j] = h;
+            const float h = silu_f32(g) * u;  // kept in fp32 on this path
+            if (!shared) static_cast<float*>(a.h_perm)[(r0 + c0 + t) * a.I + j] = h;
+            else static_cast<float*>(a.h_shared)[(c0 + t) * a.Is + j] = h;
           }
         }
       }
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
     const bool shared = item >= routed_items;
     int n0, K;
     const uint16_t* w0;
-    const uint16_t* hin;
+    const float* hin;
     int64_t r0 = 0, m = 0;
     if (!shared) {
       const int aidx = (int)(item / nrb);
@@ -158,12 +158,12 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
       if (!expert_rows(a, aidx, e, r0, m)) continue;
       K = a.I;
       w0 = a.w_down + ((int64_t)e * H + n0) * K;
-      hin = a.h_perm;
+      hin = static_cast<const float*>(a.h_perm);
     } else {
       n0 = (int)(item - routed_items) * kDownRows;
       K = a.Is;
       w0 = a.ws_down + (int64_t)n0 * K;
-      hin = a.h_shared;
+      hin = static_cast<const float*>(a.h_shared);
       m = a.T;
     }
     const int nvk = K / 8;
@@ -184,8 +184,9 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
 #pragma unroll
         for (int t = 0; t < kTok; ++t) {
           if (t < mc) {
-            float hf[8];
-            unpack8_bf16(ld_nc_u4(hin + (r0 + c0 + t) * K + v * 8), hf);
+            const float4* hp = reinterpret_cast<const float4*>(hin + (r0 + c0 + t) * K + v * 8);
+            const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
+            const float hf[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
             for (int r = 0; r < kDownRows; ++r)
               if (r < nrows) acc[r][t] = dot8_bf16(wv[r], hf, acc[r][t]);
@@ -207,48 +208,45 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
           int64_t slot;
           if (slot_token(a, r0 + c0 + t, slot) >= 0) {
             const float w = a.topk_w != nullptr ? a.topk_w[slot] : 1.0f;
-            a.y_slots[slot * H + n0 + r] = f32_to_bf16(w * mine);
+            a.y_slots[slot * H + n0 + r] = w * mine;
           }
         } else {
-          a.shared_out[(c0 + t) * H + n0 + r] = f32_to_bf16(mine);
+          a.shared_out[(c0 + t) * H + n0 + r] = mine;
         }
       }
     }
   }
 }
 
-// y[t] = bf16( sum_j float(y_slots[t*k + j]) + float(shared_out[t]) ), in
-// slot order then the shared row; one thread per 8 outputs.
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y_slots,
-                                                      const uint16_t* __restrict__ shared_out, int64_t T, int k,
-                                                      int H, uint16_t* __restrict__ y) {
-  const int nv = H / 8;
+// y[t] = bf16( sum_j y_slots[t*k + j] + shared_out[t] ), fp32 in slot order
+// then the shared row, one rounding; one thread per 4 outputs.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_slots,
+                                                      const float* __restrict__ shared_out, int64_t T, int k, int H,
+                                                      uint16_t* __restrict__ y) {
+  const int nv = H / 4;
   const int64_t n = T * nv;
-  const uint4* ys = reinterpret_cast<const uint4*>(y_slots);
-  const uint4* sh = reinterpret_cast<const uint4*>(shared_out);
-  uint4* out = reinterpret_cast<uint4*>(y);
+  const float4* ys = reinterpret_cast<const float4*>(y_slots);
+  const float4* sh = reinterpret_cast<const float4*>(shared_out);
+  uint2* out = reinterpret_cast<uint2*>(y);
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / nv;
     const int v = (int)(i - t * nv);
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
-      float f[8];
-      unpack8_bf16(__ldg(ys + (t * k + j) * nv + v), f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+      const float4 f = __ldg(ys + (t * k + j) * nv + v);
+      acc.x += f.x;
+      acc.y += f.y;
+      acc.z += f.z;
+      acc.w += f.w;
     }
     if (sh != nullptr) {
-      float f[8];
-      unpack8_bf16(__ldg(sh + i), f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+      const float4 f = __ldg(sh + i);
+      acc.x += f.x;
+      acc.y += f.y;
+      acc.z += f.z;
+      acc.w += f.w;
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    out[i] = o;
+    out[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   }
 }
 
@@ -267,10 +265,10 @@ cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const uint16_t* y_slots, const uint16_t* shared_out, int64_t T, int k, int H,
-                           uint16_t* y, cudaStream_t s) {
+cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
+                           cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int64_t n = T * (H / 8);
+  const int64_t n = T * (H / 4);
   int64_t blocks = (n + 255) / 256;
   const int64_t cap = (int64_t)sm_count() * 8;
   if (blocks > cap) blocks = cap;

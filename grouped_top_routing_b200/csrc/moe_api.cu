@@ -26,8 +26,10 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
                            int32_t* tile_base, WsHeader* hdr, cudaStream_t s);
 cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, WsHeader* hdr,
                                        cudaStream_t s);
-cudaError_t launch_combine(const uint16_t* y_slots, const uint16_t* shared_out, int64_t T, int k, int H,
-                           uint16_t* y, cudaStream_t s);
+cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
+                           cudaStream_t s);
+cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
+                               const uint16_t* x, int H, uint16_t* x_perm, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // errors, hooks, device cache
@@ -39,6 +41,7 @@ std::atomic<uint64_t> g_launches{0};
 void* g_ev_start[MOE_KERNEL_COUNT] = {};
 void* g_ev_stop[MOE_KERNEL_COUNT] = {};
 int g_sm_count[64] = {};
+int g_ffn_path = 0;  // 0 auto, 1 streaming GEMV, 2 tensor cores
 
 moe_status fail(moe_status st, const char* fmt, ...) {
   va_list ap;
@@ -196,10 +199,10 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   L.tile_cnt = take(permute_scratch_ints((int)E, T) * 4);
   L.tile_base = take(permute_scratch_ints((int)E, T) * 4);
   L.x_perm = take((size_t)R * H * 2);
-  L.h_perm = take((size_t)R * I * 2);
-  L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 2);
-  L.y_slots = take((size_t)R * H * 2);
-  L.shared_out = take((size_t)T * H * 2);
+  L.h_perm = take((size_t)R * I * 4);                  // fp32 (streaming) or bf16 (tensor cores)
+  L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 4);
+  L.y_slots = take((size_t)R * H * 4);
+  L.shared_out = take((size_t)T * H * 4);
   L.total = off;
   return L;
 }
@@ -220,10 +223,18 @@ moe_status check_ws(const moe_config& c, int64_t T, void* ws, size_t ws_bytes) {
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
+// Tensor cores once experts average at least two rows; below that (decode)
+// the streaming GEMV spreads the weight rows over every SM.
+bool use_tensor_cores(const moe_config& c, int64_t T) {
+  if (g_ffn_path == 1) return false;
+  if (g_ffn_path == 2) return true;
+  return T * c.num_experts_per_tok >= 2 * (int64_t)c.num_experts;
+}
+
 moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint16_t* x_perm,
                    const int32_t* offsets, const int32_t* tok_of, const float* topk_w, const uint16_t* wgu,
-                   const uint16_t* wd, const uint16_t* swgu, const uint16_t* swd, uint16_t* y_slots,
-                   uint16_t* shared_out, void* ws, bool active_ready, cudaStream_t s) {
+                   const uint16_t* wd, const uint16_t* swgu, const uint16_t* swd, float* y_slots, float* shared_out,
+                   void* ws, bool active_ready, cudaStream_t s) {
   const Layout L = layout(c, T);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
   int32_t* active = at<int32_t>(ws, L.active);
@@ -249,11 +260,21 @@ moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint
   a.w_down = wd;
   a.ws_gate_up = (swgu != nullptr && a.Is > 0) ? swgu : nullptr;
   a.ws_down = a.ws_gate_up != nullptr ? swd : nullptr;
-  a.h_perm = at<uint16_t>(ws, L.h_perm);
-  a.h_shared = at<uint16_t>(ws, L.h_shared);
+  a.h_perm = at<void>(ws, L.h_perm);
+  a.h_shared = at<void>(ws, L.h_shared);
   a.y_slots = y_slots;
   a.shared_out = shared_out;
-  (void)x_perm;
+  if (use_tensor_cores(c, T)) {
+    if (x_perm == nullptr) {  // the tensor-core path reads expert rows contiguously
+      uint16_t* xp = at<uint16_t>(ws, L.x_perm);
+      e = launch_gather_rows(offsets, c.num_experts, tok_of, c.num_experts_per_tok, T, x, c.hidden_size, xp, s);
+      if (e != cudaSuccess) return cuda_fail(e, "gather rows");
+      x_perm = xp;
+    }
+    e = launch_umma_ffn(a, x_perm, umma_pick_bn(T, a.k, a.E), s);
+    if (e != cudaSuccess) return cuda_fail(e, "expert ffn (tensor cores)");
+    return MOE_OK;
+  }
   e = launch_gemv_ffn(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "expert ffn");
   return MOE_OK;
@@ -342,7 +363,7 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T
 moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, const uint16_t* x_perm,
                           const int32_t* expert_offsets, const int32_t* tok_of, const float* topk_w,
                           const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* ws_gate_up,
-                          const uint16_t* ws_down, uint16_t* y_slots, uint16_t* shared_out, void* ws,
+                          const uint16_t* ws_down, float* y_slots, float* shared_out, void* ws,
                           size_t ws_bytes, void* stream) {
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
@@ -367,7 +388,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, c
                  shared_out, ws, false, as_stream(stream));
 }
 
-moe_status moe_combine(const moe_config* cfg, int64_t T, const uint16_t* y_slots, const uint16_t* shared_out,
+moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, const float* shared_out,
                        uint16_t* y, void* stream) {
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
@@ -422,12 +443,13 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   if (e != cudaSuccess) return cuda_fail(e, "route");
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* tok_of = at<int32_t>(ws, L.tok_of);
-  e = launch_permute(c, idx, T, x, offsets, at<int32_t>(ws, L.row_of), tok_of, nullptr, at<int32_t>(ws, L.active),
+  uint16_t* x_perm = use_tensor_cores(c, T) ? at<uint16_t>(ws, L.x_perm) : nullptr;
+  e = launch_permute(c, idx, T, x, offsets, at<int32_t>(ws, L.row_of), tok_of, x_perm, at<int32_t>(ws, L.active),
                      at<int32_t>(ws, L.tile_cnt), at<int32_t>(ws, L.tile_base), hdr, s);
   if (e != cudaSuccess) return cuda_fail(e, "permute");
-  uint16_t* y_slots = at<uint16_t>(ws, L.y_slots);
-  uint16_t* shared_out = has_shared ? at<uint16_t>(ws, L.shared_out) : nullptr;
-  MOE_TRY(run_ffn(c, T, x, nullptr, offsets, tok_of, w, w_gate_up, w_down, has_shared ? ws_gate_up : nullptr,
+  float* y_slots = at<float>(ws, L.y_slots);
+  float* shared_out = has_shared ? at<float>(ws, L.shared_out) : nullptr;
+  MOE_TRY(run_ffn(c, T, x, x_perm, offsets, tok_of, w, w_gate_up, w_down, has_shared ? ws_gate_up : nullptr,
                   has_shared ? ws_down : nullptr, y_slots, shared_out, ws, true, s));
   e = launch_combine(y_slots, shared_out, T, c.num_experts_per_tok, c.hidden_size, y, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine");
@@ -460,6 +482,12 @@ moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moe_status moe_set_ffn_path(int32_t path) {
+  if (path < 0 || path > 2) return fail(MOE_ERR_INVALID_ARG, "path = %d is not 0 (auto), 1 (streaming) or 2 (tensor cores)", path);
+  g_ffn_path = path;
+  return MOE_OK;
+}
 
 const char* moe_last_error(void) { return g_err; }
 

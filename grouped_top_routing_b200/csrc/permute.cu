@@ -262,6 +262,19 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
+                               const uint16_t* x, int H, uint16_t* x_perm, cudaStream_t s) {
+  const int64_t chunks = T * k * (H / 8);
+  int64_t blocks = (chunks + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  before_launch(MOE_KERNEL_PERMUTE, s);
+  gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(offsets, E, tok_of, k, T, x, H, x_perm);
+  after_launch(MOE_KERNEL_PERMUTE, s);
+  return cudaGetLastError();
+}
+
 // Rebuilds the compacted list of experts with rows from expert_offsets (used
 // when moe_expert_ffn is called on its own).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,

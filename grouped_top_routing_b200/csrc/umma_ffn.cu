@@ -1,0 +1,633 @@
+// Expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Each routed expert (and the shared MLP) is a dense contraction over the
+// tokens routed to it: the gather-matmul of mlxcel issue #838 (section
+// "Weight remap": experts stacked into switch_mlp tensors; section
+// "Architecture notes": SwiGLU experts plus one always-on shared MLP).
+//
+// Orientation: the weight rows are the MMA's M side (128 rows per operand) and
+// the expert's tokens its N side (BN columns), so an expert that received only
+// a handful of tokens still fills the 128-row tensor-core tile, and every
+// weight tile is read from HBM once per BN tokens.
+//
+//   pass GATE_UP: D0 = W_gate[n0:n0+128] . X^T, D1 = W_up[n0:n0+128] . X^T,
+//                 h[token, n0+i] = silu(D0[i]) * D1[i]  -> (h_hi, h_lo)
+//   pass DOWN   : D0 = W_down[n0:n0+128] . H^T, D1 = W_down[n0+128:n0+256] . H^T,
+//                 y_slots[slot(token), n] = w_slot * D[n]  (fp32; shared MLP: weight 1)
+//
+// h is written as two bf16 planes, h_hi = bf16(h) and h_lo = bf16(h - h_hi),
+// and the DOWN pass accumulates W.h_hi + W.h_lo from the same weight tile: the
+// SwiGLU product then carries ~16 significant bits into the down projection
+// instead of bf16's 8, at the cost of a second MMA per weight tile (no extra
+// weight bytes).
+//
+// Persistent, warp-specialised CTA (one per SM, 192 threads):
+//   warp 0      : TMA producer (one lane), STAGES-deep ring of (A0, A1, B) tiles
+//   warp 1      : TMEM allocator; one lane issues tcgen05.mma, commits to barriers
+//   warps 2..5  : epilogue; TMEM -> registers (tcgen05.ld), SwiGLU / weighting, stores
+// The two TMEM accumulator pairs are double-buffered so the epilogue of one tile
+// overlaps the main loop of the next. Tiles run (group, n-block, m-block) with
+// the m-block fastest, so CTAs that share a weight block run side by side and
+// the re-reads of that block hit L2.
+//
+// Every mbarrier wait is bounded (globaltimer, ~2 s). A wait that runs out sets
+// MOE_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag, and all roles
+// wind down: the producer waits (bounded) for its copies in flight, the MMA lane
+// waits (bounded) for its MMAs, and TMEM is freed before the CTA exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ffn.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;         // weight rows per A operand (MMA M)
+constexpr int BK = 64;          // K per stage: 64 bf16 = 128 bytes = one swizzle span
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 1025;  // routed experts (<= 1024) + the shared MLP
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+enum : int { kGateUp = 0, kDown = 1 };
+
+struct UmmaParams {
+  int64_t T;
+  int H, I, Is, k, E;
+  int has_shared;
+  const int32_t* offsets;
+  const int32_t* tok_of;
+  const int32_t* active;
+  WsHeader* hdr;
+  const float* topk_w;
+  uint16_t* h_perm;    // hi plane [T*k, I], lo plane follows
+  uint16_t* h_shared;  // hi plane [T, Is], lo plane follows
+  float* y_slots;
+  float* shared_out;
+};
+
+// ----------------------------------------------------------------------------
+// PTX wrappers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `bar` with the given parity. Returns false when
+// the CTA is aborting or the wait ran out (which raises the abort).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, WsHeader* hdr,
+                                         int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        *abort_flag = 1;
+        record_error(hdr, MOE_ERR_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kTimeoutNs) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_addr(dst)),
+      "l"(map), "r"(smem_addr(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] . B[smem]^T, bf16 inputs, fp32 accumulate, 128 x N x 16.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive fp32 columns of TMEM into registers.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major tile, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (the layout a TMA box {64, rows}
+// with CU_TENSOR_MAP_SWIZZLE_128B writes).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
+template <int N>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------
+// tile schedule
+// ----------------------------------------------------------------------------
+struct TileInfo {
+  bool shared;
+  int e, m, nb, mb;
+  int64_t r0;
+  int a0_row, a1_row, b_row, kblocks;
+};
+
+template <int BN, int MODE>
+__device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const int* pre, const int* s_e, const int* s_m,
+                                                const int* s_r0, const UmmaParams& p) {
+  int lo = 0, hi = n_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  TileInfo t;
+  t.e = s_e[lo];
+  t.shared = t.e < 0;
+  t.m = s_m[lo];
+  t.r0 = s_r0[lo];
+  const int mblocks = (t.m + BN - 1) / BN;
+  const int local = tile - pre[lo];
+  t.nb = local / mblocks;
+  t.mb = local - t.nb * mblocks;
+  int K;
+  if (MODE == kGateUp) {
+    K = p.H;
+    if (t.shared) {
+      t.a0_row = t.nb * BM;
+      t.a1_row = p.Is + t.nb * BM;
+    } else {
+      t.a0_row = t.e * 2 * p.I + t.nb * BM;
+      t.a1_row = t.a0_row + p.I;
+    }
+  } else {
+    K = t.shared ? p.Is : p.I;
+    t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * 2 * BM;
+    t.a1_row = t.a0_row + BM;
+  }
+  t.b_row = (int)t.r0 + t.mb * BN;
+  t.kblocks = (K + BK - 1) / BK;
+  return t;
+}
+
+template <int BN, int STAGES, int NB>
+struct Smem {
+  static constexpr int kA = BM * BK * 2;
+  static constexpr int kB = BN * BK * 2;
+  static constexpr int kStage = 2 * kA + NB * kB;
+  static constexpr int kBarriers = (2 * STAGES + 5) * 8;
+  static constexpr int kTables = 4 * (kMaxGroups + 1) * 4;
+  static constexpr size_t kTotal = 1024 + (size_t)STAGES * kStage + kBarriers + 16 + kTables;
+};
+
+template <int BN, int STAGES, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    umma_ffn_kernel(const __grid_constant__ CUtensorMap mapA_r, const __grid_constant__ CUtensorMap mapB_r,
+                    const __grid_constant__ CUtensorMap mapB2_r, const __grid_constant__ CUtensorMap mapA_s,
+                    const __grid_constant__ CUtensorMap mapB_s, const __grid_constant__ CUtensorMap mapB2_s,
+                    const UmmaParams p) {
+  constexpr int NB = MODE == kDown ? 2 : 1;  // DOWN reads the h_hi and h_lo planes
+  using L = Smem<BN, STAGES, NB>;
+  constexpr uint32_t kTmemCols = 4 * BN;  // two buffers x (D0, D1)
+  constexpr uint32_t kIdesc = idesc_bf16<BN>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * L::kStage);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* pre = reinterpret_cast<int*>(tmem_slot + 4);
+  int* s_e = pre + (kMaxGroups + 1);
+  int* s_m = s_e + (kMaxGroups + 1);
+  int* s_r0 = s_m + (kMaxGroups + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+
+  // ---- group table: active experts (+ shared MLP), tiles per group ----
+  const int n_act = min(max(*(volatile int*)&p.hdr->num_active, 0), p.E);
+  const int n_groups = n_act + (p.has_shared ? 1 : 0);
+  const int64_t R = p.T * p.k;
+  const int nb_routed = MODE == kGateUp ? (p.I + BM - 1) / BM : (p.H + 2 * BM - 1) / (2 * BM);
+  const int nb_shared = MODE == kGateUp ? (p.Is + BM - 1) / BM : (p.H + 2 * BM - 1) / (2 * BM);
+  for (int g = threadIdx.x; g < n_groups; g += blockDim.x) {
+    int e = -1, m = 0, tiles = 0;
+    int64_t r0 = 0;
+    if (g < n_act) {
+      e = p.active[g];
+      if (e >= 0 && e < p.E) {
+        const int64_t lo = p.offsets[e], hi = p.offsets[e + 1];
+        if (lo >= 0 && hi <= R && hi >= lo) {
+          r0 = lo;
+          m = (int)(hi - lo);
+          tiles = nb_routed * ((m + BN - 1) / BN);
+        } else if (blockIdx.x == 0) {
+          record_error(p.hdr, MOE_ERR_DEVICE_CHECK, e);
+        }
+      } else if (blockIdx.x == 0) {
+        record_error(p.hdr, MOE_ERR_DEVICE_CHECK, g);
+      }
+      if (e < 0 || e >= p.E) e = 0;  // zero tiles; keep the id in range
+    } else {
+      m = (int)p.T;
+      tiles = nb_shared * ((m + BN - 1) / BN);
+    }
+    s_e[g] = e;
+    s_m[g] = m;
+    s_r0[g] = (int)r0;
+    pre[g + 1] = tiles;
+  }
+  __syncthreads();
+  if (warp == 0) {  // inclusive scan of pre[1..n_groups] by one warp, in chunks
+    const int per = (n_groups + 31) / 32;
+    const int beg = 1 + lane * per;
+    const int end = min(beg + per, n_groups + 1);
+    int sum = 0;
+    for (int i = beg; i < end; ++i) sum += pre[i];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int i = beg; i < end; ++i) {
+      run += pre[i];
+      pre[i] = run;
+    }
+    if (lane == 0) pre[0] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int total_tiles = n_groups > 0 ? pre[n_groups] : 0;
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+        const CUtensorMap* mA = t.shared ? &mapA_s : &mapA_r;
+        const CUtensorMap* mB = t.shared ? &mapB_s : &mapB_r;
+        const CUtensorMap* mB2 = t.shared ? &mapB2_s : &mapB2_r;
+        for (int kb = 0; kb < t.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bar(&empty[s], ph ^ 1u, abort_flag, p.hdr, 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = stages + (size_t)s * L::kStage;
+          mbar_expect_tx(&full[s], L::kStage);
+          tma_load_2d(mA, &full[s], st, kb * BK, t.a0_row);
+          tma_load_2d(mA, &full[s], st + L::kA, kb * BK, t.a1_row);
+          tma_load_2d(mB, &full[s], st + 2 * L::kA, kb * BK, t.b_row);
+          if (NB == 2) tma_load_2d(mB2, &full[s], st + 2 * L::kA + L::kB, kb * BK, t.b_row);
+        }
+      }
+      // drain: the copies of the last STAGES iterations must have landed
+      for (int j = max(0, it - STAGES); j < it; ++j) drain_bar(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tcount) {
+        const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+        const int a = tcount & 1;
+        const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+        if (!wait_bar(&tempty[a], tph ^ 1u, abort_flag, p.hdr, 2)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(a * 2 * BN);
+        const uint32_t d1 = d0 + BN;
+        for (int kb = 0; kb < t.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bar(&full[s], ph, abort_flag, p.hdr, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa0 = smem_addr(stages + (size_t)s * L::kStage);
+          const uint32_t sa1 = sa0 + L::kA;
+          const uint32_t sb = sa0 + 2 * L::kA;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t bdesc = sw128_desc(sb + kk * 32);
+            const uint64_t adesc0 = sw128_desc(sa0 + kk * 32), adesc1 = sw128_desc(sa1 + kk * 32);
+            umma_bf16(d0, adesc0, bdesc, kIdesc, acc);
+            umma_bf16(d1, adesc1, bdesc, kIdesc, acc);
+            if (NB == 2) {
+              const uint64_t bdesc2 = sw128_desc(sb + L::kB + kk * 32);
+              umma_bf16(d0, adesc0, bdesc2, kIdesc, 1u);
+              umma_bf16(d1, adesc1, bdesc2, kIdesc, 1u);
+            }
+          }
+          tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        tc_commit(&tfull[a]);  // accumulators ready for the epilogue
+      }
+      tc_commit(done);
+      drain_bar(done, 0);
+    }
+  } else {
+    // ======================= epilogue (warps 2..5) =======================
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tcount) {
+      const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+      const int a = tcount & 1;
+      const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+      // one lane waits, the warp follows its verdict: the TMEM loads below are
+      // .sync.aligned and need the whole warp converged
+      int ok = 1;
+      if (lane == 0) ok = wait_bar(&tfull[a], tph, abort_flag, p.hdr, 4) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * BN);
+      const int mvalid = min(BN, t.m - t.mb * BN);
+      for (int c0 = 0; c0 < mvalid; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(taddr + c0, v0);
+        tmem_ld16(taddr + BN + c0, v1);
+        if (MODE == kGateUp) {
+          const int j = t.nb * BM + row;
+          const int width = t.shared ? p.Is : p.I;
+          if (j < width) {
+            uint16_t* hi = t.shared ? p.h_shared : p.h_perm + t.r0 * p.I;
+            const int64_t plane = t.shared ? p.T * p.Is : p.T * p.k * p.I;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = c0 + i;
+              if (c < mvalid) {
+                const float h = silu_f32(v0[i]) * v1[i];
+                const uint16_t h_hi = f32_to_bf16(h);
+                const uint16_t h_lo = f32_to_bf16(h - __uint_as_float((uint32_t)h_hi << 16));
+                const int64_t at = ((int64_t)t.mb * BN + c) * width + j;
+                hi[at] = h_hi;
+                hi[plane + at] = h_lo;
+              }
+            }
+          }
+        } else {
+          const int n0 = t.nb * 2 * BM + row;
+          const int n1 = n0 + BM;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = c0 + i;
+            if (c < mvalid) {
+              const int64_t tok_row = (int64_t)t.mb * BN + c;
+              float* out;
+              float w = 1.0f;
+              if (t.shared) {
+                out = p.shared_out + tok_row * p.H;
+              } else {
+                const int64_t slot = p.tok_of[t.r0 + tok_row];
+                if (slot < 0 || slot >= R) {
+                  record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tok_row));
+                  continue;
+                }
+                if (p.topk_w != nullptr) w = p.topk_w[slot];
+                out = p.y_slots + slot * p.H;
+              }
+              if (n0 < p.H) out[n0] = w * v0[i];
+              if (n1 < p.H) out[n1] = w * v1[i];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous), box {64 cols, box_rows}, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int MODE>
+cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel_id, cudaStream_t s) {
+  constexpr int NB = MODE == kDown ? 2 : 1;
+  const size_t smem = Smem<BN, STAGES, NB>::kTotal;
+  static_assert(Smem<BN, STAGES, NB>::kTotal <= 232448, "shared memory over the 227 KB limit");
+  cudaError_t e = cudaFuncSetAttribute(umma_ffn_kernel<BN, STAGES, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  before_launch(kernel_id, s);
+  umma_ffn_kernel<BN, STAGES, MODE>
+      <<<sm_count(), kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  after_launch(kernel_id, s);
+  return cudaGetLastError();
+}
+
+// Stage counts: gate/up stages hold A0, A1 and one token tile; down stages a
+// second token tile (the h_lo plane).
+template <int BN, int ST_GU, int ST_DN>
+cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
+  const int64_t R = a.T * a.k;
+  const bool shared = a.ws_gate_up != nullptr;
+  UmmaParams p{};
+  p.T = a.T;
+  p.H = a.H;
+  p.I = a.I;
+  p.Is = a.Is;
+  p.k = a.k;
+  p.E = a.E;
+  p.has_shared = shared ? 1 : 0;
+  p.offsets = a.offsets;
+  p.tok_of = a.tok_of;
+  p.active = a.active;
+  p.hdr = a.hdr;
+  p.topk_w = a.topk_w;
+  p.h_perm = static_cast<uint16_t*>(a.h_perm);
+  p.h_shared = static_cast<uint16_t*>(a.h_shared);
+  p.y_slots = a.y_slots;
+  p.shared_out = a.shared_out;
+  // maps: A routed, B routed, B2 routed, A shared, B shared, B2 shared
+  CUtensorMap m[6];
+
+  // pass 1: gate/up with SwiGLU
+  bool ok = make_map(&m[0], a.w_gate_up, (int64_t)a.E * 2 * a.I, a.H, BM) && make_map(&m[1], x_perm, R, a.H, BN);
+  m[2] = m[1];
+  if (shared) ok = ok && make_map(&m[3], a.ws_gate_up, 2 * (int64_t)a.Is, a.H, BM) && make_map(&m[4], a.x, a.T, a.H, BN);
+  else {
+    m[3] = m[0];
+    m[4] = m[1];
+  }
+  m[5] = m[4];
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = launch_pass<BN, ST_GU, kGateUp>(m, p, MOE_KERNEL_EXPERT_GATE_UP, s);
+  if (e != cudaSuccess) return e;
+
+  // pass 2: down projection of h_hi + h_lo, weighted scatter into slot order
+  ok = make_map(&m[0], a.w_down, (int64_t)a.E * a.H, a.I, BM) && make_map(&m[1], p.h_perm, R, a.I, BN) &&
+       make_map(&m[2], p.h_perm + R * a.I, R, a.I, BN);
+  if (shared)
+    ok = ok && make_map(&m[3], a.ws_down, a.H, a.Is, BM) && make_map(&m[4], p.h_shared, a.T, a.Is, BN) &&
+         make_map(&m[5], p.h_shared + a.T * a.Is, a.T, a.Is, BN);
+  else {
+    m[3] = m[0];
+    m[4] = m[1];
+    m[5] = m[2];
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  return launch_pass<BN, ST_DN, kDown>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
+}
+
+}  // namespace
+
+int umma_pick_bn(int64_t T, int k, int E) {
+  const int64_t R = T * k;
+  const int64_t groups = R < E ? R : E;
+  const int64_t avg = groups > 0 ? (R + groups - 1) / groups : 1;
+  if (avg <= 24) return 32;
+  if (avg <= 64) return 64;
+  return 128;
+}
+
+cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cudaStream_t s) {
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  switch (bn) {
+    case 32: return run_bn<32, 5, 5>(a, x_perm, s);
+    case 64: return run_bn<64, 5, 4>(a, x_perm, s);
+    default: return run_bn<128, 4, 3>(a, x_perm, s);
+  }
+}
+
+}  // namespace moe

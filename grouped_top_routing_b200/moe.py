@@ -24,7 +24,8 @@ KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "e
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
-           "moe_launch_count", "moe_last_error")
+           "moe_set_ffn_path", "moe_launch_count", "moe_last_error")
+FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 
 
 class MoeError(RuntimeError):
@@ -78,6 +79,7 @@ def _load():
         "moe_forward": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_check_device": (st, [vp, sz, vp]),
         "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
+        "moe_set_ffn_path": (st, [ctypes.c_int32]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -188,9 +190,9 @@ def moe_expert_ffn(cfg, x, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws
     T = x.shape[0]
     k, H = c.num_experts_per_tok, c.hidden_size
     if y_slots is None:
-        y_slots = torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
+        y_slots = torch.empty((T * k, H), dtype=torch.float32, device=x.device)
     if ws_gate_up is not None and shared_out is None:
-        shared_out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+        shared_out = torch.empty((T, H), dtype=torch.float32, device=x.device)
     _check(lib.moe_expert_ffn(ctypes.byref(c), T, _p(x), _p(x_perm), _p(expert_offsets), _p(tok_of), _p(topk_w),
                               _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y_slots), _p(shared_out),
                               ws.cptr, ws.nbytes, _stream(stream)))
@@ -222,6 +224,11 @@ def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws
     if return_routing:
         return y, idx, w
     return y
+
+
+def set_ffn_path(path: str = "auto"):
+    """Expert-FFN kernels for later calls: "auto", "streaming" or "tensor_cores"."""
+    _check(lib.moe_set_ffn_path(FFN_PATHS[path]))
 
 
 def set_kernel_timer(kernel: str, ev_start=None, ev_stop=None):

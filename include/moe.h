@@ -152,27 +152,28 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T
 
 /* Routed SwiGLU experts and the shared MLP ([ARCH], [SHARED], [GGUF]):
  *   F_e(v) = down_e( silu(gate_e v) * up_e v ),   silu(z) = z / (1 + exp(-z)),
- * fp32 accumulation, the SwiGLU product rounded to bf16 before the down
- * projection. Only experts with rows in expert_offsets are read.
- *   y_slots[t*k + j] = bf16( topk_w[t*k + j] * F_{e}(x_t) )  for the expert e
+ * fp32 accumulation. The SwiGLU product stays fp32 on the streaming (decode)
+ * path and is rounded to bf16 on the tensor-core path, whose MMA operands are
+ * bf16. Only experts with rows in expert_offsets are read.
+ *   y_slots[t*k + j] = topk_w[t*k + j] * F_{e}(x_t)  (fp32) for the expert e
  *                      holding that slot (topk_w NULL: weight 1);
- *   shared_out[t]    = bf16( F_shared(x_t) )  (when ws_gate_up is not NULL).
+ *   shared_out[t]    = F_shared(x_t)  (fp32; when ws_gate_up is not NULL).
  * x [T,H]; x_perm [T*k,H] from moe_permute, or NULL (rows are then gathered
  * from x through tok_of); expert_offsets [E+1], tok_of [T*k] from moe_permute;
- * y_slots [T*k,H] bf16 out; shared_out [T,H] bf16 out or NULL. */
+ * y_slots [T*k,H] fp32 out; shared_out [T,H] fp32 out or NULL. */
 moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, const uint16_t* x_perm,
                           const int32_t* expert_offsets, const int32_t* tok_of, const float* topk_w,
                           const uint16_t* w_gate_up, const uint16_t* w_down,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down,
-                          uint16_t* y_slots, uint16_t* shared_out,
+                          float* y_slots, float* shared_out,
                           void* ws, size_t ws_bytes, void* stream);
 
 /* Weighted combine ([ROUTER], [SHARED]: out = routed mixture + shared(x)):
- *   y[t] = bf16( sum_{j<k} float(y_slots[t*k + j]) + float(shared_out[t]) ),
- * summed in fp32 in slot order then the shared row: deterministic.
- * y_slots [T*k,H] bf16 (already weighted); shared_out [T,H] bf16 or NULL;
+ *   y[t] = bf16( sum_{j<k} y_slots[t*k + j] + shared_out[t] ),
+ * summed in fp32 in slot order then the shared row, rounded once: deterministic.
+ * y_slots [T*k,H] fp32 (already weighted); shared_out [T,H] fp32 or NULL;
  * y [T,H] bf16 out. */
-moe_status moe_combine(const moe_config* cfg, int64_t T, const uint16_t* y_slots, const uint16_t* shared_out,
+moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, const float* shared_out,
                        uint16_t* y, void* stream);
 
 /* The whole block: router logits -> route -> permute -> experts -> combine.
@@ -197,6 +198,12 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
  * (events are cudaEvent_t passed as void*; the caller owns them). Passing NULL
  * events clears the hook. Not thread-safe with concurrent launches. */
 moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop);
+
+/* Selects the expert-FFN kernels for every later call in this process:
+ * 0 = automatic (tensor cores once T*k >= 2*E, i.e. experts average two or
+ * more rows; the streaming GEMV below that), 1 = always the streaming GEMV,
+ * 2 = always the tensor-core grouped GEMM. Both compute the same block. */
+moe_status moe_set_ffn_path(int32_t path);
 
 /* Number of this library's kernel launches since load (host-side counter). */
 uint64_t moe_launch_count(void);

@@ -165,25 +165,23 @@ def test_permute_rejects_bad_ids_on_device(M):
 
 
 def test_combine_definition(M):
-    # y[t] = bf16(sum_j float(y_slots[t*k+j]) + float(shared[t])), fp32, slot order
+    # y[t] = bf16(sum_j y_slots[t*k+j] + shared[t]), fp32 in slot order, one rounding
     T, k, H = 37, 6, 256
     g = torch.Generator().manual_seed(3)
-    ys = torch.randn((T * k, H), generator=g).to(torch.bfloat16)
-    sh = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    ys = torch.randn((T * k, H), generator=g)
+    sh = torch.randn((T, H), generator=g)
     wl = G.tiny_workload(hidden_size=H, num_experts=8, num_experts_per_tok=k)
-    y = M.moe_combine(wl, ys.to(DEV), sh.to(DEV), T).cpu()
+    f = ys.numpy().reshape(T, k, H)
     acc = np.zeros((T, H), np.float32)
-    f = ys.float().numpy().reshape(T, k, H)
     for j in range(k):
         acc = (acc + f[:, j]).astype(np.float32)
-    acc = (acc + sh.float().numpy()).astype(np.float32)
+    ref0 = torch.from_numpy(acc.copy()).to(torch.bfloat16)
+    acc = (acc + sh.numpy()).astype(np.float32)
     ref = torch.from_numpy(acc).to(torch.bfloat16)
+    y = M.moe_combine(wl, ys.to(DEV), sh.to(DEV), T).cpu()
     assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
     y0 = M.moe_combine(wl, ys.to(DEV), None, T).cpu()
-    acc0 = np.zeros((T, H), np.float32)
-    for j in range(k):
-        acc0 = (acc0 + f[:, j]).astype(np.float32)
-    assert torch.equal(y0.view(torch.int16), torch.from_numpy(acc0).to(torch.bfloat16).view(torch.int16))
+    assert torch.equal(y0.view(torch.int16), ref0.view(torch.int16))
 
 
 FFN_CASES = [
@@ -196,8 +194,15 @@ FFN_CASES = [
 ]
 
 
+@pytest.fixture(params=["streaming", "tensor_cores"])
+def path(request, M):
+    M.set_ffn_path(request.param)
+    yield request.param
+    M.set_ffn_path("auto")
+
+
 @pytest.mark.parametrize("name,over", FFN_CASES, ids=[c[0] for c in FFN_CASES])
-def test_expert_ffn(M, name, over):
+def test_expert_ffn(M, name, over, path):
     if name.startswith("tiny"):
         wl = G.tiny_workload(**over)
         inp = S.inputs_to(G.make_inputs(wl, seed=0, device="cpu"), DEV)
@@ -221,10 +226,10 @@ def test_expert_ffn(M, name, over):
         t_sel, j_sel = np.nonzero(idx == e)
         Wg, Wu, Wd = O.expert_weights_f64(inp["w_gate_up"], inp["w_down"], int(e), I)
         ref[t_sel * k + j_sel] = w[t_sel, j_sel][:, None].astype(np.float64) * O.swiglu_mlp(X[t_sel], Wg, Wu, Wd)
-    S.compare(O.as_f64(y_slots), ref, f"{name} y_slots")
+    S.compare(O.as_f64(y_slots), ref, f"{name} [{path}] y_slots")
     if has_shared:
         Wg, Wu, Wd = O.shared_weights_f64(inp["ws_gate_up"], inp["ws_down"])
-        S.compare(O.as_f64(shared), O.swiglu_mlp(X, Wg, Wu, Wd), f"{name} shared")
+        S.compare(O.as_f64(shared), O.swiglu_mlp(X, Wg, Wu, Wd), f"{name} [{path}] shared")
 
 
 # ---------------------------------------------------------------------------
@@ -277,9 +282,9 @@ FORWARD_CASES = [
 
 
 @pytest.mark.parametrize("name,over", FORWARD_CASES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(FORWARD_CASES)])
-def test_forward_matches_oracle(M, name, over):
+def test_forward_matches_oracle(M, name, over, path):
     wl, inp = _inputs(name)
-    wl = dict(wl, **over, name=name)
+    wl = dict(wl, **over, name=f"{name}[{path}]")
     _forward_and_compare(M, wl, inp)
 
 
@@ -298,11 +303,13 @@ def test_forward_prefill_sampled(M, name):
     _forward_and_compare(M, dict(wl, name=name), inp, tokens=rows)
 
 
-def test_forward_skew_ties_sampled(M):
+@pytest.mark.parametrize("over", [{}, dict(norm_topk_prob=False, routed_scaling_factor=1.0)])
+def test_forward_skew_ties_sampled(M, over):
     wl, inp = _inputs("ling30_flash_skew_t16384")
+    wl = dict(wl, **over)
     T, E, k = inp["tokens"], wl["num_experts"], wl["num_experts_per_tok"]
     bias = _np_bias(inp)
-    L = O.router_logits(inp["x"], inp["router_w"]) if False else G.random_logits(T, E, S.logit_std(wl), seed=2).numpy()
+    L = G.random_logits(T, E, S.logit_std(wl), seed=2).numpy()
     toks, pairs = S.add_exact_ties(L, bias, k)
     S.check_ties_constructed(L, bias, wl, toks, pairs)
     rows = np.unique(np.concatenate([toks[:12], np.linspace(0, T - 1, 36).astype(int)]))
