@@ -63,16 +63,20 @@ def peaks():
 # ---------------------------------------------------------------------------
 
 def algorithmic(wl, T, n_unique):
-    """Bytes and flops the block must move / perform once, given the number of
-    distinct routed experts the batch touched."""
+    """Bytes each expert pass must move, and the block's flops, given the
+    number of distinct routed experts the batch touched. Activations count at
+    the width this design stores them: token rows bf16 (2 B), the SwiGLU
+    product as two bf16 planes (4 B), expert slot rows and the shared MLP
+    output fp32 (4 B)."""
     H, E, k, I, Is = (wl["hidden_size"], wl["num_experts"], wl["num_experts_per_tok"],
                       wl["moe_intermediate_size"], wl["shared_width"])
     R = T * k
     w_gate_up = (n_unique * 2 * I + 2 * Is) * H * 2
     w_down = (n_unique * I + Is) * H * 2
-    gate_up_bytes = w_gate_up + (R + T) * H * 2 + (R * I + T * Is) * 2   # weights + x rows in + h out
-    down_bytes = w_down + (R * I + T * Is) * 2 + (R + T) * H * 2          # weights + h in + rows out
-    step_bytes = (w_gate_up + w_down + E * H * 4 + 2 * T * H * 2)         # weights + router + x in + y out
+    h_elems = R * I + T * Is
+    gate_up_bytes = w_gate_up + (R + T) * H * 2 + h_elems * 4   # weights + token rows in + h planes out
+    down_bytes = w_down + h_elems * 4 + (R + T) * H * 4          # weights + h planes in + fp32 rows out
+    step_bytes = (w_gate_up + w_down + E * H * 4 + 2 * T * H * 2)  # weights + router + x in + y out
     flops = R * 6 * H * I + T * 6 * H * Is + 2 * T * H * E
     return dict(gate_up_bytes=gate_up_bytes, down_bytes=down_bytes, step_bytes=step_bytes, flops=flops)
 

@@ -16,8 +16,11 @@
 
 namespace moe {
 
-cudaError_t launch_router_logits(const moe_config& c, const uint16_t* x, int64_t T, const float* w, float* out,
-                                 cudaStream_t s);
+cudaError_t launch_router_logits_gemv(const moe_config& c, const uint16_t* x, int64_t T, const float* w, float* out,
+                                      cudaStream_t s);
+void logits_split(int64_t T, int E, int H, int* ksplit, int* kper);
+cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int64_t T, const float* w,
+                                    float* logits, uint16_t* planes, float* partials, cudaStream_t s);
 cudaError_t launch_route(const moe_config& c, const float* logits, const float* bias, int64_t T, int32_t* idx,
                          float* w, cudaStream_t s);
 size_t permute_scratch_ints(int E, int64_t T);
@@ -169,12 +172,34 @@ moe_status check_ptr(const char* name, const void* p, size_t align, bool require
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
+constexpr int64_t kLogitsGemvMaxT = 16;  // larger batches: router logits on the tensor cores
+
 struct Layout {
-  size_t hdr, logits, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
+  size_t hdr, logits, wr_planes, logit_parts, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
   size_t x_perm, h_perm, h_shared, y_slots, shared_out, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Split-K partial sums of the router logits: the largest need of any token
+// count up to T (a smaller batch can split K more ways), so that a workspace
+// sized for T serves every smaller call.
+size_t logit_partial_bytes(const moe_config& c, int64_t T) {
+  size_t best = 0;
+  auto need = [&](int64_t t) {
+    if (t <= kLogitsGemvMaxT) return;
+    int ksplit = 1, kper = 1;
+    logits_split(t, c.num_experts, c.hidden_size, &ksplit, &kper);
+    if (ksplit > 1) {
+      const size_t b = (size_t)ksplit * t * c.num_experts * 4;
+      if (b > best) best = b;
+    }
+  };
+  need(T);
+  for (int64_t t = 128; t <= T && t <= 128 * 256; t += 128) need(t);  // splits change only at 128-token steps
+  need(kLogitsGemvMaxT + 1 <= T ? kLogitsGemvMaxT + 1 : 0);
+  return best;
+}
 
 Layout layout(const moe_config& c, int64_t max_tokens) {
   const int64_t T = max_tokens > 0 ? max_tokens : 1;
@@ -190,6 +215,8 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   };
   L.hdr = take(sizeof(WsHeader));
   L.logits = take((size_t)T * E * 4);
+  L.wr_planes = take(T > kLogitsGemvMaxT ? (size_t)3 * E * H * 2 : 0);
+  L.logit_parts = take(logit_partial_bytes(c, T));
   L.topk_idx = take((size_t)R * 4);
   L.topk_w = take((size_t)R * 4);
   L.offsets = take((size_t)(E + 1) * 4);
@@ -222,6 +249,19 @@ moe_status check_ws(const moe_config& c, int64_t T, void* ws, size_t ws_bytes) {
 }
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+moe_status run_logits(const moe_config& c, const uint16_t* x, int64_t T, const float* w, float* out, void* ws,
+                      cudaStream_t s) {
+  cudaError_t e;
+  if (T <= kLogitsGemvMaxT) {
+    e = launch_router_logits_gemv(c, x, T, w, out, s);
+  } else {
+    const Layout L = layout(c, T);
+    e = launch_router_logits_tc(c, x, T, w, out, at<uint16_t>(ws, L.wr_planes), at<float>(ws, L.logit_parts), s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "router logits");
+  return MOE_OK;
+}
 
 // Tensor cores once experts average at least two rows; below that (decode)
 // the streaming GEMV spreads the weight rows over every SM.
@@ -306,16 +346,15 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 }
 
 moe_status moe_router_logits(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
-                             float* logits, void* stream) {
+                             float* logits, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
   MOE_TRY(check_ptr("x", x, 16, true));
   MOE_TRY(check_ptr("router_w", router_w, 16, true));
-  MOE_TRY(check_ptr("logits", logits, 4, true));
-  cudaError_t e = launch_router_logits(*cfg, x, T, router_w, logits, as_stream(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "router logits");
-  return MOE_OK;
+  MOE_TRY(check_ptr("logits", logits, 16, true));
+  return run_logits(*cfg, x, T, router_w, logits, ws, as_stream(stream));
 }
 
 moe_status moe_route(const moe_config* cfg, const float* logits, const float* expert_bias, int64_t T,
@@ -433,8 +472,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   cudaError_t e;
   if (logits == nullptr) {
     float* lg = at<float>(ws, L.logits);
-    e = launch_router_logits(c, x, T, router_w, lg, s);
-    if (e != cudaSuccess) return cuda_fail(e, "router logits");
+    MOE_TRY(run_logits(c, x, T, router_w, lg, ws, s));
     logits = lg;
   }
   int32_t* idx = topk_idx_out != nullptr ? topk_idx_out : at<int32_t>(ws, L.topk_idx);

@@ -12,17 +12,19 @@
 //
 //   pass GATE_UP: D0 = W_gate[n0:n0+128] . X^T, D1 = W_up[n0:n0+128] . X^T,
 //                 h[token, n0+i] = silu(D0[i]) * D1[i]  -> (h_hi, h_lo)
-//   pass DOWN   : D0 = W_down[n0:n0+128] . H^T, D1 = W_down[n0+128:n0+256] . H^T,
-//                 y_slots[slot(token), n] = w_slot * D[n]  (fp32; shared MLP: weight 1)
+//   pass DOWN   : D = W_down[n0:n0+128] . [H_hi | H_lo]^T   (one MMA of N = 2 BN),
+//                 y_slots[slot(token), n] = w_slot * (D_hi[n] + D_lo[n])
+//                 (fp32; shared MLP: weight 1)
 //
-// h is written as two bf16 planes, h_hi = bf16(h) and h_lo = bf16(h - h_hi),
-// and the DOWN pass accumulates W.h_hi + W.h_lo from the same weight tile: the
-// SwiGLU product then carries ~16 significant bits into the down projection
-// instead of bf16's 8, at the cost of a second MMA per weight tile (no extra
-// weight bytes).
+// h is written as two bf16 planes, h_hi = bf16(h) and h_lo = bf16(h - h_hi).
+// The DOWN stage holds the token tile of each plane back to back, so the pair
+// is a single B operand of 2 BN rows: one MMA per weight tile yields both
+// W.h_hi and W.h_lo, which the epilogue adds. The SwiGLU product thus carries
+// ~16 significant bits into the down projection, with no extra weight bytes
+// and no extra MMA instructions.
 //
 // Persistent, warp-specialised CTA (one per SM, 192 threads):
-//   warp 0      : TMA producer (one lane), STAGES-deep ring of (A0, A1, B) tiles
+//   warp 0      : TMA producer (one lane), STAGES-deep ring of weight and token tiles
 //   warp 1      : TMEM allocator; one lane issues tcgen05.mma, commits to barriers
 //   warps 2..5  : epilogue; TMEM -> registers (tcgen05.ld), SwiGLU / weighting, stores
 // The two TMEM accumulator pairs are double-buffered so the epilogue of one tile
@@ -49,7 +51,13 @@ constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1025;  // routed experts (<= 1024) + the shared MLP
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum : int { kGateUp = 0, kDown = 1 };
+enum : int { kGateUp = 0, kDown = 1, kLogits = 2 };
+constexpr int kLogitsBN = 128;
+// The router-logits GEMM accumulates at most this many k-blocks (32 MMAs of
+// K = 16) in one TMEM accumulator; the epilogue adds the chunk sums into the
+// output in fp32. Long tensor-core accumulation chains drift (measured: error
+// grows with the chain length), short ones stay within a few fp32 ulps.
+constexpr int kLogitsChunk = 8;
 
 struct UmmaParams {
   int64_t T;
@@ -64,6 +72,9 @@ struct UmmaParams {
   uint16_t* h_shared;  // hi plane [T, Is], lo plane follows
   float* y_slots;
   float* shared_out;
+  // router-logits mode: A = the three bf16 planes of the router weight [3E, H]
+  float* logits_out;  // [ksplit, T, E] partial sums (ksplit == 1: the logits)
+  int ksplit, kper, kbH;
 };
 
 // ----------------------------------------------------------------------------
@@ -196,11 +207,26 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
 // ----------------------------------------------------------------------------
 // tile schedule
 // ----------------------------------------------------------------------------
+// Stage = NA weight tiles (128 x 64) then NB token tiles (BN x 64), all
+// 1024-byte aligned. GATE_UP / LOGITS: NA = 2, NB = 1 (gate and up rows, or
+// two blocks of router rows, share the token tile). DOWN: NB = 2 (the h_hi and
+// h_lo token tiles, one B operand of 2 BN rows) and NA = 2 while the TMEM
+// budget allows (BN <= 64), else 1. Each accumulator is NCOL columns.
+template <int BN, int MODE>
+struct Shape {
+  static constexpr int NA = (MODE == kDown && BN > 64) ? 1 : 2;
+  static constexpr int NB = MODE == kDown ? 2 : 1;
+  static constexpr int NCOL = MODE == kDown ? 2 * BN : BN;
+  static constexpr int ROWS = NA * BM;                 // weight rows per DOWN / LOGITS tile
+  static constexpr uint32_t kTmemCols = 2 * NA * NCOL; // two buffers
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM allocation");
+};
+
 struct TileInfo {
   bool shared;
-  int e, m, nb, mb;
+  int e, m, nb, mb, ks;
   int64_t r0;
-  int a0_row, a1_row, b_row, kblocks;
+  int a0_row, a1_row, b_row, kb0, kblocks, nchunks;
 };
 
 template <int BN, int MODE>
@@ -219,6 +245,21 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
   t.r0 = s_r0[lo];
   const int mblocks = (t.m + BN - 1) / BN;
   const int local = tile - pre[lo];
+  t.kb0 = 0;
+  t.ks = 0;
+  if (MODE == kLogits) {  // one group (all tokens); split-K index fastest
+    t.ks = local % p.ksplit;
+    const int rest = local / p.ksplit;
+    t.nb = rest / mblocks;
+    t.mb = rest - t.nb * mblocks;
+    t.a0_row = t.nb * 2 * BM;
+    t.a1_row = t.a0_row + BM;
+    t.b_row = t.mb * BN;
+    t.kb0 = t.ks * p.kper;
+    t.kblocks = min(p.kper, 3 * p.kbH - t.kb0);
+    t.nchunks = (t.kblocks + kLogitsChunk - 1) / kLogitsChunk;
+    return t;
+  }
   t.nb = local / mblocks;
   t.mb = local - t.nb * mblocks;
   int K;
@@ -233,19 +274,23 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
     }
   } else {
     K = t.shared ? p.Is : p.I;
-    t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * 2 * BM;
-    t.a1_row = t.a0_row + BM;
+    t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * Shape<BN, MODE>::ROWS;
+    t.a1_row = t.a0_row + BM;  // used when the stage holds two weight tiles
   }
   t.b_row = (int)t.r0 + t.mb * BN;
   t.kblocks = (K + BK - 1) / BK;
+  t.nchunks = 1;
   return t;
 }
 
-template <int BN, int STAGES, int NB>
+// Shared-memory carve-up of one CTA.
+template <int BN, int STAGES, int MODE>
 struct Smem {
+  static constexpr int NA = Shape<BN, MODE>::NA;
+  static constexpr int NB = Shape<BN, MODE>::NB;
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = BN * BK * 2;
-  static constexpr int kStage = 2 * kA + NB * kB;
+  static constexpr int kStage = NA * kA + NB * kB;
   static constexpr int kBarriers = (2 * STAGES + 5) * 8;
   static constexpr int kTables = 4 * (kMaxGroups + 1) * 4;
   static constexpr size_t kTotal = 1024 + (size_t)STAGES * kStage + kBarriers + 16 + kTables;
@@ -257,10 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap mapB2_r, const __grid_constant__ CUtensorMap mapA_s,
                     const __grid_constant__ CUtensorMap mapB_s, const __grid_constant__ CUtensorMap mapB2_s,
                     const UmmaParams p) {
-  constexpr int NB = MODE == kDown ? 2 : 1;  // DOWN reads the h_hi and h_lo planes
-  using L = Smem<BN, STAGES, NB>;
-  constexpr uint32_t kTmemCols = 4 * BN;  // two buffers x (D0, D1)
+  using L = Smem<BN, STAGES, MODE>;
+  using SH = Shape<BN, MODE>;
+  constexpr uint32_t kTmemCols = SH::kTmemCols;
   constexpr uint32_t kIdesc = idesc_bf16<BN>();
+  constexpr uint32_t kIdescDown = idesc_bf16<(2 * BN <= 256 ? 2 * BN : 256)>();
+  static_assert(MODE != kDown || 2 * BN <= 256, "DOWN issues N = 2 BN <= 256");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -294,11 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
 
   // ---- group table: active experts (+ shared MLP), tiles per group ----
-  const int n_act = min(max(*(volatile int*)&p.hdr->num_active, 0), p.E);
-  const int n_groups = n_act + (p.has_shared ? 1 : 0);
+  const int n_act = MODE == kLogits ? 0 : min(max(*(volatile int*)&p.hdr->num_active, 0), p.E);
+  const int n_groups = MODE == kLogits ? 1 : n_act + (p.has_shared ? 1 : 0);
   const int64_t R = p.T * p.k;
-  const int nb_routed = MODE == kGateUp ? (p.I + BM - 1) / BM : (p.H + 2 * BM - 1) / (2 * BM);
-  const int nb_shared = MODE == kGateUp ? (p.Is + BM - 1) / BM : (p.H + 2 * BM - 1) / (2 * BM);
+  const int nb_routed = MODE == kGateUp ? (p.I + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
+  const int nb_shared = MODE == kGateUp ? (p.Is + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
   for (int g = threadIdx.x; g < n_groups; g += blockDim.x) {
     int e = -1, m = 0, tiles = 0;
     int64_t r0 = 0;
@@ -317,6 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         record_error(p.hdr, MOE_ERR_DEVICE_CHECK, g);
       }
       if (e < 0 || e >= p.E) e = 0;  // zero tiles; keep the id in range
+    } else if (MODE == kLogits) {
+      m = (int)p.T;
+      tiles = ((p.E + 2 * BM - 1) / (2 * BM)) * ((m + BN - 1) / BN) * p.ksplit;
     } else {
       m = (int)p.T;
       tiles = nb_shared * ((m + BN - 1) / BN);
@@ -370,11 +420,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = stages + (size_t)s * L::kStage;
+          const int gkb = t.kb0 + kb;
+          int kx = gkb * BK, a0y = t.a0_row, a1y = t.a1_row;
+          if (MODE == kLogits) {  // k-block gkb lies in weight plane gkb / kbH
+            const int piece = gkb / p.kbH;
+            kx = (gkb - piece * p.kbH) * BK;
+            a0y += piece * p.E;
+            a1y += piece * p.E;
+          }
           mbar_expect_tx(&full[s], L::kStage);
-          tma_load_2d(mA, &full[s], st, kb * BK, t.a0_row);
-          tma_load_2d(mA, &full[s], st + L::kA, kb * BK, t.a1_row);
-          tma_load_2d(mB, &full[s], st + 2 * L::kA, kb * BK, t.b_row);
-          if (NB == 2) tma_load_2d(mB2, &full[s], st + 2 * L::kA + L::kB, kb * BK, t.b_row);
+          tma_load_2d(mA, &full[s], st, kx, a0y);
+          if (L::NA == 2) tma_load_2d(mA, &full[s], st + L::kA, kx, a1y);
+          uint8_t* sb = st + L::NA * L::kA;
+          tma_load_2d(mB, &full[s], sb, kx, t.b_row);
+          if (L::NB == 2) tma_load_2d(mB2, &full[s], sb + L::kB, kx, t.b_row);
         }
       }
       // drain: the copies of the last STAGES iterations must have landed
@@ -385,42 +444,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tcount) {
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
-        const int a = tcount & 1;
-        const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
-        if (!wait_bar(&tempty[a], tph ^ 1u, abort_flag, p.hdr, 2)) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem_base + (uint32_t)(a * 2 * BN);
-        const uint32_t d1 = d0 + BN;
-        for (int kb = 0; kb < t.kblocks; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_bar(&full[s], ph, abort_flag, p.hdr, 3)) {
+        for (int ch = 0; ok && ch < t.nchunks; ++ch, ++tcount) {
+          const int a = tcount & 1;
+          const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+          if (!wait_bar(&tempty[a], tph ^ 1u, abort_flag, p.hdr, 2)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa0 = smem_addr(stages + (size_t)s * L::kStage);
-          const uint32_t sa1 = sa0 + L::kA;
-          const uint32_t sb = sa0 + 2 * L::kA;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t bdesc = sw128_desc(sb + kk * 32);
-            const uint64_t adesc0 = sw128_desc(sa0 + kk * 32), adesc1 = sw128_desc(sa1 + kk * 32);
-            umma_bf16(d0, adesc0, bdesc, kIdesc, acc);
-            umma_bf16(d1, adesc1, bdesc, kIdesc, acc);
-            if (NB == 2) {
-              const uint64_t bdesc2 = sw128_desc(sb + L::kB + kk * 32);
-              umma_bf16(d0, adesc0, bdesc2, kIdesc, 1u);
-              umma_bf16(d1, adesc1, bdesc2, kIdesc, 1u);
+          const uint32_t d0 = tmem_base + (uint32_t)(a * SH::NA * SH::NCOL);
+          const uint32_t d1 = d0 + SH::NCOL;
+          const int kb_begin = t.nchunks == 1 ? 0 : ch * kLogitsChunk;
+          const int kb_end = t.nchunks == 1 ? t.kblocks : min(kb_begin + kLogitsChunk, t.kblocks);
+          for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+            if (!wait_bar(&full[s], ph, abort_flag, p.hdr, 3)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t sa0 = smem_addr(stages + (size_t)s * L::kStage);
+            const uint32_t sb = sa0 + L::NA * L::kA;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint32_t acc = (kb > kb_begin || kk > 0) ? 1u : 0u;
+              const uint64_t bdesc = sw128_desc(sb + kk * 32);
+              if (MODE == kDown) {  // B = [h_hi tile; h_lo tile]: 2 BN rows, each D spans 2 BN columns
+                umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdescDown, acc);
+                if (SH::NA == 2) umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescDown, acc);
+              } else {
+                umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdesc, acc);
+                umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdesc, acc);
+              }
+            }
+            tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
           }
-          tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
+          if (!ok) break;
+          tc_commit(&tfull[a]);  // accumulators ready for the epilogue
         }
-        if (!ok) break;
-        tc_commit(&tfull[a]);  // accumulators ready for the epilogue
       }
       tc_commit(done);
       drain_bar(done, 0);
@@ -430,73 +494,103 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tcount) {
+    bool alive = true;
+    for (int tile = blockIdx.x; alive && tile < total_tiles; tile += gridDim.x) {
       const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
-      const int a = tcount & 1;
-      const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
-      // one lane waits, the warp follows its verdict: the TMEM loads below are
-      // .sync.aligned and need the whole warp converged
-      int ok = 1;
-      if (lane == 0) ok = wait_bar(&tfull[a], tph, abort_flag, p.hdr, 4) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * BN);
-      const int mvalid = min(BN, t.m - t.mb * BN);
-      for (int c0 = 0; c0 < mvalid; c0 += 16) {
-        float v0[16], v1[16];
-        tmem_ld16(taddr + c0, v0);
-        tmem_ld16(taddr + BN + c0, v1);
-        if (MODE == kGateUp) {
-          const int j = t.nb * BM + row;
-          const int width = t.shared ? p.Is : p.I;
-          if (j < width) {
-            uint16_t* hi = t.shared ? p.h_shared : p.h_perm + t.r0 * p.I;
-            const int64_t plane = t.shared ? p.T * p.Is : p.T * p.k * p.I;
+      for (int ch = 0; ch < t.nchunks; ++ch, ++tcount) {
+        const int a = tcount & 1;
+        const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+        // one lane waits, the warp follows its verdict: the TMEM loads below are
+        // .sync.aligned and need the whole warp converged
+        int ok = 1;
+        if (lane == 0) ok = wait_bar(&tfull[a], tph, abort_flag, p.hdr, 4) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();
+        if (!ok) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * SH::NA * SH::NCOL);
+        const int mvalid = min(BN, t.m - t.mb * BN);
+        for (int c0 = 0; c0 < mvalid; c0 += 16) {
+          float v0[16], v1[16];
+          if (MODE != kDown) {  // D0 and D1 columns c0 .. c0+15
+            tmem_ld16(taddr + c0, v0);
+            tmem_ld16(taddr + SH::NCOL + c0, v1);
+          }
+          if (MODE == kLogits) {
+            const int e0 = t.nb * 2 * BM + row, e1 = e0 + BM;
+            float* out = p.logits_out + (int64_t)t.ks * p.T * p.E;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = c0 + i;
               if (c < mvalid) {
-                const float h = silu_f32(v0[i]) * v1[i];
-                const uint16_t h_hi = f32_to_bf16(h);
-                const uint16_t h_lo = f32_to_bf16(h - __uint_as_float((uint32_t)h_hi << 16));
-                const int64_t at = ((int64_t)t.mb * BN + c) * width + j;
-                hi[at] = h_hi;
-                hi[plane + at] = h_lo;
+                const int64_t tok = (int64_t)t.mb * BN + c;
+                // chunk 0 stores, later chunks add (each thread owns its elements)
+                if (e0 < p.E) out[tok * p.E + e0] = ch == 0 ? v0[i] : out[tok * p.E + e0] + v0[i];
+                if (e1 < p.E) out[tok * p.E + e1] = ch == 0 ? v1[i] : out[tok * p.E + e1] + v1[i];
               }
             }
-          }
-        } else {
-          const int n0 = t.nb * 2 * BM + row;
-          const int n1 = n0 + BM;
+          } else if (MODE == kGateUp) {
+            const int j = t.nb * BM + row;
+            const int width = t.shared ? p.Is : p.I;
+            if (j < width) {
+              uint16_t* hi = t.shared ? p.h_shared : p.h_perm + t.r0 * p.I;
+              const int64_t plane = t.shared ? p.T * p.Is : p.T * p.k * p.I;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = c0 + i;
-            if (c < mvalid) {
-              const int64_t tok_row = (int64_t)t.mb * BN + c;
-              float* out;
-              float w = 1.0f;
-              if (t.shared) {
-                out = p.shared_out + tok_row * p.H;
-              } else {
-                const int64_t slot = p.tok_of[t.r0 + tok_row];
-                if (slot < 0 || slot >= R) {
-                  record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tok_row));
-                  continue;
+              for (int i = 0; i < 16; ++i) {
+                const int c = c0 + i;
+                if (c < mvalid) {
+                  const float h = silu_f32(v0[i]) * v1[i];
+                  const uint16_t h_hi = f32_to_bf16(h);
+                  const uint16_t h_lo = f32_to_bf16(h - __uint_as_float((uint32_t)h_hi << 16));
+                  const int64_t at = ((int64_t)t.mb * BN + c) * width + j;
+                  hi[at] = h_hi;
+                  hi[plane + at] = h_lo;
                 }
-                if (p.topk_w != nullptr) w = p.topk_w[slot];
-                out = p.y_slots + slot * p.H;
               }
-              if (n0 < p.H) out[n0] = w * v0[i];
-              if (n1 < p.H) out[n1] = w * v1[i];
+            }
+          } else {
+            const int n = t.nb * SH::ROWS + row;
+            // lane i < 16 fetches the slot and routing weight of column c0 + i;
+            // the loop takes them by shuffle: one load round trip per chunk
+            long long my_slot = -1;
+            float my_w = 1.0f;
+            if (lane < 16 && c0 + lane < mvalid) {
+              const int64_t tok_row = (int64_t)t.mb * BN + c0 + lane;
+              if (t.shared) {
+                my_slot = tok_row;
+              } else {
+                my_slot = p.tok_of[t.r0 + tok_row];
+                if (my_slot < 0 || my_slot >= R) {
+                  record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tok_row));
+                  my_slot = -1;
+                } else if (p.topk_w != nullptr) {
+                  my_w = p.topk_w[my_slot];
+                }
+              }
+            }
+            float* base = t.shared ? p.shared_out : p.y_slots;
+#pragma unroll
+            for (int acc_i = 0; acc_i < SH::NA; ++acc_i) {  // accumulator acc_i: weight rows n + acc_i * 128
+              const uint32_t ta = taddr + (uint32_t)(acc_i * SH::NCOL);
+              tmem_ld16(ta + c0, v0);       // W . h_hi
+              tmem_ld16(ta + BN + c0, v1);  // W . h_lo
+              const int nn = n + acc_i * BM;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const long long slot = __shfl_sync(0xffffffffu, my_slot, i);
+                const float w = __shfl_sync(0xffffffffu, my_w, i);
+                if (slot >= 0 && nn < p.H) base[slot * p.H + nn] = w * (v0[i] + v1[i]);
+              }
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[a]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[a]);
     }
   }
 
@@ -543,9 +637,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 
 template <int BN, int STAGES, int MODE>
 cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel_id, cudaStream_t s) {
-  constexpr int NB = MODE == kDown ? 2 : 1;
-  const size_t smem = Smem<BN, STAGES, NB>::kTotal;
-  static_assert(Smem<BN, STAGES, NB>::kTotal <= 232448, "shared memory over the 227 KB limit");
+  const size_t smem = Smem<BN, STAGES, MODE>::kTotal;
+  static_assert(Smem<BN, STAGES, MODE>::kTotal <= 232448, "shared memory over the 227 KB limit");
   cudaError_t e = cudaFuncSetAttribute(umma_ffn_kernel<BN, STAGES, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -556,8 +649,8 @@ cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel
   return cudaGetLastError();
 }
 
-// Stage counts: gate/up stages hold A0, A1 and one token tile; down stages a
-// second token tile (the h_lo plane).
+// Stage counts: gate/up stages hold two weight tiles and one token tile; down
+// stages one weight tile and the token tiles of both h planes.
 template <int BN, int ST_GU, int ST_DN>
 cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   const int64_t R = a.T * a.k;
@@ -610,7 +703,98 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   return launch_pass<BN, ST_DN, kDown>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
 }
 
+// Splits the fp32 router weight into three bf16 planes whose sum is the weight
+// (to within one fp32 ulp): hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid).
+// x is bf16, so every product x * plane is exact in fp32 and the tensor cores
+// accumulate sum_h x[t,h] * w[e,h] over K = 3H in fp32.
+__global__ void __launch_bounds__(256) split_router_weight_kernel(const float* __restrict__ w, int64_t n,
+                                                                  uint16_t* __restrict__ planes) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = __ldg(w + i);
+    const uint16_t hi = f32_to_bf16(v);
+    const float r1 = v - __uint_as_float((uint32_t)hi << 16);
+    const uint16_t mid = f32_to_bf16(r1);
+    const float r2 = r1 - __uint_as_float((uint32_t)mid << 16);
+    planes[i] = hi;
+    planes[n + i] = mid;
+    planes[2 * n + i] = f32_to_bf16(r2);
+  }
+}
+
+// logits[t, e] = sum_s part[s, t, e], s ascending.
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restrict__ part, int ksplit, int64_t n,
+                                                            float* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float acc = part[i];
+    for (int s = 1; s < ksplit; ++s) acc += part[(int64_t)s * n + i];
+    out[i] = acc;
+  }
+}
+
 }  // namespace
+
+// Split-K factor of the router-logits GEMM: enough tiles to cover the SMs when
+// the token count alone does not; every split gets at least one k-block.
+void logits_split(int64_t T, int E, int H, int* ksplit, int* kper) {
+  const int kbH = (H + BK - 1) / BK;
+  const int total = 3 * kbH;
+  const int64_t tiles = (int64_t)((E + 2 * BM - 1) / (2 * BM)) * ((T + kLogitsBN - 1) / kLogitsBN);
+  int want = (int)((128 + tiles - 1) / tiles);
+  want = want < 1 ? 1 : (want > 24 ? 24 : want);
+  if (want > total) want = total;
+  const int per = (total + want - 1) / want;
+  *kper = per;
+  *ksplit = (total + per - 1) / per;
+}
+
+cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int64_t T, const float* w,
+                                    float* logits, uint16_t* planes, float* partials, cudaStream_t s) {
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  const int E = c.num_experts, H = c.hidden_size;
+  const int64_t n = (int64_t)E * H;
+  int ksplit, kper;
+  logits_split(T, E, H, &ksplit, &kper);
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
+  before_launch(MOE_KERNEL_ROUTER_LOGITS, s);
+  split_router_weight_kernel<<<(unsigned)blocks, 256, 0, s>>>(w, n, planes);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  UmmaParams p{};
+  p.T = T;
+  p.H = H;
+  p.E = E;
+  p.k = 1;
+  p.logits_out = ksplit > 1 ? partials : logits;
+  p.ksplit = ksplit;
+  p.kper = kper;
+  p.kbH = (H + BK - 1) / BK;
+  CUtensorMap m[6];
+  if (!make_map(&m[0], planes, 3 * (int64_t)E, H, BM) || !make_map(&m[1], x, T, H, kLogitsBN))
+    return cudaErrorInvalidValue;
+  m[2] = m[1];
+  m[3] = m[0];
+  m[4] = m[1];
+  m[5] = m[1];
+  constexpr int kStages = 4;
+  const size_t smem = Smem<kLogitsBN, kStages, kLogits>::kTotal;
+  e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  umma_ffn_kernel<kLogitsBN, kStages, kLogits><<<sm_count(), kThreads, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int nk = 2;
+  if (ksplit > 1) {
+    const int64_t nl = T * E;
+    int64_t rb = (nl + 255) / 256;
+    if (rb > (int64_t)sm_count() * 8) rb = (int64_t)sm_count() * 8;
+    reduce_splits_kernel<<<(unsigned)rb, 256, 0, s>>>(partials, ksplit, nl, logits);
+    nk = 3;
+  }
+  after_launch(MOE_KERNEL_ROUTER_LOGITS, s, nk);
+  return cudaGetLastError();
+}
 
 int umma_pick_bn(int64_t T, int k, int E) {
   const int64_t R = T * k;
@@ -626,7 +810,7 @@ cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cu
   switch (bn) {
     case 32: return run_bn<32, 5, 5>(a, x_perm, s);
     case 64: return run_bn<64, 5, 4>(a, x_perm, s);
-    default: return run_bn<128, 4, 3>(a, x_perm, s);
+    default: return run_bn<128, 4, 4>(a, x_perm, s);
   }
 }
 

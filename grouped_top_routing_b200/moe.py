@@ -71,7 +71,7 @@ def _load():
     sig = {
         "moe_workspace_size": (sz, [cfgp, i64]),
         "moe_workspace_init": (st, [vp, sz, vp]),
-        "moe_router_logits": (st, [cfgp, vp, i64, vp, vp, vp]),
+        "moe_router_logits": (st, [cfgp, vp, i64, vp, vp, vp, sz, vp]),
         "moe_route": (st, [cfgp, vp, vp, i64, vp, vp, vp]),
         "moe_permute": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_expert_ffn": (st, [cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -149,12 +149,13 @@ class Workspace:
         _check(lib.moe_check_device(self.cptr, self.nbytes, _stream(stream)))
 
 
-def moe_router_logits(cfg, x, router_w, out=None, stream=None):
+def moe_router_logits(cfg, x, router_w, ws: "Workspace", out=None, stream=None):
     c = _as_cfg(cfg)
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, c.num_experts), dtype=torch.float32, device=x.device)
-    _check(lib.moe_router_logits(ctypes.byref(c), _p(x), T, _p(router_w), _p(out), _stream(stream)))
+    _check(lib.moe_router_logits(ctypes.byref(c), _p(x), T, _p(router_w), _p(out), ws.cptr, ws.nbytes,
+                                 _stream(stream)))
     return out
 
 

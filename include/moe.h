@@ -117,9 +117,13 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Router projection ([ROUTER]; router weight mlp.gate [E, H]):
  *   logits[t, e] = sum_h float(x[t, h]) * router_w[e, h]   (fp32 accumulate)
- * x [T,H] bf16, router_w [E,H] fp32, logits [T,E] fp32 out. T may be 0. */
+ * x [T,H] bf16, router_w [E,H] fp32, logits [T,E] fp32 out. T may be 0.
+ * T <= 16: an fp32 streaming GEMV over router_w. Larger T: the tensor cores,
+ * with router_w split exactly into three bf16 planes (hi + mid + lo, to one
+ * fp32 ulp) in the workspace, so every product is exact and the sum is
+ * accumulated in fp32 over K = 3H. ws / ws_bytes >= moe_workspace_size(cfg, T). */
 moe_status moe_router_logits(const moe_config* cfg, const uint16_t* x, int64_t T,
-                             const float* router_w, float* logits, void* stream);
+                             const float* router_w, float* logits, void* ws, size_t ws_bytes, void* stream);
 
 /* Router on fp32 gates ([ROUTER], [ARCH], [LING26]). Per token:
  *   s    = softmax(logits) or sigmoid(logits), each score the fp32 rounding of

@@ -114,12 +114,16 @@ def test_route_bit_exact(M, name, over):
 
 @pytest.mark.parametrize("name,T", [("ling_lite_t64", 64), ("ling26_flash_t512", 512), ("ling30_flash_decode_t1", 1),
                                     ("ling30_flash_decode_t8", 8), ("ling30_flash_decode_t32", 32),
-                                    ("ling26_flash_t512", 77)])
+                                    ("ling26_flash_t512", 77), ("ling30_flash_decode_t8", 16),
+                                    ("ling30_flash_decode_t8", 17), ("ling26_flash_prefill_t8192", 8192),
+                                    ("ling30_flash_skew_t16384", 3000)])
 def test_router_logits(M, name, T):
     wl = G.workload(name)
     inp = G.make_inputs(wl, seed=0, device="cpu", weights=False, tokens=T)
     ref = O.router_logits(inp["x"], inp["router_w"]).astype(np.float64)
-    got = M.moe_router_logits(wl, inp["x"].to(DEV), inp["router_w"].to(DEV)).cpu().numpy().astype(np.float64)
+    ws = M.Workspace(wl, T)
+    got = M.moe_router_logits(wl, inp["x"].to(DEV), inp["router_w"].to(DEV), ws).cpu().numpy().astype(np.float64)
+    ws.check()
     err = np.abs(got - ref).max()
     print(f"{name} T={T}: max |logit - oracle| = {err:.3e}")
     # fp32 accumulation over H terms of size ~0.02: a few 1e-6 typical
