@@ -6,13 +6,14 @@
 // "Shared experts are one wide MLP, not N separate experts"):
 //   h = silu(gate x) * (up x),  y = down h.
 //
-// Work items are single weight rows (gate/up pass) or blocks of kDownRows
-// rows (down pass) of the experts in the compacted active list written by the
+// Work items are single weight rows (gate/up pass) or blocks of ROWS rows
+// (down pass) of the experts in the compacted active list written by the
 // permutation, plus the shared MLP's rows. One warp per item: lanes stride the
 // row in 16-byte chunks (ld.global.nc, no L1 allocation), every token routed
 // to that expert is multiplied against the chunk, and the warp reduces with
-// shuffles. Tokens are taken kTok at a time; an expert with more rows streams
-// its weights again per group of kTok (those re-reads hit L2).
+// shuffles. Tokens are taken MT at a time (MT follows the batch, up to 8); an
+// expert with more rows streams its weights again per group of MT (those
+// re-reads hit L2), which is why larger batches take the tensor-core path.
 #include "common.cuh"
 #include "ffn.cuh"
 
@@ -20,9 +21,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kTok = 8;       // tokens per pass
-constexpr int kUnroll = 4;    // 16-byte chunks in flight per lane per row
-constexpr int kDownRows = 4;  // rows per down-projection item
+constexpr int kUnroll = 4;  // 16-byte chunks in flight per lane per weight row (gate/up pass)
 
 // Resolves the rows [r0, r0 + m) of one active expert, clamped to [0, T*k).
 __device__ __forceinline__ bool expert_rows(const FfnArgs& a, int aidx, int& e, int64_t& r0, int64_t& m) {
@@ -51,6 +50,9 @@ __device__ __forceinline__ int64_t slot_token(const FfnArgs& a, int64_t row, int
   return slot / a.k;
 }
 
+// Gate/up pass: one warp per intermediate index j of one expert, streaming its
+// gate row and up row (H bf16 each) against up to MT tokens per pass.
+template <int MT>
 __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -78,11 +80,11 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
       up = gate + (int64_t)a.Is * H;
       m = a.T;
     }
-    for (int64_t c0 = 0; c0 < m; c0 += kTok) {
-      const int mc = (int)min((int64_t)kTok, m - c0);
-      const uint16_t* xr[kTok];
+    for (int64_t c0 = 0; c0 < m; c0 += MT) {
+      const int mc = (int)min((int64_t)MT, m - c0);
+      const uint16_t* xr[MT];
 #pragma unroll
-      for (int t = 0; t < kTok; ++t) {
+      for (int t = 0; t < MT; ++t) {
         xr[t] = nullptr;
         if (t < mc) {
           int64_t tok = c0 + t, slot;
@@ -90,9 +92,9 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
           if (tok >= 0) xr[t] = a.x + tok * H;
         }
       }
-      float ag[kTok], au[kTok];
+      float ag[MT], au[MT];
 #pragma unroll
-      for (int t = 0; t < kTok; ++t) ag[t] = au[t] = 0.0f;
+      for (int t = 0; t < MT; ++t) ag[t] = au[t] = 0.0f;
       for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
         uint4 gv[kUnroll], uv[kUnroll];
 #pragma unroll
@@ -108,8 +110,8 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
           const int v = v0 + 32 * u;
           if (v < nv) {
 #pragma unroll
-            for (int t = 0; t < kTok; ++t) {
-              if (t < mc && xr[t] != nullptr) {
+            for (int t = 0; t < MT; ++t) {
+              if (xr[t] != nullptr) {
                 float xf[8];
                 unpack8_bf16(ld_nc_u4(xr[t] + v * 8), xf);
                 ag[t] = dot8_bf16(gv[u], xf, ag[t]);
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
         }
       }
 #pragma unroll
-      for (int t = 0; t < kTok; ++t) {
+      for (int t = 0; t < MT; ++t) {
         if (t < mc) {
           const float g = warp_sum(ag[t]);
           const float u = warp_sum(au[t]);
@@ -135,13 +137,17 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
   }
 }
 
+// Down pass: one warp per block of ROWS output rows of one expert; the rows
+// (I bf16 each) are streamed together against up to MT tokens' h per pass.
+template <int MT, int ROWS>
 __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
+  static_assert(ROWS * MT <= 32, "one lane per (row, token) output");
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int n_act = min(max(*(volatile int*)&a.hdr->num_active, 0), a.E);
   const int H = a.H;
-  const int nrb = (H + kDownRows - 1) / kDownRows;
+  const int nrb = (H + ROWS - 1) / ROWS;
   const int64_t routed_items = (int64_t)n_act * nrb;
   const int64_t total = routed_items + (a.ws_down != nullptr ? nrb : 0);
 
@@ -153,56 +159,56 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
     int64_t r0 = 0, m = 0;
     if (!shared) {
       const int aidx = (int)(item / nrb);
-      n0 = (int)(item - (int64_t)aidx * nrb) * kDownRows;
+      n0 = (int)(item - (int64_t)aidx * nrb) * ROWS;
       int e;
       if (!expert_rows(a, aidx, e, r0, m)) continue;
       K = a.I;
       w0 = a.w_down + ((int64_t)e * H + n0) * K;
       hin = static_cast<const float*>(a.h_perm);
     } else {
-      n0 = (int)(item - routed_items) * kDownRows;
+      n0 = (int)(item - routed_items) * ROWS;
       K = a.Is;
       w0 = a.ws_down + (int64_t)n0 * K;
       hin = static_cast<const float*>(a.h_shared);
       m = a.T;
     }
     const int nvk = K / 8;
-    const int nrows = min(kDownRows, H - n0);
-    for (int64_t c0 = 0; c0 < m; c0 += kTok) {
-      const int mc = (int)min((int64_t)kTok, m - c0);
-      float acc[kDownRows][kTok];
+    const int nrows = min(ROWS, H - n0);
+    for (int64_t c0 = 0; c0 < m; c0 += MT) {
+      const int mc = (int)min((int64_t)MT, m - c0);
+      float acc[ROWS][MT];
 #pragma unroll
-      for (int r = 0; r < kDownRows; ++r)
+      for (int r = 0; r < ROWS; ++r)
 #pragma unroll
-        for (int t = 0; t < kTok; ++t) acc[r][t] = 0.0f;
+        for (int t = 0; t < MT; ++t) acc[r][t] = 0.0f;
 #pragma unroll 2
       for (int v = lane; v < nvk; v += 32) {
-        uint4 wv[kDownRows];
+        uint4 wv[ROWS];
 #pragma unroll
-        for (int r = 0; r < kDownRows; ++r)
+        for (int r = 0; r < ROWS; ++r)
           if (r < nrows) wv[r] = ld_stream_u4(w0 + (int64_t)r * K + v * 8);
 #pragma unroll
-        for (int t = 0; t < kTok; ++t) {
+        for (int t = 0; t < MT; ++t) {
           if (t < mc) {
             const float4* hp = reinterpret_cast<const float4*>(hin + (r0 + c0 + t) * K + v * 8);
             const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
             const float hf[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-            for (int r = 0; r < kDownRows; ++r)
+            for (int r = 0; r < ROWS; ++r)
               if (r < nrows) acc[r][t] = dot8_bf16(wv[r], hf, acc[r][t]);
           }
         }
       }
       float mine = 0.0f;
 #pragma unroll
-      for (int r = 0; r < kDownRows; ++r)
+      for (int r = 0; r < ROWS; ++r)
 #pragma unroll
-        for (int t = 0; t < kTok; ++t)
+        for (int t = 0; t < MT; ++t)
           if (t < mc && r < nrows) {
             const float s = warp_sum(acc[r][t]);
-            if (lane == r * kTok + t) mine = s;
+            if (lane == r * MT + t) mine = s;
           }
-      const int r = lane / kTok, t = lane % kTok;
+      const int r = lane / MT, t = lane % MT;
       if (r < nrows && t < mc) {
         if (!shared) {
           int64_t slot;
@@ -252,17 +258,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s) {
+template <int MT, int ROWS>
+cudaError_t launch_gemv_mt(const FfnArgs& a, cudaStream_t s) {
   const int blocks = sm_count() * 4;
   before_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
-  gemv_gate_up_kernel<<<blocks, 256, 0, s>>>(a);
+  gemv_gate_up_kernel<MT><<<blocks, 256, 0, s>>>(a);
   after_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   before_launch(MOE_KERNEL_EXPERT_DOWN, s);
-  gemv_down_kernel<<<blocks, 256, 0, s>>>(a);
+  gemv_down_kernel<MT, ROWS><<<blocks, 256, 0, s>>>(a);
   after_launch(MOE_KERNEL_EXPERT_DOWN, s);
   return cudaGetLastError();
+}
+
+// Tokens per pass follow the batch (an expert has at most T rows), so the
+// single-token decode step carries one accumulator per row.
+cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s) {
+  if (a.T <= 1) return launch_gemv_mt<1, 8>(a, s);
+  if (a.T <= 2) return launch_gemv_mt<2, 8>(a, s);
+  if (a.T <= 4) return launch_gemv_mt<4, 4>(a, s);
+  return launch_gemv_mt<8, 4>(a, s);
 }
 
 cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,

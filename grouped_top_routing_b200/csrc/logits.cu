@@ -5,7 +5,7 @@
 // is [E, H]).
 //
 // This file holds the small-batch form (T <= 16): a weight-streaming GEMV, one
-// warp per expert row, 16-byte loads, every token of the batch against each
+// block per expert row, 16-byte loads, every token of the batch against each
 // row, fp32 FMA. Larger batches run on the tensor cores (umma_ffn.cu).
 #include "common.cuh"
 
@@ -15,45 +15,56 @@ namespace {
 
 constexpr int kGemvMaxT = 16;  // largest batch this kernel takes
 
-// One warp per expert row; each lane covers 8 consecutive h per step
-// (two float4 of router_w, one 16-byte bf16 chunk of x per token).
-__global__ void __launch_bounds__(256) logits_gemv_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w,
+// One block of 128 threads per expert row: thread i covers h in
+// [32 i, 32 i + 32) (eight float4 of router_w, issued together), against every
+// token of the batch; a block reduction then gives the T logits of the row.
+// With one block per row, the whole router weight is in flight at once.
+template <int MT>
+__global__ void __launch_bounds__(128) logits_gemv_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w,
                                                           float* __restrict__ out, int T, int H, int E) {
-  const int lane = threadIdx.x & 31;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int nv = H / 8;
-  for (int e = gw; e < E; e += nw) {
-    const float* wr = w + (size_t)e * H;
-    float acc[kGemvMaxT];
+  __shared__ float red[4][MT];
+  const int e = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* wr = w + (size_t)e * H;
+  float acc[MT];
 #pragma unroll
-    for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.0f;
-    for (int v = lane; v < nv; v += 32) {
-      const uint4 a = ld_stream_u4(wr + v * 8);
-      const uint4 b = ld_stream_u4(wr + v * 8 + 4);
-      float wf[8] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w),
-                     __uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w)};
+  for (int t = 0; t < MT; ++t) acc[t] = 0.0f;
+  for (int h0 = tid * 32; h0 < H; h0 += 128 * 32) {
+    float4 wv[8];
 #pragma unroll
-      for (int t = 0; t < kGemvMaxT; ++t) {
-        if (t < T) {
-          const uint4 xv = ld_nc_u4(x + (size_t)t * H + v * 8);
-          float xf[8];
-          unpack8_bf16(xv, xf);
-          float s = acc[t];
+    for (int u = 0; u < 8; ++u)
+      wv[u] = (h0 + 4 * u < H) ? __ldg(reinterpret_cast<const float4*>(wr + h0) + u) : make_float4(0, 0, 0, 0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) s = fmaf(xf[i], wf[i], s);
-          acc[t] = s;
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < kGemvMaxT; ++t) {
+    for (int t = 0; t < MT; ++t) {
       if (t < T) {
-        const float s = warp_sum(acc[t]);
-        if (lane == 0) out[(size_t)t * E + e] = s;
+        float s = acc[t];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (h0 + 8 * u < H) {
+            float xf[8];
+            unpack8_bf16(ld_nc_u4(x + (size_t)t * H + h0 + 8 * u), xf);
+            const float4 a = wv[2 * u], b = wv[2 * u + 1];
+            s = fmaf(xf[0], a.x, s);
+            s = fmaf(xf[1], a.y, s);
+            s = fmaf(xf[2], a.z, s);
+            s = fmaf(xf[3], a.w, s);
+            s = fmaf(xf[4], b.x, s);
+            s = fmaf(xf[5], b.y, s);
+            s = fmaf(xf[6], b.z, s);
+            s = fmaf(xf[7], b.w, s);
+          }
+        }
+        acc[t] = s;
       }
     }
   }
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+    const float v = warp_sum(acc[t]);
+    if (lane == 0) red[warp][t] = v;
+  }
+  __syncthreads();
+  if (tid < MT && tid < T) out[(size_t)tid * E + e] = (red[0][tid] + red[1][tid]) + (red[2][tid] + red[3][tid]);
 }
 
 }  // namespace
@@ -64,8 +75,9 @@ cudaError_t launch_router_logits_gemv(const moe_config& c, const uint16_t* x, in
   if (T > kGemvMaxT) return cudaErrorInvalidValue;
   const int H = c.hidden_size, E = c.num_experts;
   before_launch(MOE_KERNEL_ROUTER_LOGITS, s);
-  const int blocks = (E * 32 + 255) / 256;
-  logits_gemv_kernel<<<blocks, 256, 0, s>>>(x, w, out, (int)T, H, E);
+  if (T <= 1) logits_gemv_kernel<1><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
+  else if (T <= 4) logits_gemv_kernel<4><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
+  else logits_gemv_kernel<16><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
   after_launch(MOE_KERNEL_ROUTER_LOGITS, s);
   return cudaGetLastError();
 }

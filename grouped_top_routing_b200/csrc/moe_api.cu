@@ -263,12 +263,16 @@ moe_status run_logits(const moe_config& c, const uint16_t* x, int64_t T, const f
   return MOE_OK;
 }
 
-// Tensor cores once experts average at least two rows; below that (decode)
-// the streaming GEMV spreads the weight rows over every SM.
+// The streaming GEMV serves batches of up to kStreamMaxT tokens: every expert
+// then has at most that many rows, all taken in one pass over its weights, and
+// the weight rows spread over every SM. Larger batches take the tensor cores.
+constexpr int64_t kStreamMaxT = 8;
+
 bool use_tensor_cores(const moe_config& c, int64_t T) {
+  (void)c;
   if (g_ffn_path == 1) return false;
   if (g_ffn_path == 2) return true;
-  return T * c.num_experts_per_tok >= 2 * (int64_t)c.num_experts;
+  return T > kStreamMaxT;
 }
 
 moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint16_t* x_perm,

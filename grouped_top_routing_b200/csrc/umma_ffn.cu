@@ -52,10 +52,10 @@ constexpr int kMaxGroups = 1025;  // routed experts (<= 1024) + the shared MLP
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum : int { kGateUp = 0, kDown = 1, kLogits = 2 };
-constexpr int kLogitsBN = 128;
+constexpr int kLogitsBN = 32;  // token columns per logits tile; chunk sums live in registers
 // The router-logits GEMM accumulates at most this many k-blocks (32 MMAs of
-// K = 16) in one TMEM accumulator; the epilogue adds the chunk sums into the
-// output in fp32. Long tensor-core accumulation chains drift (measured: error
+// K = 16) in one TMEM accumulator; the epilogue adds the chunk sums in fp32
+// registers. Long tensor-core accumulation chains drift (measured: error
 // grows with the chain length), short ones stay within a few fp32 ulps.
 constexpr int kLogitsChunk = 8;
 
@@ -493,10 +493,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= epilogue (warps 2..5) =======================
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    constexpr int kColRegs = (BN + 31) / 32;                // token columns per lane (DOWN)
+    constexpr int kSumCols = MODE == kLogits ? BN : 1;      // running chunk sums (LOGITS)
     int tcount = 0;
     bool alive = true;
     for (int tile = blockIdx.x; alive && tile < total_tiles; tile += gridDim.x) {
       const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+      const int mvalid = min(BN, t.m - t.mb * BN);
+      // DOWN: every token column's destination slot and routing weight, fetched
+      // once per tile (column lane + 32 r in register r) before the accumulator
+      // is ready, so the stores below need no memory round trip
+      long long col_slot[kColRegs];
+      float col_w[kColRegs];
+      if (MODE == kDown) {
+#pragma unroll
+        for (int r = 0; r < kColRegs; ++r) {
+          const int c = lane + 32 * r;
+          col_slot[r] = -1;
+          col_w[r] = 1.0f;
+          if (c < mvalid) {
+            const int64_t tok_row = (int64_t)t.mb * BN + c;
+            if (t.shared) {
+              col_slot[r] = tok_row;
+            } else {
+              const long long sl = p.tok_of[t.r0 + tok_row];
+              if (sl < 0 || sl >= R) record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tok_row));
+              else col_slot[r] = sl;
+            }
+          }
+        }
+        if (!t.shared && p.topk_w != nullptr) {
+#pragma unroll
+          for (int r = 0; r < kColRegs; ++r)
+            if (col_slot[r] >= 0) col_w[r] = p.topk_w[col_slot[r]];
+        }
+      }
+      float sum0[kSumCols], sum1[kSumCols];
       for (int ch = 0; ch < t.nchunks; ++ch, ++tcount) {
         const int a = tcount & 1;
         const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
@@ -512,27 +544,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * SH::NA * SH::NCOL);
-        const int mvalid = min(BN, t.m - t.mb * BN);
-        for (int c0 = 0; c0 < mvalid; c0 += 16) {
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          if (c0 >= mvalid) break;  // warp-uniform
           float v0[16], v1[16];
-          if (MODE != kDown) {  // D0 and D1 columns c0 .. c0+15
+          if (MODE == kLogits) {
+            // chunk sums stay in registers; one fp32 add per chunk per element
             tmem_ld16(taddr + c0, v0);
             tmem_ld16(taddr + SH::NCOL + c0, v1);
-          }
-          if (MODE == kLogits) {
-            const int e0 = t.nb * 2 * BM + row, e1 = e0 + BM;
-            float* out = p.logits_out + (int64_t)t.ks * p.T * p.E;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int c = c0 + i;
-              if (c < mvalid) {
-                const int64_t tok = (int64_t)t.mb * BN + c;
-                // chunk 0 stores, later chunks add (each thread owns its elements)
-                if (e0 < p.E) out[tok * p.E + e0] = ch == 0 ? v0[i] : out[tok * p.E + e0] + v0[i];
-                if (e1 < p.E) out[tok * p.E + e1] = ch == 0 ? v1[i] : out[tok * p.E + e1] + v1[i];
-              }
+              sum0[(c0 + i) % kSumCols] = ch == 0 ? v0[i] : sum0[(c0 + i) % kSumCols] + v0[i];
+              sum1[(c0 + i) % kSumCols] = ch == 0 ? v1[i] : sum1[(c0 + i) % kSumCols] + v1[i];
             }
           } else if (MODE == kGateUp) {
+            tmem_ld16(taddr + c0, v0);
+            tmem_ld16(taddr + SH::NCOL + c0, v1);
             const int j = t.nb * BM + row;
             const int width = t.shared ? p.Is : p.I;
             if (j < width) {
@@ -553,24 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             const int n = t.nb * SH::ROWS + row;
-            // lane i < 16 fetches the slot and routing weight of column c0 + i;
-            // the loop takes them by shuffle: one load round trip per chunk
-            long long my_slot = -1;
-            float my_w = 1.0f;
-            if (lane < 16 && c0 + lane < mvalid) {
-              const int64_t tok_row = (int64_t)t.mb * BN + c0 + lane;
-              if (t.shared) {
-                my_slot = tok_row;
-              } else {
-                my_slot = p.tok_of[t.r0 + tok_row];
-                if (my_slot < 0 || my_slot >= R) {
-                  record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tok_row));
-                  my_slot = -1;
-                } else if (p.topk_w != nullptr) {
-                  my_w = p.topk_w[my_slot];
-                }
-              }
-            }
             float* base = t.shared ? p.shared_out : p.y_slots;
 #pragma unroll
             for (int acc_i = 0; acc_i < SH::NA; ++acc_i) {  // accumulator acc_i: weight rows n + acc_i * 128
@@ -580,8 +589,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int nn = n + acc_i * BM;
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const long long slot = __shfl_sync(0xffffffffu, my_slot, i);
-                const float w = __shfl_sync(0xffffffffu, my_w, i);
+                const int c = c0 + i;  // compile-time after unrolling
+                const long long slot = __shfl_sync(0xffffffffu, col_slot[c / 32], c % 32);
+                const float w = __shfl_sync(0xffffffffu, col_w[c / 32], c % 32);
                 if (slot >= 0 && nn < p.H) base[slot * p.H + nn] = w * (v0[i] + v1[i]);
               }
             }
@@ -590,6 +600,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[a]);
+      }
+      if (MODE == kLogits && alive) {  // the tile's logits, written once
+        const int e0 = t.nb * 2 * BM + row, e1 = e0 + BM;
+        float* out = p.logits_out + (int64_t)t.ks * p.T * p.E;
+#pragma unroll
+        for (int c = 0; c < kSumCols; ++c) {
+          if (c < mvalid) {
+            const int64_t tok = (int64_t)t.mb * BN + c;
+            if (e0 < p.E) out[tok * p.E + e0] = sum0[c];
+            if (e1 < p.E) out[tok * p.E + e1] = sum1[c];
+          }
+        }
       }
     }
   }
@@ -776,7 +798,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   m[3] = m[0];
   m[4] = m[1];
   m[5] = m[1];
-  constexpr int kStages = 4;
+  constexpr int kStages = 5;
   const size_t smem = Smem<kLogitsBN, kStages, kLogits>::kTotal;
   e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
