@@ -251,6 +251,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    M.set_ffn_path(args.ffn_path)
     wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
@@ -372,7 +373,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "overrides": args.set, "tokens": T, "hidden_size": wl["hidden_size"],
+        "config": {"workload": args.workload, "overrides": args.set, "ffn_path": args.ffn_path, "tokens": T, "hidden_size": wl["hidden_size"],
                    "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
@@ -401,6 +402,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=64)
     ap.add_argument("--ref-sample", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ffn-path", default="auto", choices=["auto", "streaming", "tensor_cores"],
+                    help="expert-FFN kernels (default: the library's automatic choice)")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (e.g. num_experts=64 for a small profiling case)")
     args = ap.parse_args()

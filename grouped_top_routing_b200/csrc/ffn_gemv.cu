@@ -54,6 +54,8 @@ __device__ __forceinline__ int64_t slot_token(const FfnArgs& a, int64_t row, int
 // gate row and up row (H bf16 each) against up to MT tokens per pass.
 template <int MT>
 __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -141,6 +143,8 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
 // (I bf16 each) are streamed together against up to MT tokens' h per pass.
 template <int MT, int ROWS>
 __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   static_assert(ROWS * MT <= 32, "one lane per (row, token) output");
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -229,6 +233,8 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_slots,
                                                       const float* __restrict__ shared_out, int64_t T, int k, int H,
                                                       uint16_t* __restrict__ y) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int nv = H / 4;
   const int64_t n = T * nv;
   const float4* ys = reinterpret_cast<const float4*>(y_slots);
@@ -262,12 +268,12 @@ template <int MT, int ROWS>
 cudaError_t launch_gemv_mt(const FfnArgs& a, cudaStream_t s) {
   const int blocks = sm_count() * 4;
   before_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
-  gemv_gate_up_kernel<MT><<<blocks, 256, 0, s>>>(a);
+  launch_pdl(gemv_gate_up_kernel<MT>, dim3(blocks), dim3(256), 0, s, a);
   after_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   before_launch(MOE_KERNEL_EXPERT_DOWN, s);
-  gemv_down_kernel<MT, ROWS><<<blocks, 256, 0, s>>>(a);
+  launch_pdl(gemv_down_kernel<MT, ROWS>, dim3(blocks), dim3(256), 0, s, a);
   after_launch(MOE_KERNEL_EXPERT_DOWN, s);
   return cudaGetLastError();
 }
@@ -289,7 +295,7 @@ cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_
   const int64_t cap = (int64_t)sm_count() * 8;
   if (blocks > cap) blocks = cap;
   before_launch(MOE_KERNEL_COMBINE, s);
-  combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(y_slots, shared_out, T, k, H, y);
+  launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(256), 0, s, y_slots, shared_out, T, k, H, y);
   after_launch(MOE_KERNEL_COMBINE, s);
   return cudaGetLastError();
 }

@@ -22,6 +22,8 @@ constexpr int kGemvMaxT = 16;  // largest batch this kernel takes
 template <int MT>
 __global__ void __launch_bounds__(128) logits_gemv_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w,
                                                           float* __restrict__ out, int T, int H, int E) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float red[4][MT];
   const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -75,9 +77,9 @@ cudaError_t launch_router_logits_gemv(const moe_config& c, const uint16_t* x, in
   if (T > kGemvMaxT) return cudaErrorInvalidValue;
   const int H = c.hidden_size, E = c.num_experts;
   before_launch(MOE_KERNEL_ROUTER_LOGITS, s);
-  if (T <= 1) logits_gemv_kernel<1><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
-  else if (T <= 4) logits_gemv_kernel<4><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
-  else logits_gemv_kernel<16><<<E, 128, 0, s>>>(x, w, out, (int)T, H, E);
+  if (T <= 1) launch_pdl(logits_gemv_kernel<1>, dim3(E), dim3(128), 0, s, x, w, out, (int)T, H, E);
+  else if (T <= 4) launch_pdl(logits_gemv_kernel<4>, dim3(E), dim3(128), 0, s, x, w, out, (int)T, H, E);
+  else launch_pdl(logits_gemv_kernel<16>, dim3(E), dim3(128), 0, s, x, w, out, (int)T, H, E);
   after_launch(MOE_KERNEL_ROUTER_LOGITS, s);
   return cudaGetLastError();
 }

@@ -263,10 +263,11 @@ moe_status run_logits(const moe_config& c, const uint16_t* x, int64_t T, const f
   return MOE_OK;
 }
 
-// The streaming GEMV serves batches of up to kStreamMaxT tokens: every expert
+// The streaming GEMV serves batches of up to kStreamMaxT tokens (measured on
+// B200: faster than the tensor cores at 1-2 tokens, slower from 4): every expert
 // then has at most that many rows, all taken in one pass over its weights, and
 // the weight rows spread over every SM. Larger batches take the tensor cores.
-constexpr int64_t kStreamMaxT = 8;
+constexpr int64_t kStreamMaxT = 2;
 
 bool use_tensor_cores(const moe_config& c, int64_t T) {
   (void)c;

@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int32_t* __restr
                                                           const int32_t* __restrict__ tok_of, int k, int64_t T,
                                                           const uint16_t* __restrict__ x, int H,
                                                           uint16_t* __restrict__ x_perm) {
+  pdl_launch_dependents();
+  pdl_wait();
   int64_t R = offsets[E];
   if (R < 0) R = 0;
   if (R > T * k) R = T * k;
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int32_t* __restr
 
 __global__ void __launch_bounds__(kTile) permute_count_kernel(const int32_t* __restrict__ idx, int64_t T, int k, int E,
                                                               int32_t* __restrict__ tile_cnt, WsHeader* hdr) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint32_t masks[];
   const int64_t t0 = (int64_t)blockIdx.x * kTile;
   build_masks(masks, idx, t0, T, k, E, hdr, true);
@@ -149,6 +153,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __res
                                                             int32_t* __restrict__ offsets,
                                                             int32_t* __restrict__ tile_base,
                                                             int32_t* __restrict__ active, WsHeader* hdr) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = threadIdx.x;
   int total = 0;
   if (e < E)
@@ -176,6 +182,8 @@ __global__ void __launch_bounds__(kTile) permute_scatter_kernel(const int32_t* _
                                                                 const int32_t* __restrict__ tile_base,
                                                                 int32_t* __restrict__ row_of,
                                                                 int32_t* __restrict__ tok_of) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint32_t masks[];
   const int64_t t0 = (int64_t)blockIdx.x * kTile;
   build_masks(masks, idx, t0, T, k, E, nullptr, false);
@@ -188,6 +196,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
                                                              int32_t* __restrict__ offsets, int32_t* __restrict__ row_of,
                                                              int32_t* __restrict__ tok_of, int32_t* __restrict__ active,
                                                              WsHeader* hdr) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint32_t masks[];
   int* base = reinterpret_cast<int*>(masks + E * kWords);
   for (int i = threadIdx.x; i < E * kWords; i += blockDim.x) masks[i] = 0u;
@@ -241,13 +251,13 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
   if (T <= kTile) {
     const size_t smem = mask_bytes + (size_t)E * sizeof(int);
     nk = 1;
-    permute_small_kernel<<<1, 1024, smem, s>>>(idx, T, k, E, offsets, row_of, tok_of, active, hdr);
+    launch_pdl(permute_small_kernel, dim3(1), dim3(1024), smem, s, idx, T, k, E, offsets, row_of, tok_of, active, hdr);
   } else {
     const int n_tiles = (int)((T + kTile - 1) / kTile);
     nk = 3;
-    permute_count_kernel<<<n_tiles, kTile, mask_bytes, s>>>(idx, T, k, E, tile_cnt, hdr);
-    permute_scan_kernel<<<1, 1024, 0, s>>>(tile_cnt, n_tiles, E, offsets, tile_base, active, hdr);
-    permute_scatter_kernel<<<n_tiles, kTile, mask_bytes, s>>>(idx, T, k, E, tile_base, row_of, tok_of);
+    launch_pdl(permute_count_kernel, dim3(n_tiles), dim3(kTile), mask_bytes, s, idx, T, k, E, tile_cnt, hdr);
+    launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, tile_cnt, n_tiles, E, offsets, tile_base, active, hdr);
+    launch_pdl(permute_scatter_kernel, dim3(n_tiles), dim3(kTile), mask_bytes, s, idx, T, k, E, tile_base, row_of, tok_of);
   }
   if (x_perm != nullptr) {
     const int64_t chunks = T * k * (H / 8);
@@ -255,7 +265,7 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
     const int64_t cap = (int64_t)sm_count() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(offsets, E, tok_of, k, T, x, H, x_perm);
+    launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, offsets, E, tok_of, k, T, x, H, x_perm);
     ++nk;
   }
   after_launch(MOE_KERNEL_PERMUTE, s, nk);
@@ -270,7 +280,7 @@ cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   before_launch(MOE_KERNEL_PERMUTE, s);
-  gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(offsets, E, tok_of, k, T, x, H, x_perm);
+  launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, offsets, E, tok_of, k, T, x, H, x_perm);
   after_launch(MOE_KERNEL_PERMUTE, s);
   return cudaGetLastError();
 }
@@ -279,6 +289,8 @@ cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok
 // when moe_expert_ffn is called on its own).
 __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t* __restrict__ offsets, int E,
                                                                    int32_t* __restrict__ active, WsHeader* hdr) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = threadIdx.x;
   const int has = (e < E && offsets[e + 1] > offsets[e]) ? 1 : 0;
   int n = 0;
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(1024) active_from_offsets_kernel(const int32_t
 cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, WsHeader* hdr,
                                        cudaStream_t s) {
   before_launch(MOE_KERNEL_PERMUTE, s);
-  active_from_offsets_kernel<<<1, 1024, 0, s>>>(offsets, E, active, hdr);
+  launch_pdl(active_from_offsets_kernel, dim3(1), dim3(1024), 0, s, offsets, E, active, hdr);
   after_launch(MOE_KERNEL_PERMUTE, s);
   return cudaGetLastError();
 }

@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(256) route_kernel(
     const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, int n_group,
     int topk_group, int score_fn, int norm, float scale, int32_t* __restrict__ idx_out,
     float* __restrict__ w_out) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -201,7 +203,7 @@ cudaError_t launch_route_p(const moe_config& c, const float* logits, const float
     if (e != cudaSuccess) return e;
   }
   before_launch(MOE_KERNEL_ROUTE, s);
-  route_kernel<P><<<blocks, wpb * 32, smem, s>>>(logits, bias, T, c.num_experts, c.num_experts_per_tok,
+  launch_pdl(route_kernel<P>, dim3(blocks), dim3(wpb * 32), smem, s, logits, bias, T, c.num_experts, c.num_experts_per_tok,
                                                  c.n_group, c.topk_group, c.score_function, c.norm_topk_prob,
                                                  c.routed_scaling_factor, idx, w);
   after_launch(MOE_KERNEL_ROUTE, s);

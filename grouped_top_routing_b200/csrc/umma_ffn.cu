@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap mapB2_r, const __grid_constant__ CUtensorMap mapA_s,
                     const __grid_constant__ CUtensorMap mapB_s, const __grid_constant__ CUtensorMap mapB2_s,
                     const UmmaParams p) {
+  pdl_launch_dependents();
   using L = Smem<BN, STAGES, MODE>;
   using SH = Shape<BN, MODE>;
   constexpr uint32_t kTmemCols = SH::kTmemCols;
@@ -339,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  pdl_wait();  // everything below may read what earlier launches wrote
 
   // ---- group table: active experts (+ shared MLP), tiles per group ----
   const int n_act = MODE == kLogits ? 0 : min(max(*(volatile int*)&p.hdr->num_active, 0), p.E);
@@ -665,8 +667,7 @@ cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel
                                        (int)smem);
   if (e != cudaSuccess) return e;
   before_launch(kernel_id, s);
-  umma_ffn_kernel<BN, STAGES, MODE>
-      <<<sm_count(), kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  launch_pdl(umma_ffn_kernel<BN, STAGES, MODE>, dim3(sm_count()), dim3(kThreads), smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
   after_launch(kernel_id, s);
   return cudaGetLastError();
 }
@@ -731,6 +732,8 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
 // accumulate sum_h x[t,h] * w[e,h] over K = 3H in fp32.
 __global__ void __launch_bounds__(256) split_router_weight_kernel(const float* __restrict__ w, int64_t n,
                                                                   uint16_t* __restrict__ planes) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const float v = __ldg(w + i);
     const uint16_t hi = f32_to_bf16(v);
@@ -746,6 +749,8 @@ __global__ void __launch_bounds__(256) split_router_weight_kernel(const float* _
 // logits[t, e] = sum_s part[s, t, e], s ascending.
 __global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restrict__ part, int ksplit, int64_t n,
                                                             float* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     float acc = part[i];
     for (int s = 1; s < ksplit; ++s) acc += part[(int64_t)s * n + i];
@@ -779,7 +784,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   int64_t blocks = (n + 255) / 256;
   if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
   before_launch(MOE_KERNEL_ROUTER_LOGITS, s);
-  split_router_weight_kernel<<<(unsigned)blocks, 256, 0, s>>>(w, n, planes);
+  launch_pdl(split_router_weight_kernel, dim3((unsigned)blocks), dim3(256), 0, s, w, n, planes);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   UmmaParams p{};
@@ -803,7 +808,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  umma_ffn_kernel<kLogitsBN, kStages, kLogits><<<sm_count(), kThreads, smem, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  launch_pdl(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, dim3(sm_count()), dim3(kThreads), smem, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int nk = 2;
@@ -811,7 +816,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
     const int64_t nl = T * E;
     int64_t rb = (nl + 255) / 256;
     if (rb > (int64_t)sm_count() * 8) rb = (int64_t)sm_count() * 8;
-    reduce_splits_kernel<<<(unsigned)rb, 256, 0, s>>>(partials, ksplit, nl, logits);
+    launch_pdl(reduce_splits_kernel, dim3((unsigned)rb), dim3(256), 0, s, partials, ksplit, nl, logits);
     nk = 3;
   }
   after_launch(MOE_KERNEL_ROUTER_LOGITS, s, nk);

@@ -204,7 +204,7 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
 moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop);
 
 /* Selects the expert-FFN kernels for every later call in this process:
- * 0 = automatic (the streaming GEMV for T <= 8 tokens, where each expert's
+ * 0 = automatic (the streaming GEMV for T <= 2 tokens, where each expert's
  * weights are streamed once over all SMs; the tensor-core grouped GEMM above),
  * 1 = always the streaming GEMV, 2 = always the tensor-core grouped GEMM.
  * Both compute the same block. */
