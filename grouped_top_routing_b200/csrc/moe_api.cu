@@ -535,3 +535,83 @@ moe_status moe_set_ffn_path(int32_t path) {
 const char* moe_last_error(void) { return g_err; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_permute_static: the permutation without a caller-provided workspace.
+//
+// For callers that cannot allocate device memory: code running under a host
+// framework that owns every device allocation, plugins whose host forbids
+// them, or latency-critical loops where cudaMalloc's implicit device-wide
+// synchronisation is not acceptable. Its scratch lives in one file-scope
+// device array; every GPU that loads this library holds it until exit.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+std::atomic<void*> g_static_scratch_addr[64];  // device address of g_static_scratch, per device
+
+// Scratch bytes the permutation needs for T tokens: the 256-byte header (error
+// word, active-expert count), the active-expert list, and for T > 128 the
+// per-tile counts and bases.
+size_t static_scratch_need(const moe_config& c, int64_t T) {
+  const size_t tiles = T > 128 ? permute_scratch_ints(c.num_experts, T) * 4 : 0;
+  return align256(sizeof(WsHeader)) + align256((size_t)c.num_experts * 4) + 2 * align256(tiles);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, int64_t T,
+                                         const uint16_t* x, int32_t* expert_offsets, int32_t* row_of,
+                                         int32_t* tok_of, uint16_t* x_perm, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ptr("expert_offsets", expert_offsets, 4, true));
+  if (T > 0) {
+    MOE_TRY(check_ptr("topk_idx", topk_idx, 4, true));
+    MOE_TRY(check_ptr("row_of", row_of, 4, true));
+    MOE_TRY(check_ptr("tok_of", tok_of, 4, true));
+    MOE_TRY(check_ptr("x_perm", x_perm, 16, false));
+    MOE_TRY(check_ptr("x", x, 16, x_perm != nullptr));
+  }
+  const size_t need = static_scratch_need(*cfg, T);
+  if (need > kStaticScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "T = %lld tokens over num_experts = %d needs %zu bytes of scratch; the static scratch of "
+                "moe_permute_static holds %zu bytes (use moe_permute with a workspace)",
+                (long long)T, cfg->num_experts, need, kStaticScratchBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_permute_static: current device");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+  // Set-up, once per device, with that device current: the host-side name of a
+  // __device__ array is not its device address; ask the runtime for it.
+  void* base = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+  if (base == nullptr) {
+    e = cudaGetSymbolAddress(&base, g_static_scratch);
+    if (e != cudaSuccess || base == nullptr) return cuda_fail(e, "moe_permute_static: cudaGetSymbolAddress");
+    g_static_scratch_addr[dev].store(base, std::memory_order_release);
+  }
+  cudaStream_t s = as_stream(stream);
+  char* p = static_cast<char*>(base);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p);
+  int32_t* active = reinterpret_cast<int32_t*>(p + align256(sizeof(WsHeader)));
+  const size_t tiles = T > 128 ? permute_scratch_ints(cfg->num_experts, T) * 4 : 0;
+  int32_t* tile_cnt = reinterpret_cast<int32_t*>(p + align256(sizeof(WsHeader)) + align256((size_t)cfg->num_experts * 4));
+  int32_t* tile_base = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(tile_cnt) + align256(tiles));
+  // The array keeps the previous call's contents: the header (error word and
+  // active count) must start at zero; the other regions are fully rewritten.
+  e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_permute_static: clear scratch header");
+  if (T == 0) {
+    e = cudaMemsetAsync(expert_offsets, 0, (size_t)(cfg->num_experts + 1) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_permute_static");
+    return MOE_OK;
+  }
+  e = launch_permute(*cfg, topk_idx, T, x, expert_offsets, row_of, tok_of, x_perm, active, tile_cnt, tile_base, hdr,
+                     s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_permute_static");
+  return MOE_OK;
+}

@@ -24,7 +24,7 @@ KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "e
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
-           "moe_set_ffn_path", "moe_launch_count", "moe_last_error")
+           "moe_set_ffn_path", "moe_launch_count", "moe_last_error", "moe_permute_static")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 
 
@@ -80,6 +80,7 @@ def _load():
         "moe_check_device": (st, [vp, sz, vp]),
         "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
         "moe_set_ffn_path": (st, [ctypes.c_int32]),
+        "moe_permute_static": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }

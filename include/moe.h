@@ -213,6 +213,27 @@ moe_status moe_set_ffn_path(int32_t path);
 /* Number of this library's kernel launches since load (host-side counter). */
 uint64_t moe_launch_count(void);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory (a host framework that owns every device allocation, a plugin host
+ * that forbids them, or a latency-critical loop where cudaMalloc's implicit
+ * device synchronisation is unacceptable). The pages have no counterpart: it
+ * is a packaging of the permutation above, with the same outputs bit for bit.
+ *   Scratch: one file-scope 1 MiB device array, held by every GPU that loads
+ *   this library until exit. T beyond what 1 MiB holds is rejected with
+ *   MOE_ERR_UNSUPPORTED (about 65k tokens at E = 256, 16k at E = 1024; any T
+ *   <= 128). The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Calls share the array: two calls whose work overlaps on the GPU (other
+ *   streams, other threads, other devices' calls are fine) race and corrupt
+ *   each other's results. Each call clears what must start at zero.
+ *   Invalid or repeated ids are skipped as in moe_permute; with no workspace
+ *   error word to read, a caller detects them by expert_offsets[E] < T*k.
+ * Arguments, layouts and ownership otherwise as moe_permute. Allocates nothing. */
+moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, int64_t T, const uint16_t* x,
+                              int32_t* expert_offsets, int32_t* row_of, int32_t* tok_of, uint16_t* x_perm,
+                              void* stream);
+
 /* Per-thread text of the last rejected call ("" when none). Never NULL. */
 const char* moe_last_error(void);
 
