@@ -51,7 +51,12 @@ constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1025;  // routed experts (<= 1024) + the shared MLP
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum : int { kGateUp = 0, kDown = 1, kLogits = 2 };
+// Modes. kGateUp / kDown: weight rows are the MMA's M side, the expert's
+// tokens its N side (skinny experts). kGateUpTM / kDownTM ("token-major", for
+// experts with many rows): 128 token rows are M and 256 weight rows N, one
+// 128 x 256 MMA per k-step, which reads less shared memory per flop.
+enum : int { kGateUp = 0, kDown = 1, kLogits = 2, kGateUpTM = 3, kDownTM = 4 };
+constexpr bool token_major(int mode) { return mode == kGateUpTM || mode == kDownTM; }
 constexpr int kLogitsBN = 32;  // token columns per logits tile; chunk sums live in registers
 // The router-logits GEMM accumulates at most this many k-blocks (32 MMAs of
 // K = 16) in one TMEM accumulator; the epilogue adds the chunk sums in fp32
@@ -212,13 +217,19 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
 // two blocks of router rows, share the token tile). DOWN: NB = 2 (the h_hi and
 // h_lo token tiles, one B operand of 2 BN rows) and NA = 2 while the TMEM
 // budget allows (BN <= 64), else 1. Each accumulator is NCOL columns.
+//
+// Token-major modes (BN = 128 token rows): NA = token tiles per stage (1; the
+// h_hi and h_lo planes for kDownTM), NB = 2 weight boxes of 128 rows forming
+// one B operand of 256 rows, one accumulator of NCOL = 256 columns.
 template <int BN, int MODE>
 struct Shape {
-  static constexpr int NA = (MODE == kDown && BN > 64) ? 1 : 2;
-  static constexpr int NB = MODE == kDown ? 2 : 1;
-  static constexpr int NCOL = MODE == kDown ? 2 * BN : BN;
-  static constexpr int ROWS = NA * BM;                 // weight rows per DOWN / LOGITS tile
-  static constexpr uint32_t kTmemCols = 2 * NA * NCOL; // two buffers
+  static constexpr bool TM = token_major(MODE);
+  static constexpr int NA = TM ? (MODE == kDownTM ? 2 : 1) : ((MODE == kDown && BN > 64) ? 1 : 2);
+  static constexpr int NB = TM ? 2 : (MODE == kDown ? 2 : 1);
+  static constexpr int NCOL = TM ? 256 : (MODE == kDown ? 2 * BN : BN);
+  static constexpr int NACC = TM ? 1 : NA;                         // accumulators per buffer
+  static constexpr int ROWS = TM ? (MODE == kDownTM ? 256 : BM) : NA * BM;  // weight rows per tile
+  static constexpr uint32_t kTmemCols = 2 * NACC * NCOL;           // two buffers
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM allocation");
 };
 
@@ -263,7 +274,17 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
   t.nb = local / mblocks;
   t.mb = local - t.nb * mblocks;
   int K;
-  if (MODE == kGateUp) {
+  if (token_major(MODE)) {  // a0/a1 rows: the two 128-row weight boxes; b_row: the token rows
+    if (MODE == kGateUpTM) {
+      K = p.H;
+      t.a0_row = t.shared ? t.nb * BM : t.e * 2 * p.I + t.nb * BM;
+      t.a1_row = t.shared ? p.Is + t.nb * BM : t.a0_row + p.I;
+    } else {
+      K = t.shared ? p.Is : p.I;
+      t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * 2 * BM;
+      t.a1_row = t.a0_row + BM;
+    }
+  } else if (MODE == kGateUp) {
     K = p.H;
     if (t.shared) {
       t.a0_row = t.nb * BM;
@@ -308,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTmemCols = SH::kTmemCols;
   constexpr uint32_t kIdesc = idesc_bf16<BN>();
   constexpr uint32_t kIdescDown = idesc_bf16<(2 * BN <= 256 ? 2 * BN : 256)>();
+  constexpr uint32_t kIdescTM = idesc_bf16<256>();
   static_assert(MODE != kDown || 2 * BN <= 256, "DOWN issues N = 2 BN <= 256");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -346,8 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_act = MODE == kLogits ? 0 : min(max(*(volatile int*)&p.hdr->num_active, 0), p.E);
   const int n_groups = MODE == kLogits ? 1 : n_act + (p.has_shared ? 1 : 0);
   const int64_t R = p.T * p.k;
-  const int nb_routed = MODE == kGateUp ? (p.I + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
-  const int nb_shared = MODE == kGateUp ? (p.Is + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
+  constexpr bool kGU = MODE == kGateUp || MODE == kGateUpTM;
+  const int nb_routed = kGU ? (p.I + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
+  const int nb_shared = kGU ? (p.Is + BM - 1) / BM : (p.H + SH::ROWS - 1) / SH::ROWS;
   for (int g = threadIdx.x; g < n_groups; g += blockDim.x) {
     int e = -1, m = 0, tiles = 0;
     int64_t r0 = 0;
@@ -431,11 +454,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             a1y += piece * p.E;
           }
           mbar_expect_tx(&full[s], L::kStage);
-          tma_load_2d(mA, &full[s], st, kx, a0y);
-          if (L::NA == 2) tma_load_2d(mA, &full[s], st + L::kA, kx, a1y);
           uint8_t* sb = st + L::NA * L::kA;
-          tma_load_2d(mB, &full[s], sb, kx, t.b_row);
-          if (L::NB == 2) tma_load_2d(mB2, &full[s], sb + L::kB, kx, t.b_row);
+          if (SH::TM) {  // A: token tile(s); B: the two weight boxes, back to back
+            tma_load_2d(mB, &full[s], st, kx, t.b_row);
+            if (L::NA == 2) tma_load_2d(mB2, &full[s], st + L::kA, kx, t.b_row);
+            tma_load_2d(mA, &full[s], sb, kx, a0y);
+            tma_load_2d(mA, &full[s], sb + L::kB, kx, a1y);
+          } else {
+            tma_load_2d(mA, &full[s], st, kx, a0y);
+            if (L::NA == 2) tma_load_2d(mA, &full[s], st + L::kA, kx, a1y);
+            tma_load_2d(mB, &full[s], sb, kx, t.b_row);
+            if (L::NB == 2) tma_load_2d(mB2, &full[s], sb + L::kB, kx, t.b_row);
+          }
         }
       }
       // drain: the copies of the last STAGES iterations must have landed
@@ -456,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t d0 = tmem_base + (uint32_t)(a * SH::NA * SH::NCOL);
+          const uint32_t d0 = tmem_base + (uint32_t)(a * SH::NACC * SH::NCOL);
           const uint32_t d1 = d0 + SH::NCOL;
           const int kb_begin = t.nchunks == 1 ? 0 : ch * kLogitsChunk;
           const int kb_end = t.nchunks == 1 ? t.kblocks : min(kb_begin + kLogitsChunk, t.kblocks);
@@ -474,7 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint32_t acc = (kb > kb_begin || kk > 0) ? 1u : 0u;
               const uint64_t bdesc = sw128_desc(sb + kk * 32);
-              if (MODE == kDown) {  // B = [h_hi tile; h_lo tile]: 2 BN rows, each D spans 2 BN columns
+              if (SH::TM) {  // D (128 tokens x 256 weight rows) += A_token . B_weights
+                umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdescTM, acc);
+                if (MODE == kDownTM) umma_bf16(d0, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescTM, 1u);  // h_lo
+              } else if (MODE == kDown) {  // B = [h_hi tile; h_lo tile]: 2 BN rows, each D spans 2 BN columns
                 umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdescDown, acc);
                 if (SH::NA == 2) umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescDown, acc);
               } else {
@@ -530,6 +563,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (col_slot[r] >= 0) col_w[r] = p.topk_w[col_slot[r]];
         }
       }
+      // token-major: this thread owns token row `row` of the tile; DOWN needs
+      // its destination slot and routing weight, fetched before the wait
+      const bool tm_valid = SH::TM && row < mvalid;
+      const int64_t tm_tok = (int64_t)t.mb * BN + row;
+      long long tm_slot = -1;
+      float tm_w = 1.0f;
+      if (MODE == kDownTM && tm_valid) {
+        if (t.shared) {
+          tm_slot = tm_tok;
+        } else {
+          const long long sl = p.tok_of[t.r0 + tm_tok];
+          if (sl < 0 || sl >= R) {
+            record_error(p.hdr, MOE_ERR_DEVICE_CHECK, (int)(t.r0 + tm_tok));
+          } else {
+            tm_slot = sl;
+            if (p.topk_w != nullptr) tm_w = p.topk_w[sl];
+          }
+        }
+      }
       float sum0[kSumCols], sum1[kSumCols];
       for (int ch = 0; ch < t.nchunks; ++ch, ++tcount) {
         const int a = tcount & 1;
@@ -545,10 +597,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * SH::NA * SH::NCOL);
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * SH::NACC * SH::NCOL);
+        if (MODE == kGateUpTM) {
+          // columns [0,128): gate rows nb*128 + c, [128,256): the matching up rows
+          const int width = t.shared ? p.Is : p.I;
+          uint16_t* hrow = t.shared ? p.h_shared + tm_tok * p.Is : p.h_perm + (t.r0 + tm_tok) * p.I;
+          const int64_t plane = t.shared ? p.T * p.Is : p.T * p.k * p.I;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BM; c0 += 16) {
+            float g[16], u[16];
+            tmem_ld16(taddr + c0, g);
+            tmem_ld16(taddr + BM + c0, u);
+            const int j0 = t.nb * BM + c0;
+            if (tm_valid && j0 < width) {
+              uint32_t hi2[8], lo2[8];
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                const float h0 = silu_f32(g[i]) * u[i], h1 = silu_f32(g[i + 1]) * u[i + 1];
+                const uint16_t a0 = f32_to_bf16(h0), a1 = f32_to_bf16(h1);
+                hi2[i / 2] = (uint32_t)a0 | ((uint32_t)a1 << 16);
+                lo2[i / 2] = (uint32_t)f32_to_bf16(h0 - __uint_as_float((uint32_t)a0 << 16)) |
+                             ((uint32_t)f32_to_bf16(h1 - __uint_as_float((uint32_t)a1 << 16)) << 16);
+              }
+              if (j0 + 16 <= width) {
+                uint4* dh = reinterpret_cast<uint4*>(hrow + j0);
+                uint4* dl = reinterpret_cast<uint4*>(hrow + plane + j0);
+                dh[0] = make_uint4(hi2[0], hi2[1], hi2[2], hi2[3]);
+                dh[1] = make_uint4(hi2[4], hi2[5], hi2[6], hi2[7]);
+                dl[0] = make_uint4(lo2[0], lo2[1], lo2[2], lo2[3]);
+                dl[1] = make_uint4(lo2[4], lo2[5], lo2[6], lo2[7]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  if (j0 + i < width) {
+                    hrow[j0 + i] = (uint16_t)(hi2[i / 2] >> (16 * (i & 1)));
+                    hrow[plane + j0 + i] = (uint16_t)(lo2[i / 2] >> (16 * (i & 1)));
+                  }
+                }
+              }
+            }
+          }
+        } else if (MODE == kDownTM) {
+          // columns: 256 weight rows n0 .. n0+255 (h_hi and h_lo already summed by the MMA)
+          const int n0 = t.nb * 2 * BM;
+          float* orow = t.shared ? p.shared_out + tm_tok * p.H : p.y_slots + tm_slot * p.H;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 2 * BM; c0 += 16) {
+            float v[16];
+            tmem_ld16(taddr + c0, v);
+            const int n = n0 + c0;
+            if (tm_valid && tm_slot >= 0 && n < p.H) {
+              if (n + 16 <= p.H) {
+                float4* d = reinterpret_cast<float4*>(orow + n);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  d[i] = make_float4(tm_w * v[4 * i], tm_w * v[4 * i + 1], tm_w * v[4 * i + 2], tm_w * v[4 * i + 3]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (n + i < p.H) orow[n + i] = tm_w * v[i];
+              }
+            }
+          }
+        }
 #pragma unroll
         for (int c0 = 0; c0 < BN; c0 += 16) {
-          if (c0 >= mvalid) break;  // warp-uniform
+          if (SH::TM || c0 >= mvalid) break;  // warp-uniform
           float v0[16], v1[16];
           if (MODE == kLogits) {
             // chunk sums stay in registers; one fp32 add per chunk per element
@@ -674,8 +788,9 @@ cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel
 
 // Stage counts: gate/up stages hold two weight tiles and one token tile; down
 // stages one weight tile and the token tiles of both h planes.
-template <int BN, int ST_GU, int ST_DN>
+template <int BN, int ST_GU, int ST_DN, bool TM>
 cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
+  static_assert(!TM || BN == BM, "token-major tiles hold 128 token rows");
   const int64_t R = a.T * a.k;
   const bool shared = a.ws_gate_up != nullptr;
   UmmaParams p{};
@@ -708,7 +823,7 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   }
   m[5] = m[4];
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = launch_pass<BN, ST_GU, kGateUp>(m, p, MOE_KERNEL_EXPERT_GATE_UP, s);
+  cudaError_t e = launch_pass<BN, ST_GU, TM ? kGateUpTM : kGateUp>(m, p, MOE_KERNEL_EXPERT_GATE_UP, s);
   if (e != cudaSuccess) return e;
 
   // pass 2: down projection of h_hi + h_lo, weighted scatter into slot order
@@ -723,7 +838,7 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
     m[5] = m[2];
   }
   if (!ok) return cudaErrorInvalidValue;
-  return launch_pass<BN, ST_DN, kDown>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
+  return launch_pass<BN, ST_DN, TM ? kDownTM : kDown>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
 }
 
 // Splits the fp32 router weight into three bf16 planes whose sum is the weight
@@ -823,21 +938,26 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   return cudaGetLastError();
 }
 
+// Tile shape from the mean rows per expert (R / min(R, E)): weight-major
+// tiles of BN = 32 / 64 / 128 token columns for skinny experts, token-major
+// 128 x 256 tiles (returned as 256) once experts average 96 rows or more.
 int umma_pick_bn(int64_t T, int k, int E) {
   const int64_t R = T * k;
   const int64_t groups = R < E ? R : E;
   const int64_t avg = groups > 0 ? (R + groups - 1) / groups : 1;
   if (avg <= 24) return 32;
   if (avg <= 64) return 64;
-  return 128;
+  if (avg < 96) return 128;
+  return 256;
 }
 
 cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cudaStream_t s) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   switch (bn) {
-    case 32: return run_bn<32, 5, 5>(a, x_perm, s);
-    case 64: return run_bn<64, 5, 4>(a, x_perm, s);
-    default: return run_bn<128, 4, 4>(a, x_perm, s);
+    case 32: return run_bn<32, 5, 5, false>(a, x_perm, s);
+    case 64: return run_bn<64, 5, 4, false>(a, x_perm, s);
+    case 128: return run_bn<128, 4, 4, false>(a, x_perm, s);
+    default: return run_bn<128, 4, 3, true>(a, x_perm, s);  // token-major
   }
 }
 

@@ -195,6 +195,15 @@ FFN_CASES = [
                             moe_intermediate_size=128, num_shared_experts=0, shared_width=0)),
     ("tiny_ragged", dict(tokens=13, hidden_size=136, num_experts=12, num_experts_per_tok=3,
                          moe_intermediate_size=72, shared_width=144, num_shared_experts=2)),
+    # tile shapes of the tensor-core path, picked from the mean rows per expert:
+    # ~30 rows -> 64-token tiles; ~68 -> 128-token tiles; >= 96 -> token-major
+    # 128 x 256 tiles (here with ragged widths, so the store fallbacks run)
+    ("tiny_bn64", dict(tokens=40, hidden_size=64, num_experts=8, num_experts_per_tok=6,
+                       moe_intermediate_size=64, shared_width=64)),
+    ("tiny_bn128", dict(tokens=90, hidden_size=64, num_experts=8, num_experts_per_tok=6,
+                        moe_intermediate_size=64, shared_width=64)),
+    ("tiny_token_major", dict(tokens=600, hidden_size=200, num_experts=6, num_experts_per_tok=2,
+                              moe_intermediate_size=136, shared_width=272, num_shared_experts=2)),
 ]
 
 
