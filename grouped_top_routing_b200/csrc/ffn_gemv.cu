@@ -21,7 +21,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kUnroll = 4;  // 16-byte chunks in flight per lane per weight row (gate/up pass)
+constexpr int kUnroll = 8;  // 16-byte chunks in flight per lane per weight row (gate/up pass)
 
 // Resolves the rows [r0, r0 + m) of one active expert, clamped to [0, T*k).
 __device__ __forceinline__ bool expert_rows(const FfnArgs& a, int aidx, int& e, int64_t& r0, int64_t& m) {
@@ -264,16 +264,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
+// One resident wave: as many 256-thread blocks as the kernel's register use
+// lets every SM hold at once (a second wave would double the latency chain).
+template <typename K>
+int resident_blocks(K kernel) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  return sm_count() * per_sm;
+}
+
 template <int MT, int ROWS>
 cudaError_t launch_gemv_mt(const FfnArgs& a, cudaStream_t s) {
-  const int blocks = sm_count() * 4;
   before_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
-  launch_pdl(gemv_gate_up_kernel<MT>, dim3(blocks), dim3(256), 0, s, a);
+  launch_pdl(gemv_gate_up_kernel<MT>, dim3(resident_blocks(gemv_gate_up_kernel<MT>)), dim3(256), 0, s, a);
   after_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   before_launch(MOE_KERNEL_EXPERT_DOWN, s);
-  launch_pdl(gemv_down_kernel<MT, ROWS>, dim3(blocks), dim3(256), 0, s, a);
+  launch_pdl(gemv_down_kernel<MT, ROWS>, dim3(resident_blocks(gemv_down_kernel<MT, ROWS>)), dim3(256), 0, s, a);
   after_launch(MOE_KERNEL_EXPERT_DOWN, s);
   return cudaGetLastError();
 }

@@ -57,7 +57,7 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 // 128 x 256 MMA per k-step, which reads less shared memory per flop.
 enum : int { kGateUp = 0, kDown = 1, kLogits = 2, kGateUpTM = 3, kDownTM = 4 };
 constexpr bool token_major(int mode) { return mode == kGateUpTM || mode == kDownTM; }
-constexpr int kLogitsBN = 32;  // token columns per logits tile; chunk sums live in registers
+constexpr int kLogitsBN = 64;  // token columns per logits tile; chunk sums live in registers
 // The router-logits GEMM accumulates at most this many k-blocks (32 MMAs of
 // K = 16) in one TMEM accumulator; the epilogue adds the chunk sums in fp32
 // registers. Long tensor-core accumulation chains drift (measured: error
@@ -224,7 +224,8 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
 template <int BN, int MODE>
 struct Shape {
   static constexpr bool TM = token_major(MODE);
-  static constexpr int NA = TM ? (MODE == kDownTM ? 2 : 1) : ((MODE == kDown && BN > 64) ? 1 : 2);
+  static constexpr int NA = TM ? (MODE == kDownTM ? 2 : 1)
+                               : ((MODE == kLogits || (MODE == kDown && BN > 64)) ? 1 : 2);
   static constexpr int NB = TM ? 2 : (MODE == kDown ? 2 : 1);
   static constexpr int NCOL = TM ? 256 : (MODE == kDown ? 2 * BN : BN);
   static constexpr int NACC = TM ? 1 : NA;                         // accumulators per buffer
@@ -263,8 +264,8 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
     const int rest = local / p.ksplit;
     t.nb = rest / mblocks;
     t.mb = rest - t.nb * mblocks;
-    t.a0_row = t.nb * 2 * BM;
-    t.a1_row = t.a0_row + BM;
+    t.a0_row = t.nb * BM;  // one 128-row block of router rows per tile
+    t.a1_row = t.a0_row;
     t.b_row = t.mb * BN;
     t.kb0 = t.ks * p.kper;
     t.kblocks = min(p.kper, 3 * p.kbH - t.kb0);
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (e < 0 || e >= p.E) e = 0;  // zero tiles; keep the id in range
     } else if (MODE == kLogits) {
       m = (int)p.T;
-      tiles = ((p.E + 2 * BM - 1) / (2 * BM)) * ((m + BN - 1) / BN) * p.ksplit;
+      tiles = ((p.E + BM - 1) / BM) * ((m + BN - 1) / BN) * p.ksplit;
     } else {
       m = (int)p.T;
       tiles = nb_shared * ((m + BN - 1) / BN);
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (SH::NA == 2) umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescDown, acc);
               } else {
                 umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdesc, acc);
-                umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdesc, acc);
+                if (SH::NA == 2) umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdesc, acc);
               }
             }
             tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      float sum0[kSumCols], sum1[kSumCols];
+      float sum0[kSumCols];
       for (int ch = 0; ch < t.nchunks; ++ch, ++tcount) {
         const int a = tcount & 1;
         const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
@@ -667,12 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (MODE == kLogits) {
             // chunk sums stay in registers; one fp32 add per chunk per element
             tmem_ld16(taddr + c0, v0);
-            tmem_ld16(taddr + SH::NCOL + c0, v1);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 16; ++i)
               sum0[(c0 + i) % kSumCols] = ch == 0 ? v0[i] : sum0[(c0 + i) % kSumCols] + v0[i];
-              sum1[(c0 + i) % kSumCols] = ch == 0 ? v1[i] : sum1[(c0 + i) % kSumCols] + v1[i];
-            }
           } else if (MODE == kGateUp) {
             tmem_ld16(taddr + c0, v0);
             tmem_ld16(taddr + SH::NCOL + c0, v1);
@@ -718,15 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&tempty[a]);
       }
       if (MODE == kLogits && alive) {  // the tile's logits, written once
-        const int e0 = t.nb * 2 * BM + row, e1 = e0 + BM;
+        const int e0 = t.nb * BM + row;
         float* out = p.logits_out + (int64_t)t.ks * p.T * p.E;
 #pragma unroll
         for (int c = 0; c < kSumCols; ++c) {
-          if (c < mvalid) {
-            const int64_t tok = (int64_t)t.mb * BN + c;
-            if (e0 < p.E) out[tok * p.E + e0] = sum0[c];
-            if (e1 < p.E) out[tok * p.E + e1] = sum1[c];
-          }
+          if (c < mvalid && e0 < p.E) out[((int64_t)t.mb * BN + c) * p.E + e0] = sum0[c];
         }
       }
     }
@@ -880,7 +874,7 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restr
 void logits_split(int64_t T, int E, int H, int* ksplit, int* kper) {
   const int kbH = (H + BK - 1) / BK;
   const int total = 3 * kbH;
-  const int64_t tiles = (int64_t)((E + 2 * BM - 1) / (2 * BM)) * ((T + kLogitsBN - 1) / kLogitsBN);
+  const int64_t tiles = (int64_t)((E + BM - 1) / BM) * ((T + kLogitsBN - 1) / kLogitsBN);
   int want = (int)((128 + tiles - 1) / tiles);
   want = want < 1 ? 1 : (want > 24 ? 24 : want);
   if (want > total) want = total;
@@ -918,7 +912,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   m[3] = m[0];
   m[4] = m[1];
   m[5] = m[1];
-  constexpr int kStages = 5;
+  constexpr int kStages = 8;
   const size_t smem = Smem<kLogitsBN, kStages, kLogits>::kTotal;
   e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
