@@ -255,6 +255,9 @@ def run_ours(args):
     wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
+    if args.kernel == "auto":
+        fused = args.ffn_path == "auto" and T <= M.FUSED_DECODE_MAX_TOKENS
+        args.kernel = "decode_fused" if fused else "expert_gate_up"
     if rank > 0:  # each rank its own batch (weak scaling), same weights
         g = torch.Generator(device=dev)
         g.manual_seed(rank_activation_seed(rank))
@@ -337,8 +340,11 @@ def run_ours(args):
 
     pk = peaks()
     kms = statistics.mean(kern_ms)
-    kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
-    kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
+    if args.kernel == "decode_fused":  # the whole block in one kernel
+        kbytes, kflops = work["step_bytes"], work["flops"]
+    else:
+        kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
+        kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if kflops / kbytes > ridge:
@@ -398,7 +404,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(G.WORKLOADS))
-    ap.add_argument("--kernel", default="expert_gate_up", choices=["expert_gate_up", "expert_down"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "expert_gate_up", "expert_down", "decode_fused"],
+                    help="kernel whose live timing gives the roofline (auto: the fused decode kernel when the "
+                         "library runs the block as one launch, else the gate/up expert pass)")
     ap.add_argument("--cpu-sample", type=int, default=64)
     ap.add_argument("--ref-sample", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -33,6 +33,29 @@ cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_
                            cudaStream_t s);
 cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
                                const uint16_t* x, int H, uint16_t* x_perm, cudaStream_t s);
+struct DecodeArgs {
+  const uint16_t* x;
+  int T, H, E, k, I, Is, n_group, topk_group, score_fn, norm;
+  float scale;
+  const float* router_w;
+  const float* expert_bias;
+  const float* logits_override;
+  const uint16_t* w_gate_up;
+  const uint16_t* w_down;
+  const uint16_t* ws_gate_up;
+  const uint16_t* ws_down;
+  float* logits;
+  int32_t* topk_idx_out;
+  float* topk_w_out;
+  float* h;
+  float* h_shared;
+  float* y_slots;
+  float* shared_out;
+  uint16_t* y;
+  WsHeader* hdr;
+};
+bool decode_fused_supported(int64_t T, int k, int E);
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // errors, hooks, device cache
@@ -473,6 +496,40 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  if (g_ffn_path == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts)) {
+    DecodeArgs d{};
+    d.x = x;
+    d.T = (int)T;
+    d.H = c.hidden_size;
+    d.E = c.num_experts;
+    d.k = c.num_experts_per_tok;
+    d.I = c.moe_intermediate_size;
+    d.Is = shared_width(c);
+    d.n_group = c.n_group;
+    d.topk_group = c.topk_group;
+    d.score_fn = c.score_function;
+    d.norm = c.norm_topk_prob;
+    d.scale = c.routed_scaling_factor;
+    d.router_w = router_w;
+    d.expert_bias = expert_bias;
+    d.logits_override = logits_override;
+    d.w_gate_up = w_gate_up;
+    d.w_down = w_down;
+    d.ws_gate_up = has_shared ? ws_gate_up : nullptr;
+    d.ws_down = has_shared ? ws_down : nullptr;
+    d.logits = at<float>(ws, L.logits);
+    d.topk_idx_out = topk_idx_out;
+    d.topk_w_out = topk_w_out;
+    d.h = at<float>(ws, L.h_perm);
+    d.h_shared = at<float>(ws, L.h_shared);
+    d.y_slots = at<float>(ws, L.y_slots);
+    d.shared_out = at<float>(ws, L.shared_out);
+    d.y = y;
+    d.hdr = hdr;
+    cudaError_t e = launch_decode_fused(d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fused decode");
+    return MOE_OK;
+  }
   const float* logits = logits_override;
   cudaError_t e;
   if (logits == nullptr) {
@@ -508,7 +565,7 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
   e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "read error word");
   if (word[0] == 0) return MOE_OK;
-  e = cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s);
+  e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   if (word[0] == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "device wait timed out (site %d)", word[1]);

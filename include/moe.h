@@ -100,7 +100,8 @@ typedef enum {
   MOE_KERNEL_EXPERT_GATE_UP = 3, /* routed + shared gate/up projections with SwiGLU */
   MOE_KERNEL_EXPERT_DOWN = 4,    /* routed + shared down projections, weighted */
   MOE_KERNEL_COMBINE = 5,
-  MOE_KERNEL_COUNT = 6
+  MOE_KERNEL_DECODE_FUSED = 6,   /* the whole block for 1-2 tokens in one launch (moe_forward) */
+  MOE_KERNEL_COUNT = 7
 } moe_kernel_id;
 
 /* Workspace bytes moe_permute, moe_expert_ffn and moe_forward need for up to
@@ -181,6 +182,11 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
                        uint16_t* y, void* stream);
 
 /* The whole block: router logits -> route -> permute -> experts -> combine.
+ * With the automatic expert path (moe_set_ffn_path(0)) and T <= 2 tokens, the
+ * block runs as one cooperative launch (MOE_KERNEL_DECODE_FUSED) whose phases
+ * are separated by bounded grid barriers; the routing, weights and output are
+ * those of the separate kernels, up to fp32 summation order in the logits and
+ * expert dot products.
  *   logits_override [T,E] fp32 or NULL: when given, replaces the router
  *   projection (router_w may then be NULL).
  *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
@@ -192,7 +198,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
                        uint16_t* y, int32_t* topk_idx_out, float* topk_w_out,
                        void* ws, size_t ws_bytes, void* stream);
 
-/* Synchronises `stream`, reads and clears the workspace error word. Returns
+/* Synchronises `stream`, reads and clears the workspace error word (after an
+ * error the whole 256-byte header is cleared, barrier state included). Returns
  * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT (first error recorded), or
  * MOE_ERR_CUDA if the stream itself reports an error. Blocking. */
 moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);

@@ -329,6 +329,29 @@ def test_forward_skew_ties_sampled(M, over):
     _forward_and_compare(M, dict(wl, name="skew"), inp, tokens=rows, logits=L)
 
 
+FUSED_CASES = [
+    ("ling30_flash_decode_t64", {}, 1),
+    ("ling30_flash_decode_t64", dict(norm_topk_prob=False, routed_scaling_factor=1.0), 2),
+    ("ling26_flash_t512", {}, 2),
+    ("ling_lite_t64", {}, 1),
+    ("ling_lite_t64", dict(norm_topk_prob=True, routed_scaling_factor=2.5), 2),
+]
+
+
+@pytest.mark.parametrize("name,over,T", FUSED_CASES, ids=[f"{n}-T{T}-{i}" for i, (n, _, T) in enumerate(FUSED_CASES)])
+def test_fused_decode(M, name, over, T):
+    # one launch for 1-2 tokens: routing bit-exact on given logits, output
+    # against the oracle, and the same routing when it computes the logits
+    wl, inp = _inputs(name)
+    wl = dict(wl, **over, name=f"fused-{name}")
+    sub = dict(inp, x=inp["x"][7:7 + T].contiguous(), tokens=T)
+    L = G.random_logits(T, wl["num_experts"], S.logit_std(wl), seed=11).numpy()
+    n0 = M.launch_count()
+    _forward_and_compare(M, wl, sub, logits=L)
+    assert M.launch_count() - n0 == 1, "the fused decode is a single launch"
+    _forward_and_compare(M, wl, sub)
+
+
 def test_forward_deterministic(M):
     wl, inp = _inputs("ling26_flash_t512")
     ws = M.Workspace(wl, inp["tokens"])
