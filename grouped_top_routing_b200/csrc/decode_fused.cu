@@ -3,69 +3,200 @@
 // At decode the block is bound by HBM bandwidth: it must stream the router
 // weight and the weights of the few selected experts ("only the selected
 // experts are read", page "Ling-3.0-flash-GGUF", section "Measured
-// performance") plus the shared MLP. As separate kernels the chain of six
-// launches, each a few microseconds of latency, dominates the ~20 us of
-// streaming. Here one cooperative grid (every CTA resident) runs the steps as
-// phases separated by grid barriers:
+// performance") plus the shared MLP, ~120 MB for Ling-3.0-flash, against a few
+// microseconds of arithmetic. The kernel is therefore a weight-streaming
+// engine: one CTA per SM, a producer thread that keeps a ring of shared-memory
+// stages filled with untiled bulk copies (cp.async.bulk, mbarrier completion),
+// and eight consumer warps that each take whole stages and reduce them with
+// the token rows. A stage holds 4H bytes: one fp32 router row, or one bf16
+// gate row plus the matching up row, or a block of down-projection rows.
 //
-//   A  router logits (one warp per router row, fp32 FMA) and the shared MLP's
-//      gate/up rows (they do not depend on the routing)            -> barrier
-//   B  every CTA routes the 1-2 tokens itself (route_one_token, the router
-//      kernel's own code) and lists the selected experts in shared memory:
-//      no barrier needed, each CTA already holds the routing
-//   C  gate/up rows of the selected experts, SwiGLU in fp32         -> barrier
-//   D  down rows of the selected experts (weighted by the routing) and of the
-//      shared MLP, fp32 per slot                                    -> barrier
-//   E  combine: y = bf16(sum of the k slot rows + the shared row), slot order
+// Every phase's rows are split evenly into one contiguous range per CTA, and
+// each CTA streams its ranges in this order:
 //
-// Data written in one phase and read in a later one by other CTAs is read
-// with ld.global.cg (L2), never through the read-only path. Each grid barrier
-// is bounded (globaltimer, ~2 s): a barrier that runs out records
-// MOE_ERR_TIMEOUT in the workspace and the CTA returns.
-#include "common.cuh"
+//   A  router rows (logits, fp32 FMA) and the shared MLP's gate/up rows
+//                                                            -> grid barrier
+//   S  the shared MLP's down rows: their copies start during the barrier and
+//      the routing, since they do not depend on it
+//   (every CTA routes the 1-2 tokens itself with all consumer warps: no
+//    second barrier; the producer then learns the selected experts)
+//   C  gate/up rows of the selected experts, SwiGLU in fp32; each warp adds
+//      its rows to a per-expert completion counter
+//   D  down rows of the selected experts, weighted by the routing; a block
+//      starts once its expert's counter shows all of h
+//
+// Each output row y[t, n] counts its k + 1 contributions (k slot rows and the
+// shared row); the lane that brings the last one sums them in slot order and
+// rounds once to bf16. Counters are released with a fence after the rows they
+// cover; data written in this launch is read through L2 (ld.global.cg). Every
+// wait is bounded (globaltimer, ~2 s): one that runs out records
+// MOE_ERR_TIMEOUT in the workspace and returns; the producer first waits
+// (bounded) for its copies in flight, so no copy lands after its CTA exits.
+//
+// Routing takes the same decisions as the per-token router kernel (route.cuh):
+// the same fp64 score evaluation rounded once to fp32, the same softmax sum
+// association, group scores from the multiset top-2 of each group, and the
+// top-k by (biased score descending, expert id ascending) found by ranking
+// unique 64-bit keys, first within each warp's slice of experts, then among
+// the slices' survivors, which is exact for a total order. Pages: mlxcel issue
+// #838 "add Ant Group Ling / Bailing MoE", section "Router: selection uses
+// biased scores, weights come from unbiased scores", and the model card
+// "Ling-2.6-flash-JANGTQ", paragraph "MoE routing".
+#include "decode_fused.cuh"
+#include "mbarrier.cuh"
 #include "route.cuh"
 
 namespace moe {
 
-struct DecodeArgs {
-  const uint16_t* x;  // [T, H]
-  int T, H, E, k, I, Is, n_group, topk_group, score_fn, norm;
-  float scale;
-  const float* router_w;         // [E, H] or null when logits are given
-  const float* expert_bias;      // [E] or null
-  const float* logits_override;  // [T, E] or null
-  const uint16_t* w_gate_up;     // [E, 2I, H]
-  const uint16_t* w_down;        // [E, H, I]
-  const uint16_t* ws_gate_up;    // [2Is, H] or null
-  const uint16_t* ws_down;       // [H, Is]
-  float* logits;                 // [T, E] workspace
-  int32_t* topk_idx_out;         // [T, k] or null
-  float* topk_w_out;             // [T, k] or null
-  float* h;                      // [T*k, I] workspace
-  float* h_shared;               // [T, Is] workspace
-  float* y_slots;                // [T*k, H] workspace
-  float* shared_out;             // [T, H] workspace
-  uint16_t* y;                   // [T, H] output
-  WsHeader* hdr;
-};
-
 namespace {
 
-constexpr int kFusedThreads = 256;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kFusedThreads = kConsumers + 32;  // + the producer warp
 constexpr int kFusedMaxT = 2;
-constexpr int kDownRows = 8;
-constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
+constexpr int kMaxSlots = 32;      // T * k: one warp lane per slot
+constexpr int kMaxChunk = 8;       // experts per lane in a warp's slice: 1024 / (4 warps * 32 lanes)
+constexpr int kMaxStages = 16;
+constexpr int kMinStages = 4;
+constexpr int kMaxDownRows = 16;   // rows per down block: lane t*16 + r holds (slot or token t, row r)
+constexpr int kMaxHidden = 8192;   // a stage (4H bytes) must leave room for kMinStages
+constexpr int kSmemBudget = 227 * 1024;
+constexpr uint64_t kWaitNs = 2000000000ull;
 
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
+// Stream geometry, the same on host and device.
+struct Geo {
+  int stage_bytes;  // 4H
+  int depth;        // ring stages
+  int rd, rs;       // rows per routed / shared down block
+  int nblk, nsblk;  // down blocks per expert / of the shared MLP
+};
+
+struct FusedSmem {
+  uint64_t full[kMaxStages], empty[kMaxStages], route_ready;
+  // Stage tags: the stream index a slot was last filled with. Consumer warps
+  // run ahead of one another, so a warp can reach a slot while the slot's
+  // previous fill is still in flight, when its parity would read as the phase
+  // the warp waits for; the tag shows which fill is pending.
+  volatile uint32_t tag[kMaxStages];
+  uint64_t cand[kFusedMaxT][kConsumerWarps * kMaxSlots];  // per-slice survivors (64-bit keys)
+  uint32_t gkey[kFusedMaxT][32];                          // group score keys
+  uint32_t kept[kFusedMaxT];                              // kept-group masks
+  float red[kFusedMaxT][kConsumerWarps];
+  double sum[kFusedMaxT];
+  int32_t idx[kMaxSlots];  // slot -> expert
+  float w_raw[kMaxSlots];  // unbiased score of the slot's expert
+  float w[kMaxSlots];      // routing weight
+  int32_t act_e[kMaxSlots], act_a[kMaxSlots], act_b[kMaxSlots];  // distinct expert, first slot, second slot or -1
+  int n_act;
+  int flag;
+  volatile int abort;  // a consumer warp stopped before the grid barrier
+};
+
+struct Range {
+  int lo, n;
+};
+
+// Dynamic shared memory after the ring: routing scratch ([T*E] fp32 scores,
+// [T*E] fp32 biased scores, [T*E] 64-bit keys), then the token rows (bf16)
+// and the expert bias (fp32).
+__host__ __device__ __forceinline__ size_t route_scratch_bytes(int T, int E) { return (size_t)T * E * 16; }
+__host__ __device__ __forceinline__ size_t scratch_bytes(int T, int E, int H) {
+  return route_scratch_bytes(T, E) + (size_t)T * H * 2 + (size_t)E * 4;
 }
 
-// Grid-wide barrier over gridDim.x CTAs (sense by generation). Returns false
-// if it timed out. Writes before it are visible to ld.global.cg after it.
+// Contiguous share b of G of `total` items.
+__host__ __device__ __forceinline__ Range split(int total, int b, int G) {
+  const int lo = (int)((int64_t)total * b / G), hi = (int)((int64_t)total * (b + 1) / G);
+  return {lo, hi - lo};
+}
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+// Bounded wait for the phase of `bar` with the given parity, by every lane of
+// the warp; false (in every lane) after recording a timeout.
+__device__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+  int ok = 1;
+  if (!mbar_try_wait(bar, parity)) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+      if (globaltimer() - t0 > kWaitNs) {
+        ok = 0;
+        break;
+      }
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
+  return ok != 0;
+}
+
+// Bounded wait until the producer tagged slot `tag` with stream index v.
+__device__ bool warp_wait_tag(volatile uint32_t* tag, uint32_t v, WsHeader* hdr, int site) {
+  int ok = 1;
+  if (*tag != v) {
+    const uint64_t t0 = globaltimer();
+    while (*tag != v) {
+      if (globaltimer() - t0 > kWaitNs) {
+        ok = 0;
+        break;
+      }
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
+  return ok != 0;
+}
+
+// Single-thread bounded wait (producer side).
+__device__ bool thread_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitNs) {
+      if (hdr != nullptr) record_error(hdr, MOE_ERR_TIMEOUT, site);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Lane 0 waits (bounded) until *ctr >= target; the whole warp then sees every
+// write released before the increments. False after recording a timeout.
+__device__ bool warp_wait_count(const int32_t* ctr, int target, WsHeader* hdr, int site) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && ld_acquire(ctr) < target) {
+    const uint64_t t0 = globaltimer();
+    while (ld_acquire(ctr) < target) {
+      if (globaltimer() - t0 > kWaitNs) {
+        record_error(hdr, MOE_ERR_TIMEOUT, site);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// Grid-wide barrier of the consumer threads of every CTA (sense by
+// generation). False if it timed out. Writes before it are visible to
+// ld.global.cg after it.
 __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
-  __syncthreads();
+  consumer_sync();
   if (threadIdx.x == 0) {
     int ok = 1;
     volatile uint32_t* gen = &hdr->bar_gen;
@@ -77,9 +208,9 @@ __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
       __threadfence();
       atomicAdd(&hdr->bar_gen, 1u);
     } else {
-      const uint64_t t0 = gtimer();
+      const uint64_t t0 = globaltimer();
       while (*gen == g) {
-        if (gtimer() - t0 > kBarrierTimeoutNs) {
+        if (globaltimer() - t0 > kWaitNs) {
           record_error(hdr, MOE_ERR_TIMEOUT, 100 + site);
           ok = 0;
           break;
@@ -89,282 +220,759 @@ __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
     __threadfence();
     *s_flag = ok;
   }
-  __syncthreads();
+  consumer_sync();
   return *s_flag != 0;
 }
 
-__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
 
-// silu(gate . x_t) * (up . x_t) for up to two token rows against one pair of
-// gate/up weight rows (H bf16 each), fp32. One warp; every lane gets the sums.
-__device__ __forceinline__ void gate_up_dot(const uint16_t* __restrict__ gate, const uint16_t* __restrict__ up,
-                                            const uint16_t* x0, const uint16_t* x1, int H, float* h0, float* h1) {
+// Warp reduce-scatter of N (a power of two <= 32) values per lane: returns the
+// warp total of value `which`, with which = lane >> (5 - log2 N) (the lane's
+// top log2 N bits). log2 N halving steps, then a butterfly over the rest:
+// N - 1 + 5 - log2 N shuffles instead of 5 N.
+template <int N>
+__device__ __forceinline__ float reduce_scatter(float (&v)[N]) {
   const int lane = threadIdx.x & 31;
-  const int nv = H / 8;
-  float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
-  for (int v0 = lane; v0 < nv; v0 += 32 * 8) {
-    uint4 gv[8], uv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = v0 + 32 * u;
-      if (v < nv) {
-        gv[u] = ld_stream_u4(gate + v * 8);
-        uv[u] = ld_stream_u4(up + v * 8);
-      }
-    }
+  for (int step = 0; step < ilog2(N); ++step) {
+    const int o = 16 >> step, n = N >> step;
+    const bool up = (lane & o) != 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = v0 + 32 * u;
-      if (v < nv) {
-        float xf[8];
-        unpack8_bf16(ld_nc_u4(x0 + v * 8), xf);
-        g0 = dot8_bf16(gv[u], xf, g0);
-        u0 = dot8_bf16(uv[u], xf, u0);
-        if (x1 != nullptr) {
-          unpack8_bf16(ld_nc_u4(x1 + v * 8), xf);
-          g1 = dot8_bf16(gv[u], xf, g1);
-          u1 = dot8_bf16(uv[u], xf, u1);
-        }
-      }
+    for (int i = 0; i < n / 2; ++i) {
+      const float keep = up ? v[i + n / 2] : v[i];
+      const float give = up ? v[i] : v[i + n / 2];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, give, o);
     }
   }
-  g0 = warp_sum(g0);
-  u0 = warp_sum(u0);
-  *h0 = silu_f32(g0) * u0;
-  if (x1 != nullptr) {
-    g1 = warp_sum(g1);
-    u1 = warp_sum(u1);
-    *h1 = silu_f32(g1) * u1;
-  }
+#pragma unroll
+  for (int o = 16 >> ilog2(N); o > 0; o >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+  return v[0];
 }
 
-// kDownRows rows (K bf16 each) of a down projection against up to two fp32
-// h rows (written earlier in this launch: read through L2). Lane r*2 + t ends
-// up holding the dot of row r with h row t.
-__device__ __forceinline__ float down_dot(const uint16_t* __restrict__ w0, int nrows, int K, const float* hr0,
-                                          const float* hr1) {
-  const int lane = threadIdx.x & 31;
-  const int nvk = K / 8;
-  float acc[kDownRows][2];
-#pragma unroll
-  for (int r = 0; r < kDownRows; ++r) acc[r][0] = acc[r][1] = 0.f;
-  for (int v = lane; v < nvk; v += 32) {
-    uint4 wv[kDownRows];
-#pragma unroll
-    for (int r = 0; r < kDownRows; ++r)
-      if (r < nrows) wv[r] = ld_stream_u4(w0 + (int64_t)r * K + v * 8);
-    const float4 a0 = ldcg4(hr0 + v * 8), a1 = ldcg4(hr0 + v * 8 + 4);
-    const float f0[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-    for (int r = 0; r < kDownRows; ++r)
-      if (r < nrows) acc[r][0] = dot8_bf16(wv[r], f0, acc[r][0]);
-    if (hr1 != nullptr) {
-      const float4 b0 = ldcg4(hr1 + v * 8), b1 = ldcg4(hr1 + v * 8 + 4);
-      const float f1[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int r = 0; r < kDownRows; ++r)
-        if (r < nrows) acc[r][1] = dot8_bf16(wv[r], f1, acc[r][1]);
-    }
-  }
-  float mine = 0.f;
-#pragma unroll
-  for (int r = 0; r < kDownRows; ++r)
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (r < nrows && (t == 0 || hr1 != nullptr)) {
-        const float s = warp_sum(acc[r][t]);
-        if (lane == r * 2 + t) mine = s;
-      }
-    }
-  return mine;
+// Frees a stage once every lane of the warp has read it.
+__device__ __forceinline__ void release_stage(uint64_t* empty) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
 }
 
-template <int P>
-__global__ void __launch_bounds__(kFusedThreads) decode_fused_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int T = a.T, E = a.E, k = a.k, H = a.H, I = a.I, Is = a.Is;
+// Products of one 16-byte bf16 weight chunk with 8 fp32 values, added to two
+// accumulators (even and odd elements): each dependent chain is half as long.
+__device__ __forceinline__ void dot8x2(uint4 w, const float* v, float& e, float& o) {
+  e = fmaf(bf16_lo(w.x), v[0], e);
+  o = fmaf(bf16_hi(w.x), v[1], o);
+  e = fmaf(bf16_lo(w.y), v[2], e);
+  o = fmaf(bf16_hi(w.y), v[3], o);
+  e = fmaf(bf16_lo(w.z), v[4], e);
+  o = fmaf(bf16_hi(w.z), v[5], o);
+  e = fmaf(bf16_lo(w.w), v[6], e);
+  o = fmaf(bf16_hi(w.w), v[7], o);
+}
+
+// ---------------------------------------------------------------------------
+// Stage consumers (one warp each). Lane l takes the 16-byte columns l, l + 32,
+// ... of a row: contiguous across the warp, so shared-memory reads are free of
+// bank conflicts. Token rows x come from the shared-memory copy made at
+// kernel start; h rows (written in this launch) through L2.
+// ---------------------------------------------------------------------------
+
+// One fp32 router row (H) against up to two bf16 token rows. Returns the logit
+// of token 0 in lane 0 and of token 1 in lane 16.
+__device__ __forceinline__ float router_unit(const float* w, int H, const uint16_t* xs, int T, uint64_t* empty) {
+  const int lane = threadIdx.x & 31;
+  const uint2* x0 = reinterpret_cast<const uint2*>(xs);
+  const uint2* x1 = reinterpret_cast<const uint2*>(xs + H);
+  float e0 = 0.f, o0 = 0.f, e1 = 0.f, o1 = 0.f;
+#pragma unroll 2
+  for (int c = lane; c < H / 4; c += 32) {
+    const float4 w4 = reinterpret_cast<const float4*>(w)[c];
+    const uint2 xa = x0[c];
+    e0 = fmaf(bf16_lo(xa.x), w4.x, e0);
+    o0 = fmaf(bf16_hi(xa.x), w4.y, o0);
+    e0 = fmaf(bf16_lo(xa.y), w4.z, e0);
+    o0 = fmaf(bf16_hi(xa.y), w4.w, o0);
+    if (T > 1) {
+      const uint2 xb = x1[c];
+      e1 = fmaf(bf16_lo(xb.x), w4.x, e1);
+      o1 = fmaf(bf16_hi(xb.x), w4.y, o1);
+      e1 = fmaf(bf16_lo(xb.y), w4.z, e1);
+      o1 = fmaf(bf16_hi(xb.y), w4.w, o1);
+    }
+  }
+  release_stage(empty);
+  float v[2] = {e0 + o0, e1 + o1};
+  return reduce_scatter<2>(v);
+}
+
+// One gate row and one up row (H bf16 each) against up to two token rows:
+// returns silu(gate . x_t) * (up . x_t) for token row 0 in lane 0 and for
+// token row 1 in lane 16, fp32.
+__device__ __forceinline__ float gate_up_unit(const uint16_t* gate, const uint16_t* up, int H, const uint16_t* x0,
+                                              const uint16_t* x1, uint64_t* empty) {
+  const int lane = threadIdx.x & 31;
+  float ve[4] = {0.f, 0.f, 0.f, 0.f}, vo[4] = {0.f, 0.f, 0.f, 0.f};  // gate . x0, up . x0, gate . x1, up . x1
+#pragma unroll 2
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 gv = reinterpret_cast<const uint4*>(gate)[c];
+    const uint4 uv = reinterpret_cast<const uint4*>(up)[c];
+    float xf[8];
+    unpack8_bf16(reinterpret_cast<const uint4*>(x0)[c], xf);
+    dot8x2(gv, xf, ve[0], vo[0]);
+    dot8x2(uv, xf, ve[1], vo[1]);
+    if (x1 != nullptr) {
+      unpack8_bf16(reinterpret_cast<const uint4*>(x1)[c], xf);
+      dot8x2(gv, xf, ve[2], vo[2]);
+      dot8x2(uv, xf, ve[3], vo[3]);
+    }
+  }
+  release_stage(empty);
+  float v[4] = {ve[0] + vo[0], ve[1] + vo[1], ve[2] + vo[2], ve[3] + vo[3]};
+  const float s = reduce_scatter<4>(v);                     // lane >> 3 = 2 t + (0 gate, 1 up)
+  const float up_sum = __shfl_xor_sync(0xffffffffu, s, 8);  // the up sum sits 8 lanes above the gate sum
+  return silu_f32(s) * up_sum;
+}
+
+// One 8-column chunk of up to two fp32 h rows (h1 null: the h0 values again).
+struct HChunk {
+  float4 a0, a1, b0, b1;
+};
+
+__device__ __forceinline__ HChunk load_h(const float* h0, const float* h1, int c, int nc) {
+  HChunk p;
+  if (c < nc) {
+    p.a0 = ldcg4(h0 + c * 8);
+    p.a1 = ldcg4(h0 + c * 8 + 4);
+    p.b0 = p.a0;
+    p.b1 = p.a1;
+    if (h1 != nullptr) {
+      p.b0 = ldcg4(h1 + c * 8);
+      p.b1 = ldcg4(h1 + c * 8 + 4);
+    }
+  } else {
+    p.a0 = p.a1 = p.b0 = p.b1 = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  return p;
+}
+
+// nrows (<= 16) rows of K bf16 against up to two fp32 h rows. `first` holds
+// this lane's first h chunk, loaded before the stage was waited on; each later
+// chunk is loaded one step ahead. Returns the dot of row r with h row t in
+// lane t*16 + r.
+__device__ __forceinline__ float down_unit(const uint16_t* w, int nrows, int K, const float* h0, const float* h1,
+                                           HChunk first, uint64_t* empty) {
+  const int lane = threadIdx.x & 31;
+  const int nc = K / 8;
+  const bool two = h1 != nullptr;
+  float acc[2 * kMaxDownRows];
+#pragma unroll
+  for (int i = 0; i < 2 * kMaxDownRows; ++i) acc[i] = 0.f;
+  HChunk cur = first;
+#pragma unroll 1
+  for (int c = lane; c < nc; c += 32) {
+    const HChunk nxt = load_h(h0, h1, c + 32, nc);
+    const float f0[8] = {cur.a0.x, cur.a0.y, cur.a0.z, cur.a0.w, cur.a1.x, cur.a1.y, cur.a1.z, cur.a1.w};
+    const float f1[8] = {cur.b0.x, cur.b0.y, cur.b0.z, cur.b0.w, cur.b1.x, cur.b1.y, cur.b1.z, cur.b1.w};
+#pragma unroll
+    for (int r = 0; r < kMaxDownRows; ++r) {
+      if (r < nrows) {
+        const uint4 wv = reinterpret_cast<const uint4*>(w + (size_t)r * K)[c];
+        acc[r] = dot8_bf16(wv, f0, acc[r]);
+        if (two) acc[kMaxDownRows + r] = dot8_bf16(wv, f1, acc[kMaxDownRows + r]);
+      }
+    }
+    cur = nxt;
+  }
+  release_stage(empty);
+  return reduce_scatter<2 * kMaxDownRows>(acc);
+}
+
+// Contributions to output rows a warp has stored but not yet counted (entry j
+// of lane l: the counter index tok*H + row of that lane's row in the warp's
+// j-th pending down block, or -1). They are counted whenever the warp is about
+// to block, when the list is full and at the warp's end: one fence covers
+// several blocks, and no warp waits while holding uncounted work.
+constexpr int kMaxPend = 4;
+struct Pending {
+  int pend[kMaxPend];
+  int np;  // warp-uniform number of pending down blocks
+};
+
+// y[tok, row] = bf16(sum of the k slot rows in slot order + the shared row).
+__device__ __forceinline__ void combine_row(const DecodeArgs& a, int idx) {
+  const int tok = idx / a.H, row = idx - tok * a.H;
+  float acc = 0.f;
+  for (int j = 0; j < a.k; ++j) acc += __ldcg(a.y_slots + (int64_t)(tok * a.k + j) * a.H + row);
+  if (a.ws_down != nullptr) acc += __ldcg(a.shared_out + (int64_t)tok * a.H + row);
+  a.y[idx] = f32_to_bf16(acc);
+}
+
+// Count the pending contributions: one fence, then the counter increments;
+// the lane that brings the last of an output row's k + 1 contributions
+// combines it.
+__device__ __forceinline__ void publish(const DecodeArgs& a, Pending& q, int target) {
+  __syncwarp();
+  __threadfence();
+  int32_t* rb_cnt = a.sync + kMaxSlots;
+  int last = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxPend; ++j)
+    if (j < q.np && q.pend[j] >= 0 && atomicAdd(rb_cnt + q.pend[j], 1) == target - 1) last |= 1 << j;
+  if (last != 0) {
+    __threadfence();
+#pragma unroll
+    for (int j = 0; j < kMaxPend; ++j)
+      if ((last >> j) & 1) combine_row(a, q.pend[j]);
+  }
+  q.np = 0;
+}
+
+__device__ __forceinline__ void add_pending(Pending& q, int idx) {
+#pragma unroll
+  for (int j = 0; j < kMaxPend; ++j)
+    if (j == q.np) q.pend[j] = idx;
+  ++q.np;
+}
+
+// ---------------------------------------------------------------------------
+// Routing with the consumer warps
+// ---------------------------------------------------------------------------
+
+// Unique selection key: the order key of the biased score above the
+// complemented expert id, so that a larger key is a higher score or, on a tie,
+// a lower id. Real keys are > 0 (the order key of -inf is 0x007fffff).
+__device__ __forceinline__ uint64_t sel_key(float s, int e) {
+  return ((uint64_t)route_detail::order_key(s) << 32) | (uint64_t)(~(uint32_t)e);
+}
+
+// Level 1: this warp's slice [e0, e1) of token t's experts; lane l holds the
+// keys of experts e0 + l + 32 r. Each key's rank is the number of keys of the
+// slice above it; the ones ranked below k are stored at their rank.
+template <int R>
+__device__ __forceinline__ void rank_slice(const uint64_t* key, int e0, int e1, int k, uint64_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint64_t mine[R];
+  int rank[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = e0 + lane + 32 * r;
+    mine[r] = e < e1 ? key[e] : 0ull;
+    rank[r] = 0;
+  }
+#pragma unroll 4
+  for (int j = e0; j < e1; ++j) {
+    const uint64_t kj = key[j];  // the same address in every lane: a broadcast
+#pragma unroll
+    for (int r = 0; r < R; ++r) rank[r] += kj > mine[r] ? 1 : 0;
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (e0 + lane + 32 * r < e1 && rank[r] < k) out[rank[r]] = mine[r];
+}
+
+// Routes the T tokens with the consumer warps; results land in sm (slot
+// experts, weights, the distinct experts with their slots). Ends synchronised.
+// bias: the expert bias in shared memory, or null. Scratch: [T*E] fp32
+// scores, [T*E] fp32 biased scores, [T*E] 64-bit keys (first used for the
+// softmax exponentials).
+__device__ void route_block(const DecodeArgs& a, const float* logits, const float* bias, unsigned char* scratch,
+                            FusedSmem& sm) {
+  using namespace route_detail;
+  const int T = a.T, E = a.E, k = a.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gw = blockIdx.x * (kFusedThreads / 32) + warp;
-  const int nw = gridDim.x * (kFusedThreads / 32);
-  // shared memory: per-token route scratch, routing, slot table, active list
-  float* rbuf = reinterpret_cast<float*>(smem_raw);                       // [kFusedMaxT][32*P]
-  int32_t* s_idx = reinterpret_cast<int32_t*>(rbuf + kFusedMaxT * 32 * P);  // [T*k]
-  float* s_w = reinterpret_cast<float*>(s_idx + kFusedMaxT * E);          // [T*k]
-  int32_t* s_slot = reinterpret_cast<int32_t*>(s_w + kFusedMaxT * E);     // [T][E]: slot of expert e, or -1
-  int32_t* s_active = s_slot + kFusedMaxT * E;                            // [E]
-  int* s_misc = s_active + E;                                             // [0] n_active, [1] barrier flag, [2..] scan
+  float* s_orig = reinterpret_cast<float*>(scratch);
+  float* s_sel = s_orig + T * E;
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_sel + T * E);
+  double* s_ex = reinterpret_cast<double*>(s_key);
 
-  // ---- A: router logits and the shared MLP's gate/up rows ----
-  const int n_router = a.logits_override == nullptr ? E : 0;
-  const int n_shared = a.ws_gate_up != nullptr ? Is : 0;
-  const float* logits = a.logits_override != nullptr ? a.logits_override : a.logits;
-  for (int item = gw; item < n_router + n_shared; item += nw) {
-    if (item < n_router) {
-      const float* wr = a.router_w + (int64_t)item * H;
-      float acc0 = 0.f, acc1 = 0.f;
-      for (int h4 = lane; h4 < H / 4; h4 += 32) {
-        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr) + h4);
-        const uint2 xa = __ldg(reinterpret_cast<const uint2*>(a.x) + h4);
-        acc0 = fmaf(bf16_lo(xa.x), w4.x, acc0);
-        acc0 = fmaf(bf16_hi(xa.x), w4.y, acc0);
-        acc0 = fmaf(bf16_lo(xa.y), w4.z, acc0);
-        acc0 = fmaf(bf16_hi(xa.y), w4.w, acc0);
-        if (T > 1) {
-          const uint2 xb = __ldg(reinterpret_cast<const uint2*>(a.x + H) + h4);
-          acc1 = fmaf(bf16_lo(xb.x), w4.x, acc1);
-          acc1 = fmaf(bf16_hi(xb.x), w4.y, acc1);
-          acc1 = fmaf(bf16_lo(xb.y), w4.z, acc1);
-          acc1 = fmaf(bf16_hi(xb.y), w4.w, acc1);
+  // ---- scores: fp64 evaluation, one rounding to fp32; selection copy with the bias ----
+  if (a.score_fn != MOE_SCORE_SOFTMAX) {
+    for (int t = 0; t < T; ++t)
+      for (int e = threadIdx.x; e < E; e += kConsumers) {
+        const float L = __ldcg(logits + (int64_t)t * E + e);
+        const float o = __double2float_rn(1.0 / (1.0 + exp(-(double)L)));
+        s_orig[t * E + e] = o;
+        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
+      }
+  } else {
+    float m[kFusedMaxT] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t)
+      if (t < T)
+        for (int e = threadIdx.x; e < E; e += kConsumers) {
+          const float L = __ldcg(logits + (int64_t)t * E + e);
+          s_orig[t * E + e] = L;
+          m[t] = fmaxf(m[t], L);
+        }
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t) {
+      const float mt = warp_max_f32(m[t]);
+      if (lane == 0 && t < T) sm.red[t][warp] = mt;
+    }
+    consumer_sync();
+    for (int t = 0; t < T; ++t) {
+      float mt = sm.red[t][0];
+      for (int w = 1; w < kConsumerWarps; ++w) mt = fmaxf(mt, sm.red[t][w]);
+      const double md = (double)mt;
+      for (int e = threadIdx.x; e < E; e += kConsumers) s_ex[t * E + e] = exp((double)s_orig[t * E + e] - md);
+    }
+    consumer_sync();
+    if (warp < T) {
+      // the per-token router's association: lane l sums experts l*P .. l*P+P-1
+      int P = 1;
+      while (P * 32 < E) P <<= 1;
+      double sum = 0.0;
+      for (int i = 0; i < P; ++i) {
+        const int e = lane * P + i;
+        if (e < E) sum += s_ex[warp * E + e];
+      }
+      sum = warp_sum_f64(sum);
+      if (lane == 0) sm.sum[warp] = sum;
+    }
+    consumer_sync();
+    for (int t = 0; t < T; ++t)
+      for (int e = threadIdx.x; e < E; e += kConsumers) {
+        const float o = __double2float_rn(s_ex[t * E + e] / sm.sum[t]);
+        s_orig[t * E + e] = o;
+        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
+      }
+  }
+  consumer_sync();
+
+  // ---- groups: score = top1 + top2 of the group's biased scores; keep topk_group ----
+  const bool grouped = a.n_group > 1 && a.topk_group < a.n_group;
+  const int gsz = E / a.n_group;
+  if (grouped) {
+    for (int p = warp; p < T * a.n_group; p += kConsumerWarps) {
+      const int t = p / a.n_group, g = p - t * a.n_group;
+      const float* gv = s_sel + t * E + g * gsz;
+      float top1 = -INFINITY, top2 = -INFINITY;  // NaN never enters: it fails both comparisons
+      for (int i = lane; i < gsz; i += 32) {
+        const float v = gv[i];
+        if (v > top1) {
+          top2 = top1;
+          top1 = v;
+        } else if (v > top2) {
+          top2 = v;
         }
       }
-      acc0 = warp_sum(acc0);
-      if (T > 1) acc1 = warp_sum(acc1);
-      if (lane == 0) {
-        a.logits[item] = acc0;
-        if (T > 1) a.logits[E + item] = acc1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {  // multiset top-2 of two lanes' pairs
+        const float b1 = __shfl_xor_sync(0xffffffffu, top1, o), b2 = __shfl_xor_sync(0xffffffffu, top2, o);
+        if (b1 > top1) {
+          top2 = fmaxf(top1, b2);
+          top1 = b1;
+        } else {
+          top2 = fmaxf(top2, b1);
+        }
       }
-    } else {
-      const int j = item - n_router;
-      const uint16_t* gate = a.ws_gate_up + (int64_t)j * H;
-      float h0, h1;
-      gate_up_dot(gate, gate + (int64_t)Is * H, a.x, T > 1 ? a.x + H : nullptr, H, &h0, &h1);
-      if (lane == 0) {
-        a.h_shared[j] = h0;
-        if (T > 1) a.h_shared[Is + j] = h1;
+      if (lane == 0) sm.gkey[t][g] = order_key(gsz == 1 ? top1 : __fadd_rn(top1, top2));
+    }
+    consumer_sync();
+    if (warp < T) {
+      const uint32_t gk = lane < a.n_group ? sm.gkey[warp][lane] : 0u;
+      uint32_t kept = 0;
+      for (int r = 0; r < a.topk_group; ++r) {
+        const uint32_t key = ((kept >> lane) & 1u) ? 0u : gk;
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, key);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, key == mx ? (uint32_t)lane : 0xffffffffu);
+        kept |= 1u << win;
+      }
+      if (lane == 0) sm.kept[warp] = kept;
+    }
+    consumer_sync();
+  }
+
+  // ---- selection keys (experts of dropped groups select as -inf) ----
+  for (int t = 0; t < T; ++t) {
+    const uint32_t kept = grouped ? sm.kept[t] : 0xffffffffu;
+    for (int e = threadIdx.x; e < E; e += kConsumers) {
+      const bool live = !grouped || ((kept >> (e / gsz)) & 1u);
+      s_key[t * E + e] = sel_key(live ? s_sel[t * E + e] : -INFINITY, e);
+    }
+  }
+  consumer_sync();
+
+  // ---- level 1: the k best of each warp's slice of its token's experts ----
+  const int wpt = kConsumerWarps / T;
+  {
+    const int t = warp / wpt, wl = warp - t * wpt;
+    const int chunk = (E + wpt - 1) / wpt;
+    const int e0 = min(E, wl * chunk), e1 = min(E, e0 + chunk);
+    uint64_t* out = sm.cand[t] + wl * k;
+    const int per = (e1 - e0 + 31) / 32;
+    if (per <= 2) rank_slice<2>(s_key + t * E, e0, e1, k, out);
+    else if (per <= 4) rank_slice<4>(s_key + t * E, e0, e1, k, out);
+    else rank_slice<kMaxChunk>(s_key + t * E, e0, e1, k, out);
+    for (int j = min(k, e1 - e0) + lane; j < k; j += 32) out[j] = 0ull;  // fewer experts than k: padding
+  }
+  consumer_sync();
+
+  // ---- level 2: rank the survivors of the token's slices; rank j is slot j ----
+  {
+    const int per_tok = kConsumers / T;
+    const int t = threadIdx.x / per_tok, c = threadIdx.x - t * per_tok;
+    const int nc = wpt * k;
+    if (c < nc) {
+      const uint64_t mine = sm.cand[t][c];
+      if (mine != 0ull) {
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < nc; ++j) rank += sm.cand[t][j] > mine ? 1 : 0;
+        if (rank < k) {
+          const int e = (int)(~(uint32_t)mine);
+          sm.idx[t * k + rank] = e;
+          sm.w_raw[t * k + rank] = s_orig[t * E + e];
+        }
       }
     }
   }
-  if (!grid_barrier(a.hdr, 1, s_misc + 1)) return;
+  consumer_sync();
 
-  // ---- B: every CTA routes the tokens and lists the selected experts ----
-  for (int i = threadIdx.x; i < kFusedMaxT * E; i += blockDim.x) s_slot[i] = -1;
-  if (warp < T)
-    route_one_token<P, true>(logits + (int64_t)warp * E, a.expert_bias, E, k, a.n_group, a.topk_group, a.score_fn,
-                             a.norm, a.scale, rbuf + warp * 32 * P, s_idx + warp * k, s_w + warp * k);
-  __syncthreads();
-  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-    const int t = i / k, e = s_idx[i];
-    s_slot[t * E + e] = i;  // ids are valid and distinct per token
-    if (blockIdx.x == 0) {
-      if (a.topk_idx_out != nullptr) a.topk_idx_out[i] = e;
-      if (a.topk_w_out != nullptr) a.topk_w_out[i] = s_w[i];
+  // ---- weights: renormalise (k > 1) with the 1e-20 epsilon, then scale; fp32, slot order ----
+  if (warp < T) {
+    const int t = warp;
+    const bool do_norm = a.norm && k > 1;
+    float den = 0.f;
+    if (do_norm) {
+      if (lane == 0) {
+        den = sm.w_raw[t * k];
+        for (int j = 1; j < k; ++j) den = __fadd_rn(den, sm.w_raw[t * k + j]);
+        den = __fadd_rn(den, 1e-20f);
+      }
+      den = __shfl_sync(0xffffffffu, den, 0);
+    }
+    for (int j = lane; j < k; j += 32) {
+      float w = sm.w_raw[t * k + j];
+      if (do_norm) w = __fdiv_rn(w, den);
+      sm.w[t * k + j] = __fmul_rn(w, a.scale);
     }
   }
-  __syncthreads();
-  {  // compact the selected experts in ascending id order (4 ids per thread)
-    int cnt = 0;
-    int flags[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = threadIdx.x * 4 + q;
-      flags[q] = (e < E) && (s_slot[e] >= 0 || (T > 1 && s_slot[E + e] >= 0));
-      cnt += flags[q];
-    }
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int* wsum = s_misc + 2;
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += wsum[w];
-    int pos = base + incl - cnt;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (flags[q]) s_active[pos++] = threadIdx.x * 4 + q;
-    if (threadIdx.x == blockDim.x - 1) s_misc[0] = base + incl;
-  }
-  __syncthreads();
-  const int n_act = s_misc[0];
+  consumer_sync();
 
-  // ---- C: gate/up rows of the selected experts ----
-  for (int item = gw; item < n_act * I; item += nw) {
-    const int ai = item / I, j = item - ai * I;
-    const int e = s_active[ai];
-    const int sl0 = s_slot[e], sl1 = T > 1 ? s_slot[E + e] : -1;
-    const int slA = sl0 >= 0 ? sl0 : sl1;  // first slot holding e
-    const int slB = sl0 >= 0 ? sl1 : -1;   // second (token 1), if both tokens chose e
-    const uint16_t* gate = a.w_gate_up + ((int64_t)e * 2 * I + j) * H;
-    float hA, hB;
-    gate_up_dot(gate, gate + (int64_t)I * H, a.x + (int64_t)(slA / k) * H,
-                slB >= 0 ? a.x + (int64_t)(slB / k) * H : nullptr, H, &hA, &hB);
-    if (lane == 0) {
-      a.h[(int64_t)slA * I + j] = hA;
-      if (slB >= 0) a.h[(int64_t)slB * I + j] = hB;
+  // ---- distinct experts, in order of first slot, with the slot(s) holding each ----
+  if (warp == 0) {
+    const int ns = T * k;
+    const int e = lane < ns ? sm.idx[lane] : (int)(0x40000000u | (uint32_t)lane);  // unique dummies
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    const bool first = lane < ns && (__ffs(same) - 1) == lane;
+    const uint32_t firsts = __ballot_sync(0xffffffffu, first);
+    if (first) {
+      const int pos = __popc(firsts & ((1u << lane) - 1u));
+      const uint32_t other = same & ~(1u << lane);  // the other token's slot (ids are distinct per token)
+      sm.act_e[pos] = e;
+      sm.act_a[pos] = lane;
+      sm.act_b[pos] = other != 0u ? __ffs(other) - 1 : -1;
+    }
+    if (lane == 0) sm.n_act = __popc(firsts);
+    if (blockIdx.x == 0 && lane < ns) {
+      if (a.topk_idx_out != nullptr) a.topk_idx_out[lane] = e;
+      if (a.topk_w_out != nullptr) a.topk_w_out[lane] = sm.w[lane];
     }
   }
-  if (!grid_barrier(a.hdr, 2, s_misc + 1)) return;
+  consumer_sync();
+}
 
-  // ---- D: down rows, routed (weighted, per slot) and shared ----
-  const int nrb = (H + kDownRows - 1) / kDownRows;
-  const int routed_items = n_act * nrb;
-  const int total = routed_items + (a.ws_down != nullptr ? nrb : 0);
-  for (int item = gw; item < total; item += nw) {
-    const bool shared = item >= routed_items;
-    const int ai = shared ? 0 : item / nrb;
-    const int n0 = (shared ? item - routed_items : item - ai * nrb) * kDownRows;
-    const int nrows = min(kDownRows, H - n0);
-    if (shared) {
-      const float mine = down_dot(a.ws_down + (int64_t)n0 * Is, nrows, Is, a.h_shared, T > 1 ? a.h_shared + Is : nullptr);
-      const int r = lane >> 1, t = lane & 1;
-      if (r < nrows && t < T) a.shared_out[(int64_t)t * H + n0 + r] = mine;
-    } else {
-      const int e = s_active[ai];
-      const int sl0 = s_slot[e], sl1 = T > 1 ? s_slot[E + e] : -1;
-      const int slA = sl0 >= 0 ? sl0 : sl1;
-      const int slB = sl0 >= 0 ? sl1 : -1;
-      const float mine = down_dot(a.w_down + ((int64_t)e * H + n0) * I, nrows, I, a.h + (int64_t)slA * I,
-                                  slB >= 0 ? a.h + (int64_t)slB * I : nullptr);
-      const int r = lane >> 1, t = lane & 1;
-      const int sl = t == 0 ? slA : slB;
-      if (r < nrows && sl >= 0) a.y_slots[(int64_t)sl * H + n0 + r] = s_w[sl] * mine;
+// ---------------------------------------------------------------------------
+// The stream of one CTA: a sequence of segments, each a contiguous share of
+// one kind of rows. A (router rows, then shared gate/up pairs) and S (shared
+// down blocks) are split evenly over the CTAs. Then every CTA takes a share
+// of each distinct expert's gate/up pairs (C0 .. C(n-1)) and then of each
+// one's down blocks (D0 .. D(n-1)): expert i's h is complete once every CTA
+// has passed its C share of it, long before the CTAs reach Di, so the down
+// blocks rarely wait. The shares of expert i are rotated by i*G/n CTAs so
+// that the rounding of the even split does not favour the same CTAs for every
+// expert.
+// ---------------------------------------------------------------------------
+enum SegKind { kSegA, kSegS, kSegC, kSegD };
+
+struct Seg {
+  int kind, ai;  // kind, distinct expert (C and D)
+  Range r;       // the share: rows (C), blocks (D), items (A, S)
+};
+
+__device__ __forceinline__ int num_segments(int n_act) { return 2 + 2 * n_act; }
+
+__device__ __forceinline__ Seg segment(const DecodeArgs& a, const Geo& g, int n_act, int i) {
+  const int G = gridDim.x, b = blockIdx.x;
+  Seg sg{};
+  if (i == 0) {
+    sg.kind = kSegA;
+    sg.r = split((a.logits_override == nullptr ? a.E : 0) + (a.ws_gate_up != nullptr ? a.Is : 0), b, G);
+    return sg;
+  }
+  if (i == 1) {
+    sg.kind = kSegS;
+    sg.r = split(a.ws_down != nullptr ? g.nsblk : 0, b, G);
+    return sg;
+  }
+  const int j = i - 2;
+  sg.kind = j < n_act ? kSegC : kSegD;
+  sg.ai = j < n_act ? j : j - n_act;
+  const int rb = (b + (int)((int64_t)sg.ai * G / n_act)) % G;
+  sg.r = split(sg.kind == kSegC ? a.I : g.nblk, rb, G);
+  return sg;
+}
+
+// The producer thread: issues the CTA's stream in order, unit u into ring slot
+// u % depth once the consumer of the slot's previous unit freed it.
+__device__ void producer(const DecodeArgs& a, const Geo& g, unsigned char* ring, FusedSmem& sm) {
+  const int H = a.H, I = a.I, Is = a.Is;
+  const int n_router = a.logits_override == nullptr ? a.E : 0;
+  uint32_t u = 0;
+  bool ok = true;
+  auto issue = [&](const void* src0, uint32_t n0, const void* src1, uint32_t n1) {
+    const int s = (int)(u % (uint32_t)g.depth);
+    const uint32_t n = u / (uint32_t)g.depth;
+    if (n > 0 && !thread_wait_phase(&sm.empty[s], (n - 1) & 1u, a.hdr, 400 + s)) {
+      ok = false;
+      return;
+    }
+    sm.tag[s] = u;  // the slot's previous fill is consumed: its phase is complete
+    mbar_expect_tx(&sm.full[s], n0 + n1);
+    unsigned char* dst = ring + (size_t)s * g.stage_bytes;
+    bulk_load(dst, src0, n0, &sm.full[s]);
+    if (n1 != 0) bulk_load(dst + n0, src1, n1, &sm.full[s]);
+    ++u;
+  };
+  int nseg = 2, n_act = 0;
+  for (int si = 0; ok && si < nseg; ++si) {
+    const Seg sg = segment(a, g, n_act, si);
+    for (int i = sg.r.lo; ok && i < sg.r.lo + sg.r.n; ++i) {
+      if (sg.kind == kSegA) {
+        if (i < n_router) {
+          issue(a.router_w + (int64_t)i * H, 4u * H, nullptr, 0);
+        } else {
+          const int j = i - n_router;
+          issue(a.ws_gate_up + (int64_t)j * H, 2u * H, a.ws_gate_up + (int64_t)(Is + j) * H, 2u * H);
+        }
+      } else if (sg.kind == kSegS) {
+        const int n0 = i * g.rs, rows = min(g.rs, H - n0);
+        issue(a.ws_down + (int64_t)n0 * Is, 2u * rows * Is, nullptr, 0);
+      } else if (sg.kind == kSegC) {
+        const uint16_t* gate = a.w_gate_up + ((int64_t)sm.act_e[sg.ai] * 2 * I + i) * H;
+        issue(gate, 2u * H, gate + (int64_t)I * H, 2u * H);
+      } else {
+        const int n0 = i * g.rd, rows = min(g.rd, H - n0);
+        issue(a.w_down + ((int64_t)sm.act_e[sg.ai] * H + n0) * I, 2u * rows * I, nullptr, 0);
+      }
+    }
+    if (si == 1 && ok) {  // the segments after S need this CTA's routing
+      ok = thread_wait_phase(&sm.route_ready, 0, a.hdr, 500);
+      if (ok) {
+        n_act = sm.n_act;
+        nseg = num_segments(n_act);
+      }
     }
   }
-  if (!grid_barrier(a.hdr, 3, s_misc + 1)) return;
-
-  // ---- E: y[t] = bf16( sum_j y_slots[t*k + j] + shared_out[t] ), slot order ----
-  const int nv = H / 4;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T * nv; i += gridDim.x * blockDim.x) {
-    const int t = i / nv, v = i - t * nv;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 f = ldcg4(a.y_slots + ((int64_t)(t * k + j) * H) + v * 4);
-      acc.x += f.x;
-      acc.y += f.y;
-      acc.z += f.z;
-      acc.w += f.w;
-    }
-    if (a.ws_down != nullptr) {
-      const float4 f = ldcg4(a.shared_out + (int64_t)t * H + v * 4);
-      acc.x += f.x;
-      acc.y += f.y;
-      acc.z += f.z;
-      acc.w += f.w;
-    }
-    reinterpret_cast<uint2*>(a.y)[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  if (!ok) {
+    // the consumers stopped: wait (bounded) for the copies still in flight
+    const uint32_t first = u > (uint32_t)g.depth ? u - g.depth : 0u;
+    for (uint32_t v = first; v < u; ++v)
+      thread_wait_phase(&sm.full[v % g.depth], (v / g.depth) & 1u, nullptr, 0);
   }
 }
 
-template <int P>
-size_t fused_smem(int E) {
-  return (size_t)kFusedMaxT * 32 * P * 4 + (size_t)kFusedMaxT * E * 4 * 3 + (size_t)E * 4 + 64;
+// First stream index at or after `base` that belongs to consumer warp w.
+__device__ __forceinline__ uint32_t first_unit(uint32_t base, int w) {
+  return base + (uint32_t)((w - (int)(base % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
 }
 
-template <int P>
-cudaError_t launch_fused_p(const DecodeArgs& a, cudaStream_t s) {
-  const size_t smem = fused_smem<P>(a.E);
-  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+// A consumer warp: stream units w, w + 8, ... of its CTA.
+__device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring, unsigned char* scratch,
+                         FusedSmem& sm) {
+  const int T = a.T, k = a.k, H = a.H, I = a.I, Is = a.Is, E = a.E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t* done = a.sync;  // [kMaxSlots]: gate/up rows finished per distinct expert
+
+  // counters: each CTA zeroes its share; the grid barrier orders it before use
+  const Range z = split(kMaxSlots + kFusedMaxT * H, blockIdx.x, gridDim.x);
+  for (int i = threadIdx.x; i < z.n; i += kConsumers) a.sync[z.lo + i] = 0;
+
+  // token rows and expert bias into shared memory (one coalesced pass)
+  uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + route_scratch_bytes(T, E));
+  float* bias_s = a.expert_bias != nullptr ? reinterpret_cast<float*>(xs + (size_t)T * H) : nullptr;
+  for (int i = threadIdx.x; i < T * H / 8; i += kConsumers)
+    reinterpret_cast<uint4*>(xs)[i] = ld_nc_u4(a.x + (size_t)i * 8);
+  if (bias_s != nullptr)
+    for (int e = threadIdx.x; e < E; e += kConsumers) bias_s[e] = __ldg(a.expert_bias + e);
+  consumer_sync();
+
+  const int n_router = a.logits_override == nullptr ? E : 0;
+  const float* logits = a.logits_override != nullptr ? a.logits_override : a.logits;
+  const int target = k + (a.ws_down != nullptr ? 1 : 0);
+  Pending q;
+  q.np = 0;
+  auto flush_if_pending = [&]() {
+    if (q.np > 0) publish(a, q, target);
+  };
+  // Waits for stream unit v; publishes the pending work first if it would block.
+  auto stage = [&](uint32_t v, const unsigned char** p, uint64_t** empty) {
+    const int s = (int)(v % (uint32_t)g.depth);
+    const uint32_t parity = (v / g.depth) & 1u;
+    *p = ring + (size_t)s * g.stage_bytes;
+    *empty = &sm.empty[s];
+    if (__all_sync(0xffffffffu, sm.tag[s] == v && mbar_try_wait(&sm.full[s], parity))) return true;
+    flush_if_pending();
+    return warp_wait_tag(&sm.tag[s], v, a.hdr, 300 + s) && warp_wait_phase(&sm.full[s], parity, a.hdr, 300 + s);
+  };
+
+  // ---- A: router rows and shared gate/up pairs ----
+  // A warp whose wait runs out must still reach the named barriers below (they
+  // have no timeout): it flags the CTA, and the consumers leave together after
+  // the grid barrier.
+  uint32_t base = 0;
+  {
+    const Seg sg = segment(a, g, 0, 0);
+    for (uint32_t u = first_unit(base, warp); u < base + sg.r.n; u += kConsumerWarps) {
+      const unsigned char* st;
+      uint64_t* empty;
+      if (!stage(u, &st, &empty)) {
+        sm.abort = 1;
+        break;
+      }
+      const int i = sg.r.lo + (int)(u - base);
+      if (i < n_router) {
+        const float v = router_unit(reinterpret_cast<const float*>(st), H, xs, T, empty);
+        if (lane == 0) a.logits[i] = v;
+        if (lane == 16 && T > 1) a.logits[E + i] = v;
+      } else {
+        const int j = i - n_router;
+        const uint16_t* gate = reinterpret_cast<const uint16_t*>(st);
+        const float v = gate_up_unit(gate, gate + H, H, xs, T > 1 ? xs + H : nullptr, empty);
+        if (lane == 0) a.h_shared[j] = v;
+        if (lane == 16 && T > 1) a.h_shared[Is + j] = v;
+      }
+    }
+    base += sg.r.n;
+  }
+  if (!grid_barrier(a.hdr, 1, &sm.flag) || sm.abort != 0) return;
+
+  // ---- routing; then the producer may issue the selected experts' rows ----
+  route_block(a, logits, bias_s, scratch, sm);
+  if (threadIdx.x == 0) mbar_arrive(&sm.route_ready);
+  const int n_act = sm.n_act;
+  const int tq = lane >> 4, rr = lane & 15;  // down blocks: lane t*16 + r holds (slot or token t, row r)
+
+  for (int si = 1; si < num_segments(n_act); ++si) {
+    const Seg sg = segment(a, g, n_act, si);
+    for (uint32_t u = first_unit(base, warp); u < base + sg.r.n; u += kConsumerWarps) {
+      const int i = sg.r.lo + (int)(u - base);
+      const unsigned char* st;
+      uint64_t* empty;
+      if (sg.kind == kSegS) {  // ---- shared down block ----
+        const int n0 = i * g.rs, rows = min(g.rs, H - n0);
+        const float* h1 = T > 1 ? a.h_shared + Is : nullptr;
+        const HChunk p = load_h(a.h_shared, h1, lane, Is / 8);
+        if (!stage(u, &st, &empty)) return;
+        const float v = down_unit(reinterpret_cast<const uint16_t*>(st), rows, Is, a.h_shared, h1, p, empty);
+        int idx = -1;
+        if (rr < rows && tq < T) {
+          a.shared_out[(int64_t)tq * H + n0 + rr] = v;
+          idx = tq * H + n0 + rr;
+        }
+        add_pending(q, idx);
+      } else if (sg.kind == kSegC) {  // ---- gate/up pair of a selected expert ----
+        const int slA = sm.act_a[sg.ai], slB = sm.act_b[sg.ai];
+        if (!stage(u, &st, &empty)) return;
+        const uint16_t* w = reinterpret_cast<const uint16_t*>(st);
+        const float v = gate_up_unit(w, w + H, H, xs + (slA / k) * H, slB >= 0 ? xs + (slB / k) * H : nullptr, empty);
+        // each writer lane releases its own row: the down blocks of this expert
+        // wait for I rows per slot holding it
+        if (lane == 0 || (lane == 16 && slB >= 0)) {
+          a.h[(int64_t)(lane == 0 ? slA : slB) * I + i] = v;
+          red_release_add(done + sg.ai, 1);
+        }
+      } else {  // ---- down block of a selected expert ----
+        const int ai = sg.ai, slA = sm.act_a[ai], slB = sm.act_b[ai];
+        const int n0 = i * g.rd, rows = min(g.rd, H - n0);
+        const int need = slB >= 0 ? 2 * I : I;
+        int complete = lane == 0 ? ld_acquire(done + ai) >= need : 0;
+        if (!__shfl_sync(0xffffffffu, complete, 0)) {
+          flush_if_pending();
+          if (!warp_wait_count(done + ai, need, a.hdr, 200 + ai)) return;
+        }
+        __syncwarp();
+        const float* h0 = a.h + (int64_t)slA * I;
+        const float* h1 = slB >= 0 ? a.h + (int64_t)slB * I : nullptr;
+        const HChunk p = load_h(h0, h1, lane, I / 8);
+        if (!stage(u, &st, &empty)) return;
+        const float v = down_unit(reinterpret_cast<const uint16_t*>(st), rows, I, h0, h1, p, empty);
+        const int sl = tq == 0 ? slA : slB;
+        int idx = -1;
+        if (rr < rows && sl >= 0) {
+          a.y_slots[(int64_t)sl * H + n0 + rr] = sm.w[sl] * v;
+          idx = (sl / k) * H + n0 + rr;
+        }
+        add_pending(q, idx);
+      }
+      if (q.np == kMaxPend) publish(a, q, target);
+    }
+    base += sg.r.n;
+  }
+  publish(a, q, target);
+}
+
+__global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const DecodeArgs a, const Geo g) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ FusedSmem sm;
+  unsigned char* ring = smem_raw;
+  unsigned char* scratch = smem_raw + (size_t)g.depth * g.stage_bytes;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < g.depth; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+      sm.tag[s] = 0xffffffffu;
+    }
+    mbar_init(&sm.route_ready, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x >= kConsumers) {
+    if (threadIdx.x == kConsumers) producer(a, g, ring, sm);
+    return;
+  }
+  consumer(a, g, ring, scratch, sm);
+}
+
+
+// Stream geometry for a launch; depth 0 when the shapes do not fit.
+Geo make_geo(int T, int E, int H, int I, int Is) {
+  Geo g{};
+  if (H > kMaxHidden || I > 2 * H || Is > 2 * H) return g;
+  g.stage_bytes = 4 * H;
+  const int rd = g.stage_bytes / (2 * I), rs = Is > 0 ? g.stage_bytes / (2 * Is) : 1;
+  g.rd = rd < kMaxDownRows ? rd : kMaxDownRows;
+  g.rs = rs < kMaxDownRows ? rs : kMaxDownRows;
+  g.nblk = (H + g.rd - 1) / g.rd;
+  g.nsblk = Is > 0 ? (H + g.rs - 1) / g.rs : 0;
+  const int avail = kSmemBudget - (int)sizeof(FusedSmem) - (int)scratch_bytes(T, E, H);
+  g.depth = avail / g.stage_bytes < kMaxStages ? avail / g.stage_bytes : kMaxStages;
+  if (g.depth < kMinStages) g.depth = 0;
+  return g;
+}
+
+}  // namespace
+
+size_t decode_fused_sync_ints(int H) { return (size_t)kMaxSlots + (size_t)kFusedMaxT * H; }
+
+bool decode_fused_supported(int64_t T, int k, int E, int H, int I, int Is) {
+  // at most two tokens and one warp lane per slot; a stage must hold a router row
+  return T >= 1 && T <= kFusedMaxT && k <= E && E <= 1024 && T * k <= kMaxSlots &&
+         make_geo((int)T, E, H, I, Is).depth > 0;
+}
+
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s) {
+  const Geo g = make_geo(a.T, a.E, a.H, a.I, a.Is);
+  if (g.depth == 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)g.depth * g.stage_bytes + scratch_bytes(a.T, a.E, a.H);
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel<P>, kFusedThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel, kFusedThreads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const int blocks = sm_count() * per_sm;  // every CTA resident: the grid barriers rely on it
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(blocks);
+  cfg.gridDim = dim3(sm_count());  // one CTA per SM, all resident: the grid barrier and the waits rely on it
   cfg.blockDim = dim3(kFusedThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -374,27 +982,10 @@ cudaError_t launch_fused_p(const DecodeArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   before_launch(MOE_KERNEL_DECODE_FUSED, s);
-  e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<P>, a);
+  e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a, g);
   after_launch(MOE_KERNEL_DECODE_FUSED, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
-}
-
-}  // namespace
-
-bool decode_fused_supported(int64_t T, int k, int E) {
-  // k <= E and the token count: the slot table holds two tokens
-  return T >= 1 && T <= kFusedMaxT && k <= E && E <= 1024;
-}
-
-cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s) {
-  const int per = (a.E + 31) / 32;
-  if (per <= 1) return launch_fused_p<1>(a, s);
-  if (per <= 2) return launch_fused_p<2>(a, s);
-  if (per <= 4) return launch_fused_p<4>(a, s);
-  if (per <= 8) return launch_fused_p<8>(a, s);
-  if (per <= 16) return launch_fused_p<16>(a, s);
-  return launch_fused_p<32>(a, s);
 }
 
 }  // namespace moe

@@ -1,0 +1,38 @@
+// Arguments and host entry points of the fused decode kernel (decode_fused.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct DecodeArgs {
+  const uint16_t* x;  // [T, H]
+  int T, H, E, k, I, Is, n_group, topk_group, score_fn, norm;
+  float scale;
+  const float* router_w;         // [E, H] or null when logits are given
+  const float* expert_bias;      // [E] or null
+  const float* logits_override;  // [T, E] or null
+  const uint16_t* w_gate_up;     // [E, 2I, H]
+  const uint16_t* w_down;        // [E, H, I]
+  const uint16_t* ws_gate_up;    // [2Is, H] or null
+  const uint16_t* ws_down;       // [H, Is]
+  float* logits;                 // [T, E] workspace
+  int32_t* topk_idx_out;         // [T, k] or null
+  float* topk_w_out;             // [T, k] or null
+  float* h;                      // [T*k, I] workspace
+  float* h_shared;               // [T, Is] workspace
+  float* y_slots;                // [T*k, H] workspace
+  float* shared_out;             // [T, H] workspace
+  int32_t* sync;                 // decode_fused_sync_ints(H) counters, workspace
+  uint16_t* y;                   // [T, H] output
+  WsHeader* hdr;
+};
+
+// Completion counters the kernel needs in the workspace (zeroed by the kernel).
+size_t decode_fused_sync_ints(int H);
+// Whether the fused kernel handles this batch and shape (1-2 tokens, at most 32
+// slots, hidden size up to 8192, expert widths up to twice the hidden size).
+bool decode_fused_supported(int64_t T, int k, int E, int H, int I, int Is);
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace moe

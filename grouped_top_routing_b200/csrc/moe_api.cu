@@ -12,6 +12,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "decode_fused.cuh"
 #include "ffn.cuh"
 
 namespace moe {
@@ -33,29 +34,6 @@ cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_
                            cudaStream_t s);
 cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
                                const uint16_t* x, int H, uint16_t* x_perm, cudaStream_t s);
-struct DecodeArgs {
-  const uint16_t* x;
-  int T, H, E, k, I, Is, n_group, topk_group, score_fn, norm;
-  float scale;
-  const float* router_w;
-  const float* expert_bias;
-  const float* logits_override;
-  const uint16_t* w_gate_up;
-  const uint16_t* w_down;
-  const uint16_t* ws_gate_up;
-  const uint16_t* ws_down;
-  float* logits;
-  int32_t* topk_idx_out;
-  float* topk_w_out;
-  float* h;
-  float* h_shared;
-  float* y_slots;
-  float* shared_out;
-  uint16_t* y;
-  WsHeader* hdr;
-};
-bool decode_fused_supported(int64_t T, int k, int E);
-cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // errors, hooks, device cache
@@ -199,7 +177,7 @@ constexpr int64_t kLogitsGemvMaxT = 16;  // larger batches: router logits on the
 
 struct Layout {
   size_t hdr, logits, wr_planes, logit_parts, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
-  size_t x_perm, h_perm, h_shared, y_slots, shared_out, total;
+  size_t x_perm, h_perm, h_shared, y_slots, shared_out, decode_sync, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -253,6 +231,7 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 4);
   L.y_slots = take((size_t)R * H * 4);
   L.shared_out = take((size_t)T * H * 4);
+  L.decode_sync = take(decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is) ? decode_fused_sync_ints((int)H) * 4 : 0);
   L.total = off;
   return L;
 }
@@ -496,7 +475,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
-  if (g_ffn_path == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts)) {
+  if (g_ffn_path == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size, c.moe_intermediate_size,
+                                                    shared_width(c))) {
     DecodeArgs d{};
     d.x = x;
     d.T = (int)T;
@@ -524,6 +504,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
     d.h_shared = at<float>(ws, L.h_shared);
     d.y_slots = at<float>(ws, L.y_slots);
     d.shared_out = at<float>(ws, L.shared_out);
+    d.sync = at<int32_t>(ws, L.decode_sync);
     d.y = y;
     d.hdr = hdr;
     cudaError_t e = launch_decode_fused(d, s);

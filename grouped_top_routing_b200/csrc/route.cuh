@@ -1,5 +1,5 @@
-// Router for one token, executed by one warp (shared by the router kernel and
-// the fused decode kernel).
+// Router for one token, executed by one warp, and the helpers the fused
+// decode kernel's block-wide router shares with it.
 //
 // Follows mlxcel issue #838 "add Ant Group Ling / Bailing MoE", section
 // "Router: selection uses biased scores, weights come from unbiased scores"
@@ -60,9 +60,7 @@ __device__ __forceinline__ float warp_max_f32(float v) {
 // Routes the token whose fp32 gates are Lrow[0..E): writes idx_out[0..k) (expert
 // ids, ordered by biased score descending then id ascending) and w_out[0..k)
 // (routing weights). buf: this warp's 32*P floats of shared memory.
-// kCoherent: the gates were written earlier in the same launch (by other CTAs),
-// so they are read through L2 (ld.global.cg) instead of the read-only path.
-template <int P, bool kCoherent = false>
+template <int P>
 __device__ __forceinline__ void route_one_token(const float* __restrict__ Lrow, const float* __restrict__ bias, int E,
                                                 int k, int n_group, int topk_group, int score_fn, int norm,
                                                 float scale, float* buf, int32_t* idx_out, float* w_out) {
@@ -74,7 +72,7 @@ __device__ __forceinline__ void route_one_token(const float* __restrict__ Lrow, 
 #pragma unroll
   for (int i = 0; i < P; ++i) {
     const int e = lane * P + i;
-    L[i] = (e < E) ? (kCoherent ? __ldcg(Lrow + e) : __ldg(Lrow + e)) : -INFINITY;
+    L[i] = (e < E) ? __ldg(Lrow + e) : -INFINITY;
   }
 
   // ---- score function: fp64 evaluation, one rounding to fp32 ----
