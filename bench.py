@@ -62,6 +62,42 @@ def peaks():
 # algorithmic work of one step (counted from the step's actual routing)
 # ---------------------------------------------------------------------------
 
+# DRAM traffic per launch of the roofline kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum, one ncu capture of this script's own default command
+# for the workload), with a hash of the kernel's source files at capture time.
+# The figure is reported only while those sources are unchanged and the run
+# uses the captured configuration.
+KERNEL_SOURCES = {
+    "expert_gate_up": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
+    "expert_down": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
+    "decode_fused": ["decode_fused.cu", "decode_fused.cuh", "route.cuh", "mbarrier.cuh", "common.cuh"],
+}
+MEASURED_TRAFFIC = {
+    ("expert_gate_up", "ling26_flash_t512"): (2886553984, "0e81a7fa77706bc4"),
+    ("expert_down", "ling26_flash_t512"): (1491579904, "0e81a7fa77706bc4"),
+    ("decode_fused", "ling30_flash_decode_t1"): (123433984, "20ccce4ad41dea1b"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "grouped_top_routing_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        h.update(name.encode())
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str):
+    """Bytes per launch from the capture, or None when it no longer applies."""
+    entry = MEASURED_TRAFFIC.get((kernel, workload))
+    if entry is None or overrides or ffn_path != "auto":
+        return None
+    return entry[0] if kernel_source_hash(kernel) == entry[1] else None
+
+
 def algorithmic(wl, T, n_unique):
     """Bytes each expert pass must move, and the block's flops, given the
     number of distinct routed experts the batch touched. Activations count at
@@ -345,19 +381,20 @@ def run_ours(args):
     else:
         kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
         kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
+    traffic = measured_traffic(args.kernel, args.workload, args.set, args.ffn_path)
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if kflops / kbytes > ridge:
         achieved = kflops / (kms / 1e3) / 1e12
         roofline = {"bound": "tensor", "kernel": args.kernel, "achieved": achieved, "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                    "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
                     "peak_source": pk["source"] + " (bf16 burst)", "algorithmic_flops": kflops,
                     "algorithmic_bytes": kbytes, "kernel_ms": kms,
                     "hbm_gbs": kbytes / (kms / 1e3) / 1e9}
     else:
         achieved = kbytes / (kms / 1e3) / 1e9
         roofline = {"bound": "hbm", "kernel": args.kernel, "achieved": achieved, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
+                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"],
                     "algorithmic_bytes": kbytes, "algorithmic_flops": kflops, "kernel_ms": kms,
                     "tflops": kflops / (kms / 1e3) / 1e12}
     step_gbs = work["step_bytes"] / (ms_per_step / 1e3) / 1e9
