@@ -30,6 +30,7 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
                            int32_t* tile_base, WsHeader* hdr, cudaStream_t s);
 cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* active, WsHeader* hdr,
                                        cudaStream_t s);
+cudaError_t launch_identity_route(int64_t T, int32_t* offsets, int32_t* tok_of, float* w, cudaStream_t s);
 cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
                            cudaStream_t s);
 cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
@@ -327,6 +328,35 @@ moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint
   return MOE_OK;
 }
 
+// The dense-prefix MLP as a block of one expert, one slot per token, weight 1
+// and no shared MLP: the expert kernels then compute exactly the dense MLP.
+moe_config dense_config(int32_t hidden_size, int32_t intermediate_size) {
+  moe_config c{};
+  c.hidden_size = hidden_size;
+  c.num_experts = 1;
+  c.num_experts_per_tok = 1;
+  c.n_group = 1;
+  c.topk_group = 1;
+  c.score_function = MOE_SCORE_SOFTMAX;
+  c.norm_topk_prob = 0;
+  c.routed_scaling_factor = 1.0f;
+  c.moe_intermediate_size = intermediate_size;
+  c.num_shared_experts = 0;
+  c.moe_shared_expert_intermediate_size = 0;
+  return c;
+}
+
+moe_status validate_dense(int32_t hidden_size, int32_t intermediate_size) {
+  MOE_TRY(check_range("hidden_size", hidden_size, 1, kMaxHidden));
+  MOE_TRY(check_range("intermediate_size", intermediate_size, 1, kMaxIntermediate));
+  if (hidden_size % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden_size = %d is not a multiple of 8 (16-byte rows)", hidden_size);
+  if (intermediate_size % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "intermediate_size = %d is not a multiple of 8 (16-byte rows)",
+                intermediate_size);
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -571,6 +601,41 @@ moe_status moe_set_ffn_path(int32_t path) {
 }
 
 const char* moe_last_error(void) { return g_err; }
+
+size_t moe_dense_mlp_workspace_size(int32_t hidden_size, int32_t intermediate_size, int64_t max_tokens) {
+  if (validate_dense(hidden_size, intermediate_size) != MOE_OK) return 0;
+  const moe_config c = dense_config(hidden_size, intermediate_size);
+  if (check_tokens(c, max_tokens) != MOE_OK) return 0;
+  g_err[0] = '\0';
+  return layout(c, max_tokens).total;
+}
+
+moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const uint16_t* x, int64_t T,
+                         const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* y, void* ws, size_t ws_bytes,
+                         void* stream) {
+  MOE_TRY(validate_dense(hidden_size, intermediate_size));
+  const moe_config c = dense_config(hidden_size, intermediate_size);
+  MOE_TRY(check_tokens(c, T));
+  MOE_TRY(check_ws(c, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr("x", x, 16, true));
+  MOE_TRY(check_ptr("w_gate_up", w_gate_up, 16, true));
+  MOE_TRY(check_ptr("w_down", w_down, 16, true));
+  MOE_TRY(check_ptr("y", y, 16, true));
+  const Layout L = layout(c, T);
+  cudaStream_t s = as_stream(stream);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* tok_of = at<int32_t>(ws, L.tok_of);
+  float* w = at<float>(ws, L.topk_w);
+  float* y_slots = at<float>(ws, L.y_slots);
+  cudaError_t e = launch_identity_route(T, offsets, tok_of, w, s);
+  if (e != cudaSuccess) return cuda_fail(e, "dense routing");
+  // one expert and one slot per token: the permuted rows are the token rows
+  MOE_TRY(run_ffn(c, T, x, x, offsets, tok_of, w, w_gate_up, w_down, nullptr, nullptr, y_slots, nullptr, ws, false, s));
+  e = launch_combine(y_slots, nullptr, T, 1, hidden_size, y, s);
+  if (e != cudaSuccess) return cuda_fail(e, "dense output");
+  return MOE_OK;
+}
 
 }  // extern "C"
 

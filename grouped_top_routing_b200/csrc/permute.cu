@@ -307,4 +307,32 @@ cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* a
   return cudaGetLastError();
 }
 
+// The routing of a dense MLP seen as a block of one expert with one slot per
+// token and weight 1.0: offsets {0, T}, row r holds slot r, every weight 1.
+__global__ void __launch_bounds__(256) identity_route_kernel(int64_t T, int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ tok_of, float* __restrict__ w) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T; i += stride) {
+    tok_of[i] = (int32_t)i;
+    w[i] = 1.0f;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    offsets[0] = 0;
+    offsets[1] = (int32_t)T;
+  }
+}
+
+cudaError_t launch_identity_route(int64_t T, int32_t* offsets, int32_t* tok_of, float* w, cudaStream_t s) {
+  int64_t blocks = (T + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  before_launch(MOE_KERNEL_PERMUTE, s);
+  launch_pdl(identity_route_kernel, dim3((unsigned)blocks), dim3(256), 0, s, T, offsets, tok_of, w);
+  after_launch(MOE_KERNEL_PERMUTE, s);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -174,6 +174,28 @@ def make_inputs(wl: dict, seed: int = 0, device="cpu", tokens: int | None = None
     return out
 
 
+# Dense-prefix MLP of Ling-2.6-flash: hidden 4096, intermediate 9216 (model card
+# "Ling-2.6-flash-JANGTQ", section "Architecture (bailing_hybrid)", layer table).
+LING26_DENSE = dict(hidden_size=4096, intermediate_size=9216)
+
+
+def make_dense_inputs(hidden_size: int, intermediate_size: int, tokens: int, seed: int = 0, device="cpu") -> dict:
+    """Weights and token rows of a dense SwiGLU MLP: gate/up [2*Id, H] with std
+    1/sqrt(H), down [H, Id] with std 1/sqrt(Id), x ~ N(0, 1); all bf16."""
+    device = torch.device(device)
+    H, Id = hidden_size, intermediate_size
+    gw = torch.Generator(device=device)
+    gw.manual_seed(seed)
+    gx = torch.Generator(device=device)
+    gx.manual_seed(seed + ACT_SEED_OFFSET)
+    return {
+        "tokens": tokens,
+        "w_gate_up": _normal((2 * Id, H), 1.0 / math.sqrt(H), gw, device, torch.bfloat16),
+        "w_down": _normal((H, Id), 1.0 / math.sqrt(Id), gw, device, torch.bfloat16),
+        "x": _normal((tokens, H), 1.0, gx, device, torch.bfloat16),
+    }
+
+
 def random_logits(T: int, E: int, std: float, seed: int = 0, device="cpu") -> torch.Tensor:
     """fp32 logits [T, E] ~ N(0, std), for routing-only tests."""
     gen = torch.Generator(device=torch.device(device))

@@ -26,7 +26,8 @@ FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch at
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
-           "moe_set_ffn_path", "moe_launch_count", "moe_last_error", "moe_permute_static")
+           "moe_set_ffn_path", "moe_launch_count", "moe_last_error", "moe_permute_static",
+           "moe_dense_mlp_workspace_size", "moe_dense_mlp")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 
 
@@ -83,6 +84,8 @@ def _load():
         "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
         "moe_set_ffn_path": (st, [ctypes.c_int32]),
         "moe_permute_static": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp]),
+        "moe_dense_mlp_workspace_size": (sz, [ctypes.c_int32, ctypes.c_int32, i64]),
+        "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -134,10 +137,11 @@ def moe_workspace_size(cfg, max_tokens: int) -> int:
 
 
 class Workspace:
-    """A device workspace sized by moe_workspace_size, header zeroed."""
+    """A device workspace sized by moe_workspace_size (or, given nbytes, of that
+    size), header zeroed."""
 
-    def __init__(self, cfg, max_tokens: int, device="cuda"):
-        self.nbytes = moe_workspace_size(cfg, max_tokens)
+    def __init__(self, cfg, max_tokens: int, device="cuda", nbytes: int | None = None):
+        self.nbytes = moe_workspace_size(cfg, max_tokens) if nbytes is None else int(nbytes)
         self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
         base = self.buf.data_ptr()
         self.ptr = (base + 255) & ~255
@@ -243,3 +247,22 @@ def set_kernel_timer(kernel: str, ev_start=None, ev_stop=None):
 
 def launch_count() -> int:
     return int(lib.moe_launch_count())
+
+
+def dense_mlp_workspace(hidden_size: int, intermediate_size: int, max_tokens: int, device="cuda") -> Workspace:
+    """Workspace for moe_dense_mlp."""
+    n = lib.moe_dense_mlp_workspace_size(int(hidden_size), int(intermediate_size), int(max_tokens))
+    if n == 0:
+        raise MoeError(1, last_error())
+    return Workspace(None, max_tokens, device=device, nbytes=n)
+
+
+def moe_dense_mlp(x, w_gate_up, w_down, ws: Workspace, y=None, stream=None):
+    """Dense-prefix SwiGLU MLP: w_gate_up [2*Id, H] (gate rows first), w_down [H, Id]."""
+    T, H = x.shape
+    Id = w_down.shape[1]
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib.moe_dense_mlp(int(H), int(Id), _p(x), T, _p(w_gate_up), _p(w_down), _p(y), ws.cptr, ws.nbytes,
+                             _stream(stream)))
+    return y

@@ -23,6 +23,11 @@
  *             (bailing_hybrid)", paragraph "MoE routing".
  *   [GGUF]    page "Ling-3.0-flash-GGUF", "Measured performance": decode reads
  *             only the selected experts' weights.
+ *   [DENSE]   mlxcel issue #838, "Architecture notes": the first
+ *             first_k_dense_replace layers use a plain MLP at
+ *             intermediate_size instead of the MoE block; model card
+ *             "Ling-2.6-flash-JANGTQ", "Architecture (bailing_hybrid)", layer
+ *             table: layer 0 is a dense MLP of intermediate size 9216.
  *
  * Conventions for every entry point:
  *   - Pointers are DEVICE pointers unless stated otherwise. bf16 tensors are
@@ -182,11 +187,13 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
                        uint16_t* y, void* stream);
 
 /* The whole block: router logits -> route -> permute -> experts -> combine.
- * With the automatic expert path (moe_set_ffn_path(0)) and T <= 2 tokens, the
- * block runs as one cooperative launch (MOE_KERNEL_DECODE_FUSED) whose phases
- * are separated by bounded grid barriers; the routing, weights and output are
- * those of the separate kernels, up to fp32 summation order in the logits and
- * expert dot products.
+ * With the automatic expert path (moe_set_ffn_path(0)), T <= 2 tokens, at most
+ * 32 slots (T*k), E <= 1024 and H <= 8192, the block runs as one cooperative
+ * launch (MOE_KERNEL_DECODE_FUSED): a weight-streaming kernel, one CTA per SM,
+ * with one bounded grid barrier and bounded per-expert and per-row counters.
+ * Its routing (indices and weights) is bit-identical to moe_route on the same
+ * logits; its logits and output equal those of the separate kernels up to the
+ * fp32 summation order of the dot products.
  *   logits_override [T,E] fp32 or NULL: when given, replaces the router
  *   projection (router_w may then be NULL).
  *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
@@ -197,6 +204,18 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
                        const uint16_t* ws_gate_up, const uint16_t* ws_down,
                        uint16_t* y, int32_t* topk_idx_out, float* topk_w_out,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* The dense-prefix MLP ([DENSE]): y = W_down (silu(W_gate x) * (W_up x)), bf16
+ * in and out, fp32 accumulation, on the expert kernels of moe_expert_ffn (the
+ * MLP is run as a block of one expert, one slot per token, weight 1.0).
+ *   w_gate_up [2*intermediate_size, hidden_size] bf16: rows [0, Id) gate_proj,
+ *   rows [Id, 2Id) up_proj. w_down [hidden_size, intermediate_size] bf16.
+ *   x, y [T, hidden_size] bf16. hidden_size and intermediate_size must be
+ *   multiples of 8. ws / ws_bytes >= moe_dense_mlp_workspace_size(.., T). */
+size_t moe_dense_mlp_workspace_size(int32_t hidden_size, int32_t intermediate_size, int64_t max_tokens);
+moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const uint16_t* x, int64_t T,
+                         const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* y,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace error word (after an
  * error the whole 256-byte header is cleared, barrier state included). Returns

@@ -25,6 +25,11 @@ Sources (page title, then section):
   (bailing_hybrid)", paragraph "MoE routing": sigmoid, 8 groups, top-4
   groups, top-8 experts, e_score_correction_bias for selection only, "same
   math as DeepSeek-V3".
+* [DENSE]  mlxcel issue #838, section "Architecture notes": the first
+  first_k_dense_replace layers use a plain MLP at intermediate_size instead
+  of the MoE block; model card "Ling-2.6-flash-JANGTQ", section
+  "Architecture (bailing_hybrid)", layer table: layer 0 is a dense MLP of
+  intermediate size 9216.
 
 Precision. The pages fix the router's precision: the score function runs in
 float32 and the weights stay float32 through normalisation and scaling
@@ -287,6 +292,15 @@ def swiglu_mlp(X: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.n
     g = X @ w_gate.T
     u = X @ w_up.T
     return (silu(g) * u) @ w_down.T
+
+
+def dense_mlp(x, w_gate_up, w_down) -> np.ndarray:
+    """The dense-prefix MLP [DENSE]: down_proj(silu(gate_proj(x)) * up_proj(x))
+    with the gate/up weights stacked [2*Id, H] (gate rows first) and down_proj
+    [H, Id]; fp64 on the exact upcast of the bf16 inputs."""
+    wgu = as_f64(w_gate_up)
+    Id = wgu.shape[0] // 2
+    return swiglu_mlp(as_f64(x), wgu[:Id], wgu[Id:], as_f64(w_down))
 
 
 def expert_weights_f64(w_gate_up, w_down, e: int, I: int):

@@ -186,3 +186,33 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+DENSE_BAD = [
+    # hidden, intermediate, tokens, ws given, status, field named in the message
+    (0, 9216, 1, True, 1, "hidden_size"),
+    (4100, 9216, 1, True, 2, "hidden_size"),
+    (4096, 0, 1, True, 1, "intermediate_size"),
+    (4096, 9217, 1, True, 2, "intermediate_size"),
+    (4096, 1 << 20, 1, True, 1, "intermediate_size"),
+    (4096, 9216, -1, True, 1, "T"),
+    (4096, 9216, 4, False, 3, "workspace"),
+]
+
+
+@pytest.mark.parametrize("H,Id,T,with_ws,status,field", DENSE_BAD)
+def test_dense_mlp_rejects_before_launch(M, H, Id, T, with_ws, status, field):
+    # Host-side rejection: nothing is launched, so this runs without a GPU.
+    fake = ctypes.c_void_p(1 << 20)
+    ws = fake if with_ws else None
+    n0 = M.lib.moe_launch_count()
+    st = M.lib.moe_dense_mlp(H, Id, fake, T, fake, fake, fake, ws, 1 << 40, None)
+    assert st == status, (st, M.last_error())
+    assert field in M.last_error()
+    assert M.lib.moe_launch_count() == n0
+
+
+def test_dense_mlp_workspace_size(M):
+    assert M.lib.moe_dense_mlp_workspace_size(4096, 9216, 64) > 64 * 4096 * 4  # at least the fp32 rows
+    assert M.lib.moe_dense_mlp_workspace_size(4096, 9217, 64) == 0
+    assert "intermediate_size" in M.last_error()

@@ -327,6 +327,37 @@ def test_scale_zero_leaves_shared_only():
     check_scale_zero_leaves_shared_only()
 
 
+def test_dense_mlp_brute_force():
+    # [DENSE]: y[t, n] = sum_i Wd[n, i] * silu(g_i) * u_i with g_i = Wg[i] . x_t and
+    # u_i = Wu[i] . x_t, written out with Python floats and math.exp (no numpy
+    # matmul), gate rows first in the stacked weight.
+    H, Id, T = 8, 4, 3
+    inp = G.make_dense_inputs(H, Id, T, seed=3)
+    y = O.dense_mlp(inp["x"], inp["w_gate_up"], inp["w_down"])
+    x, wgu, wd = O.as_f64(inp["x"]), O.as_f64(inp["w_gate_up"]), O.as_f64(inp["w_down"])
+    assert y.shape == (T, H)
+    for t in range(T):
+        h = []
+        for i in range(Id):
+            g = sum(float(wgu[i, c]) * float(x[t, c]) for c in range(H))
+            u = sum(float(wgu[Id + i, c]) * float(x[t, c]) for c in range(H))
+            h.append(g / (1.0 + math.exp(-g)) * u)
+        for n in range(H):
+            ref = sum(float(wd[n, i]) * h[i] for i in range(Id))
+            assert abs(y[t, n] - ref) <= 1e-12 * (1.0 + abs(ref)), (t, n, y[t, n], ref)
+
+
+def test_dense_mlp_is_a_one_expert_softmax_block():
+    # A softmax over a single expert scores exactly 1, so a block with one routed
+    # expert, k = 1, scale 1 and no shared MLP computes that expert's MLP: the
+    # dense MLP with the expert's weights.
+    wl, inp = _tiny_inputs(seed=12, num_experts=1, num_experts_per_tok=1, score_function="softmax",
+                           norm_topk_prob=False, routed_scaling_factor=1.0, num_shared_experts=0, shared_width=0)
+    y = O.moe_block(inp, wl)["y"]
+    ref = O.dense_mlp(inp["x"], inp["w_gate_up"][0], inp["w_down"][0])
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-13), np.abs(y - ref).max()
+
+
 def test_permutation_definition():
     rng = np.random.default_rng(10)
     T, E, k = 37, 12, 3

@@ -452,3 +452,42 @@ def test_forward_zero_tokens_and_launch_count(M):
                   inp["ws_down"], ws)
     ws.check()
     assert M.launch_count() > n0
+
+
+# ---------------------------------------------------------------------------
+# dense-prefix MLP (moe_dense_mlp): the Ling-2.6-flash layer-0 MLP (hidden
+# 4096, intermediate 9216) on both expert paths, and small ragged shapes
+# ---------------------------------------------------------------------------
+DENSE_CASES = [
+    # hidden, intermediate, tokens, expert path
+    (4096, 9216, 1, "auto"),          # streaming (T <= 2)
+    (4096, 9216, 2, "auto"),
+    (4096, 9216, 5, "auto"),          # tensor cores, one partial token tile
+    (4096, 9216, 130, "auto"),        # token-major tiles: one full, one ragged
+    (4096, 9216, 9, "streaming"),
+    (192, 200, 37, "streaming"),      # K and N not multiples of the tile sizes
+    (192, 200, 37, "tensor_cores"),
+    (64, 32, 1, "tensor_cores"),
+]
+
+
+@pytest.mark.parametrize("H,Id,T,path", DENSE_CASES, ids=[f"H{c[0]}-I{c[1]}-T{c[2]}-{c[3]}" for c in DENSE_CASES])
+def test_dense_mlp(M, H, Id, T, path):
+    inp = G.make_dense_inputs(H, Id, T, seed=21, device=DEV)
+    ws = M.dense_mlp_workspace(H, Id, T)
+    M.set_ffn_path(path)
+    try:
+        y = M.moe_dense_mlp(inp["x"], inp["w_gate_up"], inp["w_down"], ws)
+        ws.check()
+    finally:
+        M.set_ffn_path("auto")
+    ref = O.dense_mlp(inp["x"], inp["w_gate_up"], inp["w_down"])
+    S.compare(O.as_f64(y), ref, f"dense MLP H={H} Id={Id} T={T} {path}")
+
+
+def test_dense_mlp_zero_tokens_launches_nothing(M):
+    inp = G.make_dense_inputs(64, 32, 1, seed=2, device=DEV)
+    ws = M.dense_mlp_workspace(64, 32, 1)
+    n0 = M.launch_count()
+    y = M.moe_dense_mlp(inp["x"][:0], inp["w_gate_up"], inp["w_down"], ws)
+    assert y.shape == (0, 64) and M.launch_count() == n0
