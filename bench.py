@@ -98,17 +98,18 @@ def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str):
     return entry[0] if kernel_source_hash(kernel) == entry[1] else None
 
 
-def algorithmic(wl, T, n_unique):
+def algorithmic(wl, T, n_unique, weight_bytes=2.0):
     """Bytes each expert pass must move, and the block's flops, given the
-    number of distinct routed experts the batch touched. Activations count at
-    the width this design stores them: token rows bf16 (2 B), the SwiGLU
-    product as two bf16 planes (4 B), expert slot rows and the shared MLP
-    output fp32 (4 B)."""
+    number of distinct routed experts the batch touched. Expert weights count
+    weight_bytes per element (2 for bf16; 1 + 4 / group for 8-bit affine codes
+    with a bf16 scale and bias per group). Activations count at the width this
+    design stores them: token rows bf16 (2 B), the SwiGLU product as two bf16
+    planes or fp32 (4 B), expert slot rows and the shared MLP output fp32 (4 B)."""
     H, E, k, I, Is = (wl["hidden_size"], wl["num_experts"], wl["num_experts_per_tok"],
                       wl["moe_intermediate_size"], wl["shared_width"])
     R = T * k
-    w_gate_up = (n_unique * 2 * I + 2 * Is) * H * 2
-    w_down = (n_unique * I + Is) * H * 2
+    w_gate_up = int((n_unique * 2 * I + 2 * Is) * H * weight_bytes)
+    w_down = int((n_unique * I + Is) * H * weight_bytes)
     h_elems = R * I + T * Is
     gate_up_bytes = w_gate_up + (R + T) * H * 2 + h_elems * 4   # weights + token rows in + h planes out
     down_bytes = w_down + h_elems * 4 + (R + T) * H * 4          # weights + h planes in + fp32 rows out
@@ -291,8 +292,9 @@ def run_ours(args):
     wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
+    q8 = G.make_q8_weights(wl, seed=0, device=dev, group_size=args.q8) if args.q8 else None
     if args.kernel == "auto":
-        fused = args.ffn_path == "auto" and T <= M.FUSED_DECODE_MAX_TOKENS
+        fused = args.ffn_path == "auto" and T <= M.FUSED_DECODE_MAX_TOKENS and q8 is None
         args.kernel = "decode_fused" if fused else "expert_gate_up"
     if rank > 0:  # each rank its own batch (weak scaling), same weights
         g = torch.Generator(device=dev)
@@ -304,6 +306,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(x=None):
+        if q8 is not None:
+            return M.moe_forward_q8(wl, inp["x"] if x is None else x, inp["router_w"], inp["expert_bias"], q8, ws, y=y)
         return M.moe_forward(wl, inp["x"] if x is None else x, inp["router_w"], inp["expert_bias"],
                              inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"], inp["ws_down"], ws, y=y)
 
@@ -317,7 +321,7 @@ def run_ours(args):
     _, idx, _ = M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
                               inp["ws_gate_up"], inp["ws_down"], ws, return_routing=True)
     n_unique = int(torch.unique(idx).numel())
-    work = algorithmic(wl, T, n_unique)
+    work = algorithmic(wl, T, n_unique, 1.0 + 4.0 / args.q8 if q8 is not None else 2.0)
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -381,7 +385,7 @@ def run_ours(args):
     else:
         kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
         kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
-    traffic = measured_traffic(args.kernel, args.workload, args.set, args.ffn_path)
+    traffic = None if q8 is not None else measured_traffic(args.kernel, args.workload, args.set, args.ffn_path)
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if kflops / kbytes > ridge:
@@ -421,6 +425,7 @@ def run_ours(args):
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
                    "experts_touched": n_unique, "parallelism": f"replicas x{world} (token batches)",
+                   "expert_weights": f"8-bit affine, group {args.q8}" if q8 is not None else "bf16",
                    "l2": "256 MiB L2 flush between timed steps; expert weights >> 126 MB L2"},
         "step_hbm_gbs": step_gbs, "step_tflops": step_tflops,
         "roofline": roofline,
@@ -429,6 +434,113 @@ def run_ours(args):
                 "d2h_bytes_per_step": int(y_host.numel() * 2)},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def dense_algorithmic(H, Id, T):
+    """Bytes of each pass and flops of the dense MLP: weights once, token rows
+    bf16 in, the SwiGLU product at 4 B per element, fp32 rows out of the down
+    pass."""
+    gate_up_bytes = 2 * Id * H * 2 + T * H * 2 + T * Id * 4
+    down_bytes = H * Id * 2 + T * Id * 4 + T * H * 4
+    return dict(gate_up_bytes=gate_up_bytes, down_bytes=down_bytes, step_bytes=3 * H * Id * 2 + 2 * T * H * 2,
+                gate_up_flops=2 * T * H * 2 * Id, flops=2 * T * H * 3 * Id)
+
+
+def run_dense(args):
+    """The dense-prefix MLP (moe_dense_mlp) on the Ling-2.6-flash layer-0 shape
+    (hidden 4096, intermediate 9216), one GPU, T = args.dense tokens."""
+    from grouped_top_routing_b200 import moe as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H, Id, T = G.LING26_DENSE["hidden_size"], G.LING26_DENSE["intermediate_size"], args.dense
+    inp = G.make_dense_inputs(H, Id, T, seed=0, device=dev)
+    ws = M.dense_mlp_workspace(H, Id, T)
+    y = torch.empty_like(inp["x"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x=None):
+        return M.moe_dense_mlp(inp["x"] if x is None else x, inp["w_gate_up"], inp["w_down"], ws, y=y)
+
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in kev:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    launches0 = M.launch_count()
+    with ClockSampler(0) as clk:
+        for i in range(K):
+            flush.zero_()  # L2 flush, outside the timed events
+            M.set_kernel_timer("expert_gate_up", kev[i][0], kev[i][1])
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        M.set_kernel_timer("expert_gate_up")
+        torch.cuda.synchronize(dev)
+    launches = M.launch_count() - launches0
+    ws.check()
+    ms_per_step = sum(a.elapsed_time(b) for a, b in ev) / K
+    kms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        eev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in eev) / K
+
+    work = dense_algorithmic(H, Id, T)
+    pk = peaks()
+    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    kb, kf = work["gate_up_bytes"], work["gate_up_flops"]
+    if kf / kb > ridge:
+        achieved = kf / (kms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "expert_gate_up", "achieved": achieved, "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                    "peak_source": pk["source"] + " (bf16 burst)", "algorithmic_flops": kf, "algorithmic_bytes": kb,
+                    "kernel_ms": kms}
+    else:
+        achieved = kb / (kms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "expert_gate_up", "achieved": achieved, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
+                    "algorithmic_bytes": kb, "algorithmic_flops": kf, "kernel_ms": kms}
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import moe_oracle as O
+        n = min(T, 8)
+        t0 = time.perf_counter()
+        O.dense_mlp(inp["x"][:n], inp["w_gate_up"], inp["w_down"])
+        secs = time.perf_counter() - t0
+        cpu = {"value": n / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {n} tokens, fp64 numpy oracle, one pass", "seconds": secs}
+    line = {
+        "metric": "dense-prefix MLP tokens/s at 1 B200 (Ling-2.6-flash layer 0)", "value": T / (ms_per_step / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": warm, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"ling26_flash_dense_mlp_t{T}", "hidden_size": H, "intermediate_size": Id,
+                   "tokens": T, "l2": "256 MiB L2 flush between timed steps; weights 226 MB > 126 MB L2"},
+        "step_hbm_gbs": work["step_bytes"] / (ms_per_step / 1e3) / 1e9,
+        "roofline": roofline, "cpu_baseline": cpu,
+        "e2e": {"value": T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2)},
+        "gpu_launches": int(launches), "clocks": clk.summary(),
     }
     print(json.dumps(line))
     return 0
@@ -451,7 +563,13 @@ def main():
                     help="expert-FFN kernels (default: the library's automatic choice)")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (e.g. num_experts=64 for a small profiling case)")
+    ap.add_argument("--q8", type=int, default=0, metavar="GROUP",
+                    help="run the block with 8-bit affine expert weights of this group size (32, 64 or 128)")
+    ap.add_argument("--dense", type=int, default=0, metavar="TOKENS",
+                    help="time the dense-prefix MLP (Ling-2.6-flash layer 0) on TOKENS tokens instead of the block")
     args = ap.parse_args()
+    if args.dense > 0:
+        return run_dense(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -5,6 +5,14 @@
 
 namespace moe {
 
+// 8-bit affine weight matrix: for each row and each group of `group`
+// consecutive inputs, w = scale * q + bias (q uint8, scale and bias bf16).
+struct Q8Mat {
+  const uint8_t* q;       // [rows, K]
+  const uint16_t* scale;  // [rows, K / group]
+  const uint16_t* bias;   // [rows, K / group]
+};
+
 struct FfnArgs {
   const uint16_t* x;          // [T, H]
   int64_t T;
@@ -22,6 +30,11 @@ struct FfnArgs {
   void* h_shared;             // [T, Is]: same element type as h_perm
   float* y_slots;             // [T*k, H]
   float* shared_out;          // [T, H]
+  // 8-bit affine weights (streaming path only): group > 0 selects them for the
+  // routed experts; the shared MLP is 8-bit when qs_gate_up.q is set, else bf16.
+  int group;
+  Q8Mat q_gate_up, q_down;    // [E*2I, H], [E*H, I]
+  Q8Mat qs_gate_up, qs_down;  // [2Is, H], [H, Is]
 };
 
 cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s);

@@ -8,7 +8,11 @@
 //
 // Work items are single weight rows (gate/up pass) or blocks of ROWS rows
 // (down pass) of the experts in the compacted active list written by the
-// permutation, plus the shared MLP's rows. One warp per item: lanes stride the
+// permutation, plus the shared MLP's rows. Weights are bf16, or 8-bit affine
+// (w = scale * q + bias per group of inputs, scale and bias bf16: the 8-bit
+// recipes of the pages "Ling-3.0-tiny-8bit-XL-mlx", section "XL Quantization
+// Recipe", and "Ling-2.6-flash-JANGTQ", quantization summary), dequantised in
+// the stream. One warp per item: lanes stride the
 // row in 16-byte chunks (ld.global.nc, no L1 allocation), every token routed
 // to that expert is multiplied against the chunk, and the warp reduces with
 // shuffles. Tokens are taken MT at a time (MT follows the batch, up to 8); an
@@ -50,9 +54,99 @@ __device__ __forceinline__ int64_t slot_token(const FfnArgs& a, int64_t row, int
   return slot / a.k;
 }
 
-// Gate/up pass: one warp per intermediate index j of one expert, streaming its
-// gate row and up row (H bf16 each) against up to MT tokens per pass.
+constexpr int kUnrollQ = 4;  // 16-byte chunks in flight per lane per 8-bit weight row
+
+__device__ __forceinline__ float bf16_word(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
+// Sum of the 16 products of one 16-byte chunk of 8-bit affine weights
+// (w = s * q + b, one fp32 rounding) with 16 fp32 values.
+__device__ __forceinline__ float dot16_q8(uint4 q, float s, float b, const float* v, float acc) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float qi = (float)((w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+    acc = fmaf(fmaf(s, qi, b), v[i], acc);
+  }
+  return acc;
+}
+
+// Gate and up dot products of one bf16 row pair (H each) against up to MT
+// token rows (xr[t]; null: no token).
 template <int MT>
+__device__ __forceinline__ void rowpair_bf16(const uint16_t* gate, const uint16_t* up, int H,
+                                             const uint16_t* const (&xr)[MT], float (&ag)[MT], float (&au)[MT]) {
+  const int lane = threadIdx.x & 31, nv = H / 8;
+  for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+    uint4 gv[kUnroll], uv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+        gv[u] = ld_stream_u4(gate + v * 8);
+        uv[u] = ld_stream_u4(up + v * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (xr[t] != nullptr) {
+            float xf[8];
+            unpack8_bf16(ld_nc_u4(xr[t] + v * 8), xf);
+            ag[t] = dot8_bf16(gv[u], xf, ag[t]);
+            au[t] = dot8_bf16(uv[u], xf, au[t]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// The same for rows rg (gate) and ru (up) of an 8-bit affine matrix.
+template <int MT>
+__device__ __forceinline__ void rowpair_q8(const Q8Mat& m, int64_t rg, int64_t ru, int H, int group,
+                                           const uint16_t* const (&xr)[MT], float (&ag)[MT], float (&au)[MT]) {
+  const int lane = threadIdx.x & 31, nv = H / 16, ng = H / group;
+  const uint8_t* gq = m.q + rg * H;
+  const uint8_t* uq = m.q + ru * H;
+  for (int v0 = lane; v0 < nv; v0 += 32 * kUnrollQ) {
+    uint4 gv[kUnrollQ], uv[kUnrollQ];
+#pragma unroll
+    for (int u = 0; u < kUnrollQ; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+        gv[u] = ld_stream_u4(gq + v * 16);
+        uv[u] = ld_stream_u4(uq + v * 16);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnrollQ; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+        const int g = v * 16 / group;  // a 16-element chunk lies in one group
+        const float sg = bf16_word(__ldg(m.scale + rg * ng + g)), bg = bf16_word(__ldg(m.bias + rg * ng + g));
+        const float su = bf16_word(__ldg(m.scale + ru * ng + g)), bu = bf16_word(__ldg(m.bias + ru * ng + g));
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (xr[t] != nullptr) {
+            float xf[16];
+            unpack8_bf16(ld_nc_u4(xr[t] + v * 16), xf);
+            unpack8_bf16(ld_nc_u4(xr[t] + v * 16 + 8), xf + 8);
+            ag[t] = dot16_q8(gv[u], sg, bg, xf, ag[t]);
+            au[t] = dot16_q8(uv[u], su, bu, xf, au[t]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Gate/up pass: one warp per intermediate index j of one expert, streaming its
+// gate row and up row (bf16, or 8-bit affine when Q8) against up to MT tokens
+// per pass.
+template <int MT, bool Q8>
 __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
   pdl_launch_dependents();
   pdl_wait();
@@ -61,25 +155,20 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int n_act = min(max(*(volatile int*)&a.hdr->num_active, 0), a.E);
   const int64_t routed_items = (int64_t)n_act * a.I;
-  const int64_t total = routed_items + (a.ws_gate_up != nullptr ? a.Is : 0);
-  const int H = a.H, nv = H / 8;
+  const bool has_shared = a.ws_gate_up != nullptr || (Q8 && a.qs_gate_up.q != nullptr);
+  const int64_t total = routed_items + (has_shared ? a.Is : 0);
+  const int H = a.H;
 
   for (int64_t item = gw; item < total; item += nw) {
     const bool shared = item >= routed_items;
-    int j;
-    const uint16_t *gate, *up;
+    int j, e = 0;
     int64_t r0 = 0, m = 0;
     if (!shared) {
       const int aidx = (int)(item / a.I);
       j = (int)(item - (int64_t)aidx * a.I);
-      int e;
       if (!expert_rows(a, aidx, e, r0, m)) continue;
-      gate = a.w_gate_up + ((int64_t)e * 2 * a.I + j) * H;
-      up = gate + (int64_t)a.I * H;
     } else {
       j = (int)(item - routed_items);
-      gate = a.ws_gate_up + (int64_t)j * H;
-      up = gate + (int64_t)a.Is * H;
       m = a.T;
     }
     for (int64_t c0 = 0; c0 < m; c0 += MT) {
@@ -97,32 +186,23 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
       float ag[MT], au[MT];
 #pragma unroll
       for (int t = 0; t < MT; ++t) ag[t] = au[t] = 0.0f;
-      for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
-        uint4 gv[kUnroll], uv[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nv) {
-            gv[u] = ld_stream_u4(gate + v * 8);
-            uv[u] = ld_stream_u4(up + v * 8);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nv) {
-#pragma unroll
-            for (int t = 0; t < MT; ++t) {
-              if (xr[t] != nullptr) {
-                float xf[8];
-                unpack8_bf16(ld_nc_u4(xr[t] + v * 8), xf);
-                ag[t] = dot8_bf16(gv[u], xf, ag[t]);
-                au[t] = dot8_bf16(uv[u], xf, au[t]);
-              }
-            }
-          }
-        }
+      // the row pair: 8-bit (routed rows when Q8; shared rows when 8-bit too) or bf16
+      const Q8Mat* qm = nullptr;
+      int64_t rg, ru;
+      const uint16_t* wbase;
+      if (!shared) {
+        rg = (int64_t)e * 2 * a.I + j;
+        ru = rg + a.I;
+        wbase = a.w_gate_up;
+        if (Q8) qm = &a.q_gate_up;
+      } else {
+        rg = j;
+        ru = (int64_t)a.Is + j;
+        wbase = a.ws_gate_up;
+        if (Q8 && a.qs_gate_up.q != nullptr) qm = &a.qs_gate_up;
       }
+      if (Q8 && qm != nullptr) rowpair_q8<MT>(*qm, rg, ru, H, a.group, xr, ag, au);
+      else rowpair_bf16<MT>(wbase + rg * H, wbase + ru * H, H, xr, ag, au);
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         if (t < mc) {
@@ -139,9 +219,71 @@ __global__ void __launch_bounds__(256) gemv_gate_up_kernel(FfnArgs a) {
   }
 }
 
-// Down pass: one warp per block of ROWS output rows of one expert; the rows
-// (I bf16 each) are streamed together against up to MT tokens' h per pass.
+// ROWS bf16 rows (K each, row r at w0 + r*K) against up to MT fp32 h rows
+// (hin + (hrow0 + t) * K).
 template <int MT, int ROWS>
+__device__ __forceinline__ void rows_bf16(const uint16_t* w0, int nrows, int K, const float* hin, int64_t hrow0,
+                                          int mc, float (&acc)[ROWS][MT]) {
+  const int lane = threadIdx.x & 31, nvk = K / 8;
+#pragma unroll 2
+  for (int v = lane; v < nvk; v += 32) {
+    uint4 wv[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+      if (r < nrows) wv[r] = ld_stream_u4(w0 + (int64_t)r * K + v * 8);
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      if (t < mc) {
+        const float4* hp = reinterpret_cast<const float4*>(hin + (hrow0 + t) * K + v * 8);
+        const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
+        const float hf[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r)
+          if (r < nrows) acc[r][t] = dot8_bf16(wv[r], hf, acc[r][t]);
+      }
+    }
+  }
+}
+
+// The same for rows row0 .. row0 + nrows of an 8-bit affine matrix.
+template <int MT, int ROWS>
+__device__ __forceinline__ void rows_q8(const Q8Mat& m, int64_t row0, int nrows, int K, int group, const float* hin,
+                                        int64_t hrow0, int mc, float (&acc)[ROWS][MT]) {
+  const int lane = threadIdx.x & 31, nv = K / 16, ng = K / group;
+  for (int v = lane; v < nv; v += 32) {
+    const int g = v * 16 / group;
+    uint4 wv[ROWS];
+    float sc[ROWS], bi[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      if (r < nrows) {
+        wv[r] = ld_stream_u4(m.q + (row0 + r) * K + v * 16);
+        sc[r] = bf16_word(__ldg(m.scale + (row0 + r) * ng + g));
+        bi[r] = bf16_word(__ldg(m.bias + (row0 + r) * ng + g));
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      if (t < mc) {
+        const float4* hp = reinterpret_cast<const float4*>(hin + (hrow0 + t) * K + v * 16);
+        float hf[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 h4 = __ldg(hp + i);
+          hf[4 * i] = h4.x, hf[4 * i + 1] = h4.y, hf[4 * i + 2] = h4.z, hf[4 * i + 3] = h4.w;
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r)
+          if (r < nrows) acc[r][t] = dot16_q8(wv[r], sc[r], bi[r], hf, acc[r][t]);
+      }
+    }
+  }
+}
+
+// Down pass: one warp per block of ROWS output rows of one expert; the rows
+// (I each, bf16 or 8-bit affine when Q8) are streamed together against up to
+// MT tokens' h per pass.
+template <int MT, int ROWS, bool Q8>
 __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
   pdl_launch_dependents();
   pdl_wait();
@@ -153,30 +295,26 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
   const int H = a.H;
   const int nrb = (H + ROWS - 1) / ROWS;
   const int64_t routed_items = (int64_t)n_act * nrb;
-  const int64_t total = routed_items + (a.ws_down != nullptr ? nrb : 0);
+  const bool has_shared = a.ws_down != nullptr || (Q8 && a.qs_down.q != nullptr);
+  const int64_t total = routed_items + (has_shared ? nrb : 0);
 
   for (int64_t item = gw; item < total; item += nw) {
     const bool shared = item >= routed_items;
-    int n0, K;
-    const uint16_t* w0;
+    int n0, K, e = 0;
     const float* hin;
     int64_t r0 = 0, m = 0;
     if (!shared) {
       const int aidx = (int)(item / nrb);
       n0 = (int)(item - (int64_t)aidx * nrb) * ROWS;
-      int e;
       if (!expert_rows(a, aidx, e, r0, m)) continue;
       K = a.I;
-      w0 = a.w_down + ((int64_t)e * H + n0) * K;
       hin = static_cast<const float*>(a.h_perm);
     } else {
       n0 = (int)(item - routed_items) * ROWS;
       K = a.Is;
-      w0 = a.ws_down + (int64_t)n0 * K;
       hin = static_cast<const float*>(a.h_shared);
       m = a.T;
     }
-    const int nvk = K / 8;
     const int nrows = min(ROWS, H - n0);
     for (int64_t c0 = 0; c0 < m; c0 += MT) {
       const int mc = (int)min((int64_t)MT, m - c0);
@@ -185,24 +323,11 @@ __global__ void __launch_bounds__(256) gemv_down_kernel(FfnArgs a) {
       for (int r = 0; r < ROWS; ++r)
 #pragma unroll
         for (int t = 0; t < MT; ++t) acc[r][t] = 0.0f;
-#pragma unroll 2
-      for (int v = lane; v < nvk; v += 32) {
-        uint4 wv[ROWS];
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r)
-          if (r < nrows) wv[r] = ld_stream_u4(w0 + (int64_t)r * K + v * 8);
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          if (t < mc) {
-            const float4* hp = reinterpret_cast<const float4*>(hin + (r0 + c0 + t) * K + v * 8);
-            const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
-            const float hf[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r)
-              if (r < nrows) acc[r][t] = dot8_bf16(wv[r], hf, acc[r][t]);
-          }
-        }
-      }
+      const Q8Mat* qm = nullptr;
+      const int64_t row0 = shared ? n0 : (int64_t)e * H + n0, hrow0 = shared ? c0 : r0 + c0;
+      if (Q8) qm = shared ? (a.qs_down.q != nullptr ? &a.qs_down : nullptr) : &a.q_down;
+      if (Q8 && qm != nullptr) rows_q8<MT, ROWS>(*qm, row0, nrows, K, a.group, hin, hrow0, mc, acc);
+      else rows_bf16<MT, ROWS>((shared ? a.ws_down : a.w_down) + row0 * K, nrows, K, hin, hrow0, mc, acc);
       float mine = 0.0f;
 #pragma unroll
       for (int r = 0; r < ROWS; ++r)
@@ -273,26 +398,32 @@ int resident_blocks(K kernel) {
   return sm_count() * per_sm;
 }
 
-template <int MT, int ROWS>
+template <int MT, int ROWS, bool Q8>
 cudaError_t launch_gemv_mt(const FfnArgs& a, cudaStream_t s) {
   before_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
-  launch_pdl(gemv_gate_up_kernel<MT>, dim3(resident_blocks(gemv_gate_up_kernel<MT>)), dim3(256), 0, s, a);
+  launch_pdl(gemv_gate_up_kernel<MT, Q8>, dim3(resident_blocks(gemv_gate_up_kernel<MT, Q8>)), dim3(256), 0, s, a);
   after_launch(MOE_KERNEL_EXPERT_GATE_UP, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   before_launch(MOE_KERNEL_EXPERT_DOWN, s);
-  launch_pdl(gemv_down_kernel<MT, ROWS>, dim3(resident_blocks(gemv_down_kernel<MT, ROWS>)), dim3(256), 0, s, a);
+  launch_pdl(gemv_down_kernel<MT, ROWS, Q8>, dim3(resident_blocks(gemv_down_kernel<MT, ROWS, Q8>)), dim3(256), 0, s,
+             a);
   after_launch(MOE_KERNEL_EXPERT_DOWN, s);
   return cudaGetLastError();
+}
+
+template <bool Q8>
+cudaError_t launch_gemv_fmt(const FfnArgs& a, cudaStream_t s) {
+  if (a.T <= 1) return launch_gemv_mt<1, 8, Q8>(a, s);
+  if (a.T <= 2) return launch_gemv_mt<2, 8, Q8>(a, s);
+  if (a.T <= 4) return launch_gemv_mt<4, 4, Q8>(a, s);
+  return launch_gemv_mt<8, 4, Q8>(a, s);
 }
 
 // Tokens per pass follow the batch (an expert has at most T rows), so the
 // single-token decode step carries one accumulator per row.
 cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s) {
-  if (a.T <= 1) return launch_gemv_mt<1, 8>(a, s);
-  if (a.T <= 2) return launch_gemv_mt<2, 8>(a, s);
-  if (a.T <= 4) return launch_gemv_mt<4, 4>(a, s);
-  return launch_gemv_mt<8, 4>(a, s);
+  return a.group > 0 ? launch_gemv_fmt<true>(a, s) : launch_gemv_fmt<false>(a, s);
 }
 
 cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,

@@ -279,10 +279,14 @@ bool use_tensor_cores(const moe_config& c, int64_t T) {
   return T > kStreamMaxT;
 }
 
+Q8Mat q8mat(const moe_q8_matrix& m) { return Q8Mat{m.q, m.scale, m.bias}; }
+
+// q8: 8-bit affine expert weights (dequantised by the streaming kernels), or
+// null for bf16 weights.
 moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint16_t* x_perm,
                    const int32_t* offsets, const int32_t* tok_of, const float* topk_w, const uint16_t* wgu,
                    const uint16_t* wd, const uint16_t* swgu, const uint16_t* swd, float* y_slots, float* shared_out,
-                   void* ws, bool active_ready, cudaStream_t s) {
+                   void* ws, bool active_ready, cudaStream_t s, const moe_q8_weights* q8 = nullptr) {
   const Layout L = layout(c, T);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
   int32_t* active = at<int32_t>(ws, L.active);
@@ -312,6 +316,20 @@ moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint
   a.h_shared = at<void>(ws, L.h_shared);
   a.y_slots = y_slots;
   a.shared_out = shared_out;
+  if (q8 != nullptr) {
+    a.group = q8->group_size;
+    a.q_gate_up = q8mat(q8->gate_up);
+    a.q_down = q8mat(q8->down);
+    if (q8->shared_gate_up.q != nullptr && a.Is > 0) {
+      a.qs_gate_up = q8mat(q8->shared_gate_up);
+      a.qs_down = q8mat(q8->shared_down);
+      a.ws_gate_up = nullptr;
+      a.ws_down = nullptr;
+    }
+    e = launch_gemv_ffn(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "expert ffn (8-bit)");
+    return MOE_OK;
+  }
   if (use_tensor_cores(c, T)) {
     if (x_perm == nullptr) {  // the tensor-core path reads expert rows contiguously
       uint16_t* xp = at<uint16_t>(ws, L.x_perm);
@@ -344,6 +362,50 @@ moe_config dense_config(int32_t hidden_size, int32_t intermediate_size) {
   c.num_shared_experts = 0;
   c.moe_shared_expert_intermediate_size = 0;
   return c;
+}
+
+moe_status check_q8_matrix(const char* name, const moe_q8_matrix& m) {
+  char field[64];
+  std::snprintf(field, sizeof field, "%s.q", name);
+  MOE_TRY(check_ptr(field, m.q, 16, true));
+  std::snprintf(field, sizeof field, "%s.scale", name);
+  MOE_TRY(check_ptr(field, m.scale, 16, true));
+  std::snprintf(field, sizeof field, "%s.bias", name);
+  MOE_TRY(check_ptr(field, m.bias, 16, true));
+  return MOE_OK;
+}
+
+// 8-bit weights: group size, divisibility of every row length by it, and the
+// pointers (the shared MLP either 8-bit or bf16, as the config requires).
+moe_status validate_q8(const moe_config& c, const moe_q8_weights* w, const uint16_t* ws_gate_up,
+                       const uint16_t* ws_down) {
+  if (w == nullptr) return fail(MOE_ERR_INVALID_ARG, "8-bit weights (w) is NULL");
+  const int g = w->group_size;
+  if (g != 32 && g != 64 && g != 128)
+    return fail(MOE_ERR_UNSUPPORTED, "group_size = %d is not 32, 64 or 128", g);
+  const int Is = shared_width(c);
+  if (c.hidden_size % g != 0) return fail(MOE_ERR_UNSUPPORTED, "hidden_size = %d not divisible by group_size = %d", c.hidden_size, g);
+  if (c.moe_intermediate_size % g != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_intermediate_size = %d not divisible by group_size = %d",
+                c.moe_intermediate_size, g);
+  MOE_TRY(check_q8_matrix("gate_up", w->gate_up));
+  MOE_TRY(check_q8_matrix("down", w->down));
+  const bool shared_q8 = w->shared_gate_up.q != nullptr;
+  if (Is == 0) {
+    if (shared_q8 || ws_gate_up != nullptr)
+      return fail(MOE_ERR_INVALID_ARG, "shared MLP weights given but the config has no shared MLP");
+    return MOE_OK;
+  }
+  if (shared_q8) {
+    if (Is % g != 0) return fail(MOE_ERR_UNSUPPORTED, "shared MLP width %d not divisible by group_size = %d", Is, g);
+    if (ws_gate_up != nullptr) return fail(MOE_ERR_INVALID_ARG, "shared MLP given both as 8-bit and as bf16 (ws_gate_up)");
+    MOE_TRY(check_q8_matrix("shared_gate_up", w->shared_gate_up));
+    MOE_TRY(check_q8_matrix("shared_down", w->shared_down));
+    return MOE_OK;
+  }
+  MOE_TRY(check_ptr("ws_gate_up", ws_gate_up, 16, true));
+  MOE_TRY(check_ptr("ws_down", ws_down, 16, true));
+  return MOE_OK;
 }
 
 moe_status validate_dense(int32_t hidden_size, int32_t intermediate_size) {
@@ -634,6 +696,52 @@ moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const u
   MOE_TRY(run_ffn(c, T, x, x, offsets, tok_of, w, w_gate_up, w_down, nullptr, nullptr, y_slots, nullptr, ws, false, s));
   e = launch_combine(y_slots, nullptr, T, 1, hidden_size, y, s);
   if (e != cudaSuccess) return cuda_fail(e, "dense output");
+  return MOE_OK;
+}
+
+moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
+                          const float* expert_bias, const float* logits_override, const moe_q8_weights* w,
+                          const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y, int32_t* topk_idx_out,
+                          float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  const moe_config& c = *cfg;
+  MOE_TRY(validate_q8(c, w, ws_gate_up, ws_down));
+  if (T == 0) return MOE_OK;
+  const bool has_shared = shared_width(c) > 0;
+  MOE_TRY(check_ptr("x", x, 16, true));
+  MOE_TRY(check_ptr("logits_override", logits_override, 4, false));
+  MOE_TRY(check_ptr("router_w", router_w, 16, logits_override == nullptr));
+  MOE_TRY(check_ptr("expert_bias", expert_bias, 4, false));
+  MOE_TRY(check_ptr("y", y, 16, true));
+  MOE_TRY(check_ptr("topk_idx_out", topk_idx_out, 4, false));
+  MOE_TRY(check_ptr("topk_w_out", topk_w_out, 4, false));
+  const Layout L = layout(c, T);
+  cudaStream_t s = as_stream(stream);
+  WsHeader* hdr = at<WsHeader>(ws, L.hdr);
+  const float* logits = logits_override;
+  cudaError_t e;
+  if (logits == nullptr) {
+    float* lg = at<float>(ws, L.logits);
+    MOE_TRY(run_logits(c, x, T, router_w, lg, ws, s));
+    logits = lg;
+  }
+  int32_t* idx = topk_idx_out != nullptr ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+  float* tw = topk_w_out != nullptr ? topk_w_out : at<float>(ws, L.topk_w);
+  e = launch_route(c, logits, expert_bias, T, idx, tw, s);
+  if (e != cudaSuccess) return cuda_fail(e, "route");
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* tok_of = at<int32_t>(ws, L.tok_of);
+  e = launch_permute(c, idx, T, x, offsets, at<int32_t>(ws, L.row_of), tok_of, nullptr, at<int32_t>(ws, L.active),
+                     at<int32_t>(ws, L.tile_cnt), at<int32_t>(ws, L.tile_base), hdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute");
+  float* y_slots = at<float>(ws, L.y_slots);
+  float* shared_out = has_shared ? at<float>(ws, L.shared_out) : nullptr;
+  MOE_TRY(run_ffn(c, T, x, nullptr, offsets, tok_of, tw, nullptr, nullptr, has_shared ? ws_gate_up : nullptr,
+                  has_shared ? ws_down : nullptr, y_slots, shared_out, ws, true, s, w));
+  e = launch_combine(y_slots, shared_out, T, c.num_experts_per_tok, c.hidden_size, y, s);
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
   return MOE_OK;
 }
 

@@ -174,6 +174,39 @@ def make_inputs(wl: dict, seed: int = 0, device="cpu", tokens: int | None = None
     return out
 
 
+def _q8_matrix(shape, group_size, gen, device):
+    """Codes, scales and biases of an 8-bit affine matrix [..., R, K] whose
+    dequantised weights are about N(0, 1/sqrt(K)): codes 128 + 40 N(0, 1)
+    clipped to [0, 255], scale (sigma / 40) * U(0.75, 1.25) per group, bias
+    -128 * scale + N(0, sigma / 16) per group (scale and bias bf16)."""
+    K = shape[-1]
+    sigma = 1.0 / math.sqrt(K)
+    gshape = tuple(shape[:-1]) + (K // group_size,)
+    q = (torch.randn(shape, generator=gen, device=device) * 40.0 + 128.0).round_().clamp_(0, 255).to(torch.uint8)
+    scale = (torch.rand(gshape, generator=gen, device=device) * 0.5 + 0.75) * (sigma / 40.0)
+    bias = -128.0 * scale + torch.randn(gshape, generator=gen, device=device) * (sigma / 16.0)
+    return q, scale.to(torch.bfloat16), bias.to(torch.bfloat16)
+
+
+def make_q8_weights(wl: dict, seed: int = 0, device="cpu", group_size: int = 64, shared: bool = True) -> dict:
+    """8-bit affine expert weights for a workload (drawn directly, seeded):
+    gate_up [E, 2I, H], down [E, H, I] and, when ``shared``, the shared MLP's
+    [2Is, H] and [H, Is]; each a (q, scale, bias) triple."""
+    device = torch.device(device)
+    H, E, I, Is = wl["hidden_size"], wl["num_experts"], wl["moe_intermediate_size"], wl["shared_width"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 77)
+    parts = [_q8_matrix((1, 2 * I, H), group_size, gen, device) for _ in range(E)]
+    gate_up = tuple(torch.cat([p[i] for p in parts]) for i in range(3))
+    parts = [_q8_matrix((1, H, I), group_size, gen, device) for _ in range(E)]
+    down = tuple(torch.cat([p[i] for p in parts]) for i in range(3))
+    out = {"group_size": group_size, "gate_up": gate_up, "down": down, "shared_gate_up": None, "shared_down": None}
+    if shared and Is > 0:
+        out["shared_gate_up"] = _q8_matrix((2 * Is, H), group_size, gen, device)
+        out["shared_down"] = _q8_matrix((H, Is), group_size, gen, device)
+    return out
+
+
 # Dense-prefix MLP of Ling-2.6-flash: hidden 4096, intermediate 9216 (model card
 # "Ling-2.6-flash-JANGTQ", section "Architecture (bailing_hybrid)", layer table).
 LING26_DENSE = dict(hidden_size=4096, intermediate_size=9216)

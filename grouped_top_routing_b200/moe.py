@@ -27,7 +27,7 @@ FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch at
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
            "moe_set_ffn_path", "moe_launch_count", "moe_last_error", "moe_permute_static",
-           "moe_dense_mlp_workspace_size", "moe_dense_mlp")
+           "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 
 
@@ -65,6 +65,27 @@ def config_from_workload(wl: dict) -> MoeConfig:
     )
 
 
+class Q8Matrix(ctypes.Structure):
+    """moe_q8_matrix: codes [R, K] uint8, scale and bias [R, K / group_size] bf16."""
+    _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+
+
+class Q8Weights(ctypes.Structure):
+    """moe_q8_weights."""
+    _fields_ = [("group_size", ctypes.c_int32), ("gate_up", Q8Matrix), ("down", Q8Matrix),
+                ("shared_gate_up", Q8Matrix), ("shared_down", Q8Matrix)]
+
+
+def q8_weights(q8: dict) -> Q8Weights:
+    """ctypes view of a dict of (q, scale, bias) tensor triples (see inputs.make_q8_weights)."""
+    def mat(t):
+        if t is None:
+            return Q8Matrix(None, None, None)
+        return Q8Matrix(*(ctypes.c_void_p(x.data_ptr()) for x in t))
+    return Q8Weights(int(q8["group_size"]), mat(q8["gate_up"]), mat(q8["down"]), mat(q8.get("shared_gate_up")),
+                     mat(q8.get("shared_down")))
+
+
 def _load():
     if not os.path.exists(library_path):
         raise ImportError(f"{library_path} is not built; run `python -m grouped_top_routing_b200.build`")
@@ -86,6 +107,7 @@ def _load():
         "moe_permute_static": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp]),
         "moe_dense_mlp_workspace_size": (sz, [ctypes.c_int32, ctypes.c_int32, i64]),
         "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp]),
+        "moe_forward_q8": (st, [cfgp, vp, i64, vp, vp, vp, ctypes.POINTER(Q8Weights), vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -265,4 +287,26 @@ def moe_dense_mlp(x, w_gate_up, w_down, ws: Workspace, y=None, stream=None):
         y = torch.empty_like(x)
     _check(lib.moe_dense_mlp(int(H), int(Id), _p(x), T, _p(w_gate_up), _p(w_down), _p(y), ws.cptr, ws.nbytes,
                              _stream(stream)))
+    return y
+
+
+def moe_forward_q8(cfg, x, router_w, expert_bias, q8: dict, ws: Workspace, ws_gate_up=None, ws_down=None,
+                   logits_override=None, y=None, return_routing=False, stream=None):
+    """The block with 8-bit affine expert weights (q8 as in inputs.make_q8_weights);
+    the shared MLP is q8's when present, else the bf16 ws_gate_up / ws_down."""
+    c = _as_cfg(cfg)
+    T = x.shape[0]
+    k = c.num_experts_per_tok
+    if y is None:
+        y = torch.empty_like(x)
+    idx = w = None
+    if return_routing:
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    qw = q8_weights(q8)
+    _check(lib.moe_forward_q8(ctypes.byref(c), _p(x), T, _p(router_w), _p(expert_bias), _p(logits_override),
+                              ctypes.byref(qw), _p(ws_gate_up), _p(ws_down), _p(y), _p(idx), _p(w), ws.cptr,
+                              ws.nbytes, _stream(stream)))
+    if return_routing:
+        return y, idx, w
     return y

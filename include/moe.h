@@ -23,6 +23,12 @@
  *             (bailing_hybrid)", paragraph "MoE routing".
  *   [GGUF]    page "Ling-3.0-flash-GGUF", "Measured performance": decode reads
  *             only the selected experts' weights.
+ *   [Q8]      model card "Ling-3.0-tiny-8bit-XL-mlx", "XL Quantization Recipe"
+ *             (routed experts and the dense MLP 8-bit; router and shared
+ *             experts bf16); model card "Ling-2.6-flash-JANGTQ", quantization
+ *             summary (8-bit affine on the shared experts and the layer-0
+ *             dense MLP); mlxcel issue #838, "Upstream sanitize" (quantized
+ *             expert tensors carry weight, scales and biases; group size 64).
  *   [DENSE]   mlxcel issue #838, "Architecture notes": the first
  *             first_k_dense_replace layers use a plain MLP at
  *             intermediate_size instead of the MoE block; model card
@@ -216,6 +222,35 @@ size_t moe_dense_mlp_workspace_size(int32_t hidden_size, int32_t intermediate_si
 moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const uint16_t* x, int64_t T,
                          const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* y,
                          void* ws, size_t ws_bytes, void* stream);
+
+/* 8-bit affine weights ([Q8]): for each row and each group of `group_size`
+ * consecutive inputs, w = scale * q + bias, with q uint8 and scale, bias bf16
+ * (raw bits). A matrix of R rows and K inputs: q [R, K], scale and bias
+ * [R, K / group_size], all row-major, 16-byte aligned. */
+typedef struct {
+  const uint8_t*  q;
+  const uint16_t* scale;
+  const uint16_t* bias;
+} moe_q8_matrix;
+
+typedef struct {
+  int32_t group_size;           /* 32, 64 or 128; divides H, I and Is */
+  moe_q8_matrix gate_up;        /* routed experts: R = E*2I, K = H (rows as w_gate_up) */
+  moe_q8_matrix down;           /* routed experts: R = E*H,  K = I (rows as w_down) */
+  moe_q8_matrix shared_gate_up; /* R = 2Is, K = H; q NULL: the shared MLP is bf16 (ws_* of moe_forward_q8) */
+  moe_q8_matrix shared_down;    /* R = H, K = Is */
+} moe_q8_weights;
+
+/* The whole block with 8-bit affine expert weights, dequantised in the
+ * streaming expert kernels (every T; the router projection stays fp32). The
+ * shared MLP is 8-bit when w->shared_gate_up.q is set, else bf16 from
+ * ws_gate_up / ws_down (the XL recipe keeps it bf16). Routing, permutation and
+ * combine are those of moe_forward. H, I and Is must be multiples of 16 (one
+ * 16-byte chunk of codes per lane step). ws / ws_bytes >= moe_workspace_size. */
+moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
+                          const float* expert_bias, const float* logits_override, const moe_q8_weights* w,
+                          const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y,
+                          int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace error word (after an
  * error the whole 256-byte header is cleared, barrier state included). Returns

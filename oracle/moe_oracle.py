@@ -25,6 +25,12 @@ Sources (page title, then section):
   (bailing_hybrid)", paragraph "MoE routing": sigmoid, 8 groups, top-4
   groups, top-8 experts, e_score_correction_bias for selection only, "same
   math as DeepSeek-V3".
+* [Q8]     model card "Ling-3.0-tiny-8bit-XL-mlx", section "XL Quantization
+  Recipe" (routed experts 8-bit); model card "Ling-2.6-flash-JANGTQ",
+  quantization summary (8-bit affine on the shared experts); mlxcel issue
+  #838, section "Upstream sanitize" (quantized expert tensors carry weight,
+  scales and biases; group size 64). The affine form: for each row and each
+  group of g consecutive inputs, w = scale * q + bias.
 * [DENSE]  mlxcel issue #838, section "Architecture notes": the first
   first_k_dense_replace layers use a plain MLP at intermediate_size instead
   of the MoE block; model card "Ling-2.6-flash-JANGTQ", section
@@ -301,6 +307,43 @@ def dense_mlp(x, w_gate_up, w_down) -> np.ndarray:
     wgu = as_f64(w_gate_up)
     Id = wgu.shape[0] // 2
     return swiglu_mlp(as_f64(x), wgu[:Id], wgu[Id:], as_f64(w_down))
+
+
+def dequant_affine(q, scale, bias, group_size: int) -> np.ndarray:
+    """8-bit affine weights [Q8]: w[..., c] = scale[..., c // g] * q[..., c] +
+    bias[..., c // g] with q uint8 and scale, bias bf16; exact in fp64."""
+    qf = as_f64(q)
+    s = np.repeat(as_f64(scale), group_size, axis=-1)
+    b = np.repeat(as_f64(bias), group_size, axis=-1)
+    return s * qf + b
+
+
+class _DequantStack:
+    """Expert-indexed view of stacked 8-bit weights (q [E, R, K], scale and
+    bias [E, R, K / g]) that dequantises one expert when indexed."""
+
+    def __init__(self, mat, group_size: int):
+        self.q, self.scale, self.bias = mat
+        self.g = group_size
+
+    def __getitem__(self, e):
+        return dequant_affine(self.q[e], self.scale[e], self.bias[e], self.g)
+
+
+def moe_block_q8(inp: dict, cfg: dict, q8: dict, logits=None, tokens=None) -> dict:
+    """The MoE block with 8-bit affine expert weights [Q8]: every expert's
+    weights dequantised, then the block exactly as ``moe_block``. ``q8`` holds
+    group_size and (q, scale, bias) triples gate_up [E, 2I, H], down [E, H, I]
+    and, when the shared MLP is 8-bit, shared_gate_up [2Is, H] and shared_down
+    [H, Is]; otherwise the shared MLP is ``inp``'s bf16 one."""
+    g = q8["group_size"]
+    view = dict(inp)
+    view["w_gate_up"] = _DequantStack(q8["gate_up"], g)
+    view["w_down"] = _DequantStack(q8["down"], g)
+    if q8.get("shared_gate_up") is not None:
+        view["ws_gate_up"] = dequant_affine(*q8["shared_gate_up"], g)
+        view["ws_down"] = dequant_affine(*q8["shared_down"], g)
+    return moe_block(view, cfg, logits=logits, tokens=tokens)
 
 
 def expert_weights_f64(w_gate_up, w_down, e: int, I: int):

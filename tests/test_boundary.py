@@ -216,3 +216,47 @@ def test_dense_mlp_workspace_size(M):
     assert M.lib.moe_dense_mlp_workspace_size(4096, 9216, 64) > 64 * 4096 * 4  # at least the fp32 rows
     assert M.lib.moe_dense_mlp_workspace_size(4096, 9217, 64) == 0
     assert "intermediate_size" in M.last_error()
+
+
+def _q8(M, group=64, shared=True, misalign=None):
+    fake = 1 << 20
+    def mat(name):
+        if name.startswith("shared") and not shared:
+            return M.Q8Matrix(None, None, None)
+        p = [ctypes.c_void_p(fake), ctypes.c_void_p(fake), ctypes.c_void_p(fake)]
+        if misalign == name:
+            p[0] = ctypes.c_void_p(fake + 8)
+        return M.Q8Matrix(*p)
+    return M.Q8Weights(group, mat("gate_up"), mat("down"), mat("shared_gate_up"), mat("shared_down"))
+
+
+Q8_BAD = [
+    # description, weights factory args, bf16 shared given, status, text in the message
+    ("group 48", dict(group=48), False, 2, "group_size"),
+    ("group 256", dict(group=256), False, 2, "group_size"),
+    ("unaligned codes", dict(misalign="down"), False, 1, "down.q"),
+    ("shared twice", dict(), True, 1, "both"),
+    ("shared missing", dict(shared=False), False, 1, "ws_gate_up"),
+]
+
+
+@pytest.mark.parametrize("what,wargs,bf16_shared,status,text", Q8_BAD, ids=[b[0] for b in Q8_BAD])
+def test_forward_q8_rejects_before_launch(M, what, wargs, bf16_shared, status, text):
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    w = _q8(M, **wargs)
+    n0 = M.lib.moe_launch_count()
+    st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, ctypes.byref(w),
+                              fake if bf16_shared else None, fake if bf16_shared else None, fake, None, None,
+                              fake, 1 << 40, None)
+    assert st == status, (st, M.last_error())
+    assert text in M.last_error(), M.last_error()
+    assert M.lib.moe_launch_count() == n0
+
+
+def test_forward_q8_rejects_null_weights(M):
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, None, None, None, fake, None, None,
+                              fake, 1 << 40, None)
+    assert st == 1 and "NULL" in M.last_error()

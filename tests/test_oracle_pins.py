@@ -358,6 +358,45 @@ def test_dense_mlp_is_a_one_expert_softmax_block():
     assert np.allclose(y, ref, rtol=1e-13, atol=1e-13), np.abs(y - ref).max()
 
 
+def test_dequant_affine_brute_force():
+    # [Q8]: w[r, c] = scale[r, c // g] * q[r, c] + bias[r, c // g], written out
+    # element by element with Python floats.
+    wl = G.tiny_workload(num_experts=2, num_experts_per_tok=1, hidden_size=64, moe_intermediate_size=32, shared_width=32)
+    q8 = G.make_q8_weights(wl, seed=4, group_size=32)
+    q, sc, bi = q8["down"]  # [E, H, I] = [2, 64, 32]: one group per row
+    w = O.dequant_affine(q, sc, bi, 32)
+    qn, sn, bn = q.numpy(), O.as_f64(sc), O.as_f64(bi)
+    q, sc, bi = q8["gate_up"]  # [2, 64, 64]: two groups per row
+    w2 = O.dequant_affine(q, sc, bi, 32)
+    qn2, sn2, bn2 = q.numpy(), O.as_f64(sc), O.as_f64(bi)
+    for e in range(2):
+        for r in range(64):
+            for c in range(32):
+                assert w[e, r, c] == float(sn[e, r, 0]) * int(qn[e, r, c]) + float(bn[e, r, 0])
+            for c in range(64):
+                assert w2[e, r, c] == float(sn2[e, r, c // 32]) * int(qn2[e, r, c]) + float(bn2[e, r, c // 32])
+
+
+def test_q8_block_with_integer_weights_is_the_bf16_block():
+    # scale 1/64 and bias -2 dequantise to q/64 - 2, which bf16 holds exactly
+    # (at most 8 significant bits): the 8-bit block must then equal the bf16
+    # block on those values.
+    wl, inp = _tiny_inputs(seed=13, num_experts=4, num_experts_per_tok=2, score_function="sigmoid", bias="normal",
+                           routed_scaling_factor=2.5)
+    g = 32
+    q8 = G.make_q8_weights(wl, seed=13, group_size=g)
+    for key in ("gate_up", "down", "shared_gate_up", "shared_down"):
+        q, sc, bi = q8[key]
+        q8[key] = (q, torch.full_like(sc, 1.0 / 64.0), torch.full_like(bi, -2.0))
+    ints = {key: (q8[key][0].to(torch.float32) / 64.0 - 2.0).to(torch.bfloat16)
+            for key in ("gate_up", "down", "shared_gate_up", "shared_down")}
+    bf = dict(inp, w_gate_up=ints["gate_up"], w_down=ints["down"], ws_gate_up=ints["shared_gate_up"],
+              ws_down=ints["shared_down"])
+    a = O.moe_block_q8(inp, wl, q8)["y"]
+    b = O.moe_block(bf, wl)["y"]
+    assert np.array_equal(a, b)
+
+
 def test_permutation_definition():
     rng = np.random.default_rng(10)
     T, E, k = 37, 12, 3

@@ -491,3 +491,44 @@ def test_dense_mlp_zero_tokens_launches_nothing(M):
     n0 = M.launch_count()
     y = M.moe_dense_mlp(inp["x"][:0], inp["w_gate_up"], inp["w_down"], ws)
     assert y.shape == (0, 64) and M.launch_count() == n0
+
+
+# ---------------------------------------------------------------------------
+# 8-bit affine expert weights (moe_forward_q8), dequantised in the streaming
+# kernels: routing bit-exact on given logits, output against the oracle on the
+# dequantised weights
+# ---------------------------------------------------------------------------
+Q8_CASES = [
+    # workload, tokens, group size, shared MLP 8-bit (else bf16, the XL recipe)
+    ("ling30_flash_decode_t1", 1, 64, True),
+    ("ling30_flash_decode_t8", 2, 64, False),
+    ("ling30_flash_decode_t8", 8, 64, True),
+    ("ling26_flash_t512", 17, 128, True),    # grouped routing; 17 tokens: several token passes
+    ("ling_lite_t64", 5, 64, True),          # softmax, Is = 2I
+    ("tiny_q8", 37, 32, True),
+]
+
+
+@pytest.mark.parametrize("name,T,group,shared", Q8_CASES, ids=[f"{c[0]}-T{c[1]}-g{c[2]}-{'q8' if c[3] else 'bf16'}shared"
+                                                               for c in Q8_CASES])
+def test_forward_q8(M, name, T, group, shared):
+    if name == "tiny_q8":
+        wl = G.tiny_workload(tokens=T, hidden_size=64, num_experts=48, num_experts_per_tok=5, n_group=4, topk_group=2,
+                             score_function="sigmoid", bias="normal", moe_intermediate_size=96, shared_width=96,
+                             routed_scaling_factor=2.5, name="tiny_q8")
+        inp = G.make_inputs(wl, seed=4, device=DEV)
+    else:
+        wl, inp = _inputs(name)
+    q8 = G.make_q8_weights(wl, seed=3, device=DEV, group_size=group, shared=shared)
+    x = inp["x"][:T].contiguous()
+    L = G.random_logits(T, wl["num_experts"], S.logit_std(wl), seed=31).numpy()
+    ws = M.Workspace(wl, T)
+    y, idx, w = M.moe_forward_q8(wl, x, inp["router_w"], inp["expert_bias"], q8, ws,
+                                 ws_gate_up=None if shared else inp["ws_gate_up"],
+                                 ws_down=None if shared else inp["ws_down"],
+                                 logits_override=torch.from_numpy(L).to(DEV), return_routing=True)
+    ws.check()
+    ref = O.moe_block_q8(dict(inp, x=x, tokens=T), wl, q8, logits=L)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), np.asarray(ref["w"], np.float32).view(np.uint32))
+    S.compare(O.as_f64(y), ref["y"], f"q8 {name} T={T} group {group}")
