@@ -50,12 +50,12 @@ namespace moe {
 
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 12;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kFusedThreads = kConsumers + 32;  // + the producer warp
 constexpr int kFusedMaxT = 2;
 constexpr int kMaxSlots = 32;      // T * k: one warp lane per slot
-constexpr int kMaxChunk = 8;       // experts per lane in a warp's slice: 1024 / (4 warps * 32 lanes)
+constexpr int kMaxChunk = 8;       // experts per lane in a warp's slice: 1024 / (6 warps * 32 lanes), rounded up
 constexpr int kMaxStages = 16;
 constexpr int kMinStages = 4;
 constexpr int kMaxDownRows = 16;   // rows per down block: lane t*16 + r holds (slot or token t, row r)
@@ -90,6 +90,7 @@ struct FusedSmem {
   int n_act;
   int flag;
   volatile int abort;  // a consumer warp stopped before the grid barrier
+  unsigned int next_unit;  // the next stream unit a consumer warp may claim
 };
 
 struct Range {
@@ -97,11 +98,11 @@ struct Range {
 };
 
 // Dynamic shared memory after the ring: routing scratch ([T*E] fp32 scores,
-// [T*E] fp32 biased scores, [T*E] 64-bit keys), then the token rows (bf16)
-// and the expert bias (fp32).
+// [T*E] fp32 biased scores, [T*E] 64-bit keys), then the token rows (fp32,
+// converted once) and the expert bias (fp32).
 __host__ __device__ __forceinline__ size_t route_scratch_bytes(int T, int E) { return (size_t)T * E * 16; }
 __host__ __device__ __forceinline__ size_t scratch_bytes(int T, int E, int H) {
-  return route_scratch_bytes(T, E) + (size_t)T * H * 2 + (size_t)E * 4;
+  return route_scratch_bytes(T, E) + (size_t)T * H * 4 + (size_t)E * 4;
 }
 
 // Contiguous share b of G of `total` items.
@@ -277,25 +278,25 @@ __device__ __forceinline__ void dot8x2(uint4 w, const float* v, float& e, float&
 
 // One fp32 router row (H) against up to two bf16 token rows. Returns the logit
 // of token 0 in lane 0 and of token 1 in lane 16.
-__device__ __forceinline__ float router_unit(const float* w, int H, const uint16_t* xs, int T, uint64_t* empty) {
+__device__ __forceinline__ float router_unit(const float* w, int H, const float* xs, int T, uint64_t* empty) {
   const int lane = threadIdx.x & 31;
-  const uint2* x0 = reinterpret_cast<const uint2*>(xs);
-  const uint2* x1 = reinterpret_cast<const uint2*>(xs + H);
+  const float4* x0 = reinterpret_cast<const float4*>(xs);
+  const float4* x1 = reinterpret_cast<const float4*>(xs + H);
   float e0 = 0.f, o0 = 0.f, e1 = 0.f, o1 = 0.f;
 #pragma unroll 2
   for (int c = lane; c < H / 4; c += 32) {
     const float4 w4 = reinterpret_cast<const float4*>(w)[c];
-    const uint2 xa = x0[c];
-    e0 = fmaf(bf16_lo(xa.x), w4.x, e0);
-    o0 = fmaf(bf16_hi(xa.x), w4.y, o0);
-    e0 = fmaf(bf16_lo(xa.y), w4.z, e0);
-    o0 = fmaf(bf16_hi(xa.y), w4.w, o0);
+    const float4 xa = x0[c];
+    e0 = fmaf(xa.x, w4.x, e0);
+    o0 = fmaf(xa.y, w4.y, o0);
+    e0 = fmaf(xa.z, w4.z, e0);
+    o0 = fmaf(xa.w, w4.w, o0);
     if (T > 1) {
-      const uint2 xb = x1[c];
-      e1 = fmaf(bf16_lo(xb.x), w4.x, e1);
-      o1 = fmaf(bf16_hi(xb.x), w4.y, o1);
-      e1 = fmaf(bf16_lo(xb.y), w4.z, e1);
-      o1 = fmaf(bf16_hi(xb.y), w4.w, o1);
+      const float4 xb = x1[c];
+      e1 = fmaf(xb.x, w4.x, e1);
+      o1 = fmaf(xb.y, w4.y, o1);
+      e1 = fmaf(xb.z, w4.z, e1);
+      o1 = fmaf(xb.w, w4.w, o1);
     }
   }
   release_stage(empty);
@@ -306,22 +307,23 @@ __device__ __forceinline__ float router_unit(const float* w, int H, const uint16
 // One gate row and one up row (H bf16 each) against up to two token rows:
 // returns silu(gate . x_t) * (up . x_t) for token row 0 in lane 0 and for
 // token row 1 in lane 16, fp32.
-__device__ __forceinline__ float gate_up_unit(const uint16_t* gate, const uint16_t* up, int H, const uint16_t* x0,
-                                              const uint16_t* x1, uint64_t* empty) {
+__device__ __forceinline__ float gate_up_unit(const uint16_t* gate, const uint16_t* up, int H, const float* x0,
+                                              const float* x1, uint64_t* empty) {
   const int lane = threadIdx.x & 31;
   float ve[4] = {0.f, 0.f, 0.f, 0.f}, vo[4] = {0.f, 0.f, 0.f, 0.f};  // gate . x0, up . x0, gate . x1, up . x1
 #pragma unroll 2
   for (int c = lane; c < H / 8; c += 32) {
     const uint4 gv = reinterpret_cast<const uint4*>(gate)[c];
     const uint4 uv = reinterpret_cast<const uint4*>(up)[c];
-    float xf[8];
-    unpack8_bf16(reinterpret_cast<const uint4*>(x0)[c], xf);
+    const float4 a0 = reinterpret_cast<const float4*>(x0)[2 * c], a1 = reinterpret_cast<const float4*>(x0)[2 * c + 1];
+    const float xf[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     dot8x2(gv, xf, ve[0], vo[0]);
     dot8x2(uv, xf, ve[1], vo[1]);
     if (x1 != nullptr) {
-      unpack8_bf16(reinterpret_cast<const uint4*>(x1)[c], xf);
-      dot8x2(gv, xf, ve[2], vo[2]);
-      dot8x2(uv, xf, ve[3], vo[3]);
+      const float4 b0 = reinterpret_cast<const float4*>(x1)[2 * c], b1 = reinterpret_cast<const float4*>(x1)[2 * c + 1];
+      const float xg[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      dot8x2(gv, xg, ve[2], vo[2]);
+      dot8x2(uv, xg, ve[3], vo[3]);
     }
   }
   release_stage(empty);
@@ -712,56 +714,98 @@ __device__ __forceinline__ Seg segment(const DecodeArgs& a, const Geo& g, int n_
   return sg;
 }
 
-// The producer thread: issues the CTA's stream in order, unit u into ring slot
-// u % depth once the consumer of the slot's previous unit freed it.
-__device__ void producer(const DecodeArgs& a, const Geo& g, unsigned char* ring, FusedSmem& sm) {
+// The global rows of one stream unit: up to two contiguous pieces.
+struct UnitSrc {
+  const void* p0;
+  const void* p1;
+  uint32_t n0, n1;
+};
+
+__device__ __forceinline__ UnitSrc unit_src(const DecodeArgs& a, const Geo& g, const FusedSmem& sm, const Seg& sg,
+                                           int i) {
   const int H = a.H, I = a.I, Is = a.Is;
   const int n_router = a.logits_override == nullptr ? a.E : 0;
+  UnitSrc u{nullptr, nullptr, 0u, 0u};
+  if (sg.kind == kSegA) {
+    if (i < n_router) {
+      u.p0 = a.router_w + (int64_t)i * H;
+      u.n0 = 4u * H;
+    } else {
+      const int j = i - n_router;
+      u.p0 = a.ws_gate_up + (int64_t)j * H;
+      u.p1 = a.ws_gate_up + (int64_t)(Is + j) * H;
+      u.n0 = u.n1 = 2u * H;
+    }
+  } else if (sg.kind == kSegS) {
+    const int n0 = i * g.rs, rows = min(g.rs, H - n0);
+    u.p0 = a.ws_down + (int64_t)n0 * Is;
+    u.n0 = 2u * rows * Is;
+  } else if (sg.kind == kSegC) {
+    const uint16_t* gate = a.w_gate_up + ((int64_t)sm.act_e[sg.ai] * 2 * I + i) * H;
+    u.p0 = gate;
+    u.p1 = gate + (int64_t)I * H;
+    u.n0 = u.n1 = 2u * H;
+  } else {
+    const int n0 = i * g.rd, rows = min(g.rd, H - n0);
+    u.p0 = a.w_down + ((int64_t)sm.act_e[sg.ai] * H + n0) * I;
+    u.n0 = 2u * rows * I;
+  }
+  return u;
+}
+
+// A position in the CTA's stream: segment si, item i of its share.
+struct Cursor {
+  int si, i;
+  Seg sg;
+};
+
+// Moves c past finished segments to its next unit; false when none is left in
+// the first nseg segments (c then stays on its last segment, so that it can
+// resume once nseg grows).
+__device__ __forceinline__ bool cursor_valid(const DecodeArgs& a, const Geo& g, int n_act, int nseg, Cursor& c) {
+  while (c.i >= c.sg.r.lo + c.sg.r.n) {
+    if (c.si + 1 >= nseg) return false;
+    ++c.si;
+    c.sg = segment(a, g, n_act, c.si);
+    c.i = c.sg.r.lo;
+  }
+  return true;
+}
+
+// The producer thread: issues the CTA's stream in order, unit u into ring slot
+// u % depth once the consumer of the slot's previous unit freed it. (Bulk L2
+// prefetches of the units ahead of the ring were measured here and made the
+// step 1.5x slower.)
+__device__ void producer(const DecodeArgs& a, const Geo& g, unsigned char* ring, FusedSmem& sm) {
   uint32_t u = 0;
   bool ok = true;
-  auto issue = [&](const void* src0, uint32_t n0, const void* src1, uint32_t n1) {
+  int nseg = 2, n_act = 0;  // the segments after S need this CTA's routing
+  Cursor c{0, 0, segment(a, g, 0, 0)};
+  c.i = c.sg.r.lo;
+  for (;;) {
+    if (!cursor_valid(a, g, n_act, nseg, c)) {
+      if (nseg > 2) break;
+      // end of S: wait for the routing, then continue with the selected experts
+      ok = thread_wait_phase(&sm.route_ready, 0, a.hdr, 500);
+      if (!ok) break;
+      n_act = sm.n_act;
+      nseg = num_segments(n_act);
+      continue;
+    }
     const int s = (int)(u % (uint32_t)g.depth);
     const uint32_t n = u / (uint32_t)g.depth;
     if (n > 0 && !thread_wait_phase(&sm.empty[s], (n - 1) & 1u, a.hdr, 400 + s)) {
       ok = false;
-      return;
+      break;
     }
+    const UnitSrc q = unit_src(a, g, sm, c.sg, c.i);
     sm.tag[s] = u;  // the slot's previous fill is consumed: its phase is complete
-    mbar_expect_tx(&sm.full[s], n0 + n1);
+    mbar_expect_tx(&sm.full[s], q.n0 + q.n1);
     unsigned char* dst = ring + (size_t)s * g.stage_bytes;
-    bulk_load(dst, src0, n0, &sm.full[s]);
-    if (n1 != 0) bulk_load(dst + n0, src1, n1, &sm.full[s]);
+    bulk_load(dst, q.p0, q.n0, &sm.full[s]);
+    if (q.n1 != 0) bulk_load(dst + q.n0, q.p1, q.n1, &sm.full[s]);
+    ++c.i;
     ++u;
-  };
-  int nseg = 2, n_act = 0;
-  for (int si = 0; ok && si < nseg; ++si) {
-    const Seg sg = segment(a, g, n_act, si);
-    for (int i = sg.r.lo; ok && i < sg.r.lo + sg.r.n; ++i) {
-      if (sg.kind == kSegA) {
-        if (i < n_router) {
-          issue(a.router_w + (int64_t)i * H, 4u * H, nullptr, 0);
-        } else {
-          const int j = i - n_router;
-          issue(a.ws_gate_up + (int64_t)j * H, 2u * H, a.ws_gate_up + (int64_t)(Is + j) * H, 2u * H);
-        }
-      } else if (sg.kind == kSegS) {
-        const int n0 = i * g.rs, rows = min(g.rs, H - n0);
-        issue(a.ws_down + (int64_t)n0 * Is, 2u * rows * Is, nullptr, 0);
-      } else if (sg.kind == kSegC) {
-        const uint16_t* gate = a.w_gate_up + ((int64_t)sm.act_e[sg.ai] * 2 * I + i) * H;
-        issue(gate, 2u * H, gate + (int64_t)I * H, 2u * H);
-      } else {
-        const int n0 = i * g.rd, rows = min(g.rd, H - n0);
-        issue(a.w_down + ((int64_t)sm.act_e[sg.ai] * H + n0) * I, 2u * rows * I, nullptr, 0);
-      }
-    }
-    if (si == 1 && ok) {  // the segments after S need this CTA's routing
-      ok = thread_wait_phase(&sm.route_ready, 0, a.hdr, 500);
-      if (ok) {
-        n_act = sm.n_act;
-        nseg = num_segments(n_act);
-      }
-    }
   }
   if (!ok) {
     // the consumers stopped: wait (bounded) for the copies still in flight
@@ -771,12 +815,17 @@ __device__ void producer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
   }
 }
 
-// First stream index at or after `base` that belongs to consumer warp w.
-__device__ __forceinline__ uint32_t first_unit(uint32_t base, int w) {
-  return base + (uint32_t)((w - (int)(base % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
+// The next unclaimed stream unit of the CTA, for the whole warp. Warps claim
+// units in stream order as they become free, so a warp that drew short units
+// takes more of them: no warp is left with a static share that outlasts the
+// others.
+__device__ __forceinline__ uint32_t claim_unit(FusedSmem& sm) {
+  uint32_t u = 0;
+  if ((threadIdx.x & 31) == 0) u = atomicAdd(&sm.next_unit, 1u);
+  return __shfl_sync(0xffffffffu, u, 0);
 }
 
-// A consumer warp: stream units w, w + 8, ... of its CTA.
+// A consumer warp: claims its CTA's stream units in order (claim_unit).
 __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring, unsigned char* scratch,
                          FusedSmem& sm) {
   const int T = a.T, k = a.k, H = a.H, I = a.I, Is = a.Is, E = a.E;
@@ -787,11 +836,15 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
   const Range z = split(kMaxSlots + kFusedMaxT * H, blockIdx.x, gridDim.x);
   for (int i = threadIdx.x; i < z.n; i += kConsumers) a.sync[z.lo + i] = 0;
 
-  // token rows and expert bias into shared memory (one coalesced pass)
-  uint16_t* xs = reinterpret_cast<uint16_t*>(scratch + route_scratch_bytes(T, E));
-  float* bias_s = a.expert_bias != nullptr ? reinterpret_cast<float*>(xs + (size_t)T * H) : nullptr;
-  for (int i = threadIdx.x; i < T * H / 8; i += kConsumers)
-    reinterpret_cast<uint4*>(xs)[i] = ld_nc_u4(a.x + (size_t)i * 8);
+  // token rows (as fp32) and expert bias into shared memory (one coalesced pass)
+  float* xs = reinterpret_cast<float*>(scratch + route_scratch_bytes(T, E));
+  float* bias_s = a.expert_bias != nullptr ? xs + (size_t)T * H : nullptr;
+  for (int i = threadIdx.x; i < T * H / 8; i += kConsumers) {
+    float f[8];
+    unpack8_bf16(ld_nc_u4(a.x + (size_t)i * 8), f);
+    reinterpret_cast<float4*>(xs)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(xs)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
   if (bias_s != nullptr)
     for (int e = threadIdx.x; e < E; e += kConsumers) bias_s[e] = __ldg(a.expert_bias + e);
   consumer_sync();
@@ -819,17 +872,23 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
   // A warp whose wait runs out must still reach the named barriers below (they
   // have no timeout): it flags the CTA, and the consumers leave together after
   // the grid barrier.
-  uint32_t base = 0;
+  uint32_t carried;  // a unit claimed past phase A, processed after the routing
   {
     const Seg sg = segment(a, g, 0, 0);
-    for (uint32_t u = first_unit(base, warp); u < base + sg.r.n; u += kConsumerWarps) {
+    for (;;) {
+      const uint32_t u = claim_unit(sm);
+      if (u >= (uint32_t)sg.r.n) {
+        carried = u;
+        break;
+      }
       const unsigned char* st;
       uint64_t* empty;
       if (!stage(u, &st, &empty)) {
         sm.abort = 1;
+        carried = 0xffffffffu;
         break;
       }
-      const int i = sg.r.lo + (int)(u - base);
+      const int i = sg.r.lo + (int)u;
       if (i < n_router) {
         const float v = router_unit(reinterpret_cast<const float*>(st), H, xs, T, empty);
         if (lane == 0) a.logits[i] = v;
@@ -842,7 +901,6 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
         if (lane == 16 && T > 1) a.h_shared[Is + j] = v;
       }
     }
-    base += sg.r.n;
   }
   if (!grid_barrier(a.hdr, 1, &sm.flag) || sm.abort != 0) return;
 
@@ -852,9 +910,17 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
   const int n_act = sm.n_act;
   const int tq = lane >> 4, rr = lane & 15;  // down blocks: lane t*16 + r holds (slot or token t, row r)
 
-  for (int si = 1; si < num_segments(n_act); ++si) {
-    const Seg sg = segment(a, g, n_act, si);
-    for (uint32_t u = first_unit(base, warp); u < base + sg.r.n; u += kConsumerWarps) {
+  const int nseg = num_segments(n_act);
+  int si = 0;        // segment of the last claimed unit
+  uint32_t base = 0;  // its first stream index
+  Seg sg = segment(a, g, n_act, 0);
+  for (uint32_t u = carried;; u = claim_unit(sm)) {
+    while (si < nseg && u >= base + (uint32_t)sg.r.n) {  // segments are visited in order
+      base += sg.r.n;
+      if (++si < nseg) sg = segment(a, g, n_act, si);
+    }
+    if (si >= nseg) break;
+    {
       const int i = sg.r.lo + (int)(u - base);
       const unsigned char* st;
       uint64_t* empty;
@@ -906,7 +972,6 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
       }
       if (q.np == kMaxPend) publish(a, q, target);
     }
-    base += sg.r.n;
   }
   publish(a, q, target);
 }
@@ -924,6 +989,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const De
     }
     mbar_init(&sm.route_ready, 1);
     sm.abort = 0;
+    sm.next_unit = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
