@@ -74,9 +74,9 @@ KERNEL_SOURCES = {
     "decode_fused": ["decode_fused.cu", "decode_fused.cuh", "route.cuh", "mbarrier.cuh", "common.cuh"],
 }
 MEASURED_TRAFFIC = {
-    ("expert_gate_up", "ling26_flash_t512"): (2886553984, "0e81a7fa77706bc4"),
-    ("expert_down", "ling26_flash_t512"): (1491579904, "0e81a7fa77706bc4"),
-    ("decode_fused", "ling30_flash_decode_t1"): (123433984, "20ccce4ad41dea1b"),
+    ("expert_gate_up", "ling26_flash_t512"): (2887062656, "9f13a7c16c1856c3"),
+    ("expert_down", "ling26_flash_t512"): (1491627008, "9f13a7c16c1856c3"),
+    ("decode_fused", "ling30_flash_decode_t1"): (123498240, "71a362315a9d03f1"),
 }
 
 
