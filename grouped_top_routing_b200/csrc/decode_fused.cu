@@ -62,6 +62,10 @@ constexpr int kMaxDownRows = 16;   // rows per down block: lane t*16 + r holds (
 constexpr int kMaxHidden = 8192;   // a stage (4H bytes) must leave room for kMinStages
 constexpr int kSmemBudget = 227 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
+// Every poll loop sleeps this long between polls, so a waiting warp (the
+// producer above all, which shares a scheduler with consumer warps) leaves
+// the issue slots to the warps doing the work.
+constexpr unsigned kBackoffNs = 32;
 
 // Stream geometry, the same on host and device.
 struct Geo {
@@ -136,6 +140,7 @@ __device__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, i
         ok = 0;
         break;
       }
+      __nanosleep(kBackoffNs);
     }
   }
   ok = __all_sync(0xffffffffu, ok);
@@ -153,6 +158,7 @@ __device__ bool warp_wait_tag(volatile uint32_t* tag, uint32_t v, WsHeader* hdr,
         ok = 0;
         break;
       }
+      __nanosleep(kBackoffNs);
     }
   }
   ok = __all_sync(0xffffffffu, ok);
@@ -169,6 +175,7 @@ __device__ bool thread_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr,
       if (hdr != nullptr) record_error(hdr, MOE_ERR_TIMEOUT, site);
       return false;
     }
+    __nanosleep(kBackoffNs);
   }
   return true;
 }
@@ -185,7 +192,7 @@ __device__ bool warp_wait_count(const int32_t* ctr, int target, WsHeader* hdr, i
         ok = 0;
         break;
       }
-      __nanosleep(32);
+      __nanosleep(kBackoffNs);
     }
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -216,6 +223,7 @@ __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
           ok = 0;
           break;
         }
+        __nanosleep(kBackoffNs);
       }
     }
     __threadfence();
