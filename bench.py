@@ -71,7 +71,8 @@ def peaks():
 KERNEL_SOURCES = {
     "expert_gate_up": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
     "expert_down": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
-    "decode_fused": ["decode_fused.cu", "decode_fused.cuh", "route.cuh", "mbarrier.cuh", "common.cuh"],
+    "decode_fused": ["decode_fused.cu", "decode_tc.cu", "decode_fused.cuh", "fused_common.cuh", "route_block.cuh",
+                     "route.cuh", "mbarrier.cuh", "common.cuh"],
 }
 MEASURED_TRAFFIC = {
     ("expert_gate_up", "ling26_flash_t512"): (2887062656, "9f13a7c16c1856c3"),
@@ -91,10 +92,10 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str):
+def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decode_kernel: str = "auto"):
     """Bytes per launch from the capture, or None when it no longer applies."""
     entry = MEASURED_TRAFFIC.get((kernel, workload))
-    if entry is None or overrides or ffn_path != "auto":
+    if entry is None or overrides or ffn_path != "auto" or decode_kernel != "auto":
         return None
     return entry[0] if kernel_source_hash(kernel) == entry[1] else None
 
@@ -290,6 +291,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     M.set_ffn_path(args.ffn_path)
+    M.set_decode_kernel(args.decode_kernel)
     wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
@@ -433,7 +435,7 @@ def run_ours(args):
     else:
         kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
         kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
-    traffic = None if q8 is not None else measured_traffic(args.kernel, args.workload, args.set, args.ffn_path)
+    traffic = None if q8 is not None else measured_traffic(args.kernel, args.workload, args.set, args.ffn_path, args.decode_kernel)
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if kflops / kbytes > ridge:
@@ -468,7 +470,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "overrides": args.set, "ffn_path": args.ffn_path, "tokens": T, "hidden_size": wl["hidden_size"],
+        "config": {"workload": args.workload, "overrides": args.set, "ffn_path": args.ffn_path,
+                   "decode_kernel": args.decode_kernel, "tokens": T, "hidden_size": wl["hidden_size"],
                    "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
@@ -612,6 +615,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "streaming", "tensor_cores"],
                     help="expert-FFN kernels (default: the library's automatic choice)")
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"],
+                    help="fused decode kernel for 1-2 tokens (default: the library's choice, the CUDA-core kernel)")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (e.g. num_experts=64 for a small profiling case)")
     ap.add_argument("--q8", type=int, default=0, metavar="GROUP",

@@ -1,14 +1,13 @@
 // Fused decode: the whole MoE block for 1-2 tokens in one launch.
 //
-// At decode the block is bound by HBM bandwidth: it must stream the router
-// weight and the weights of the few selected experts ("only the selected
-// experts are read", page "Ling-3.0-flash-GGUF", section "Measured
-// performance") plus the shared MLP, ~120 MB for Ling-3.0-flash, against a few
-// microseconds of arithmetic. The kernel is therefore a weight-streaming
-// engine: one CTA per SM, a producer thread that keeps a ring of shared-memory
-// stages filled with untiled bulk copies (cp.async.bulk, mbarrier completion),
-// and eight consumer warps that each take whole stages and reduce them with
-// the token rows. A stage holds 4H bytes: one fp32 router row, or one bf16
+// At decode the block is bound by HBM bandwidth: it streams the router weight,
+// the shared MLP and, of the routed experts, only the few that were selected
+// (page "Ling-3.0-flash-GGUF", section "Measured performance"): ~120 MB for
+// Ling-3.0-flash against a few microseconds of arithmetic. The kernel is
+// therefore a weight-streaming engine: one CTA per SM, a producer thread that
+// keeps a ring of shared-memory stages filled with untiled bulk copies
+// (cp.async.bulk, mbarrier completion), and twelve consumer warps that each
+// take whole stages and reduce them with the token rows on the CUDA cores. A stage holds 4H bytes: one fp32 router row, or one bf16
 // gate row plus the matching up row, or a block of down-projection rows.
 //
 // Every phase's rows are split evenly into one contiguous range per CTA, and
@@ -33,39 +32,29 @@
 // MOE_ERR_TIMEOUT in the workspace and returns; the producer first waits
 // (bounded) for its copies in flight, so no copy lands after its CTA exits.
 //
-// Routing takes the same decisions as the per-token router kernel (route.cuh):
-// the same fp64 score evaluation rounded once to fp32, the same softmax sum
-// association, group scores from the multiset top-2 of each group, and the
-// top-k by (biased score descending, expert id ascending) found by ranking
-// unique 64-bit keys, first within each warp's slice of experts, then among
-// the slices' survivors, which is exact for a total order. Pages: mlxcel issue
-// #838 "add Ant Group Ling / Bailing MoE", section "Router: selection uses
-// biased scores, weights come from unbiased scores", and the model card
-// "Ling-2.6-flash-JANGTQ", paragraph "MoE routing".
+// The routing (route_block.cuh) takes the same decisions as the per-token
+// router kernel, bit for bit.
 #include "decode_fused.cuh"
 #include "mbarrier.cuh"
-#include "route.cuh"
+#include "fused_common.cuh"
+#include "route_block.cuh"
 
 namespace moe {
 
 namespace {
 
+using namespace fused;
+
 constexpr int kConsumerWarps = 12;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kFusedThreads = kConsumers + 32;  // + the producer warp
 constexpr int kFusedMaxT = 2;
-constexpr int kMaxSlots = 32;      // T * k: one warp lane per slot
-constexpr int kMaxChunk = 8;       // experts per lane in a warp's slice: 1024 / (6 warps * 32 lanes), rounded up
 constexpr int kMaxStages = 16;
 constexpr int kMinStages = 4;
 constexpr int kMaxDownRows = 16;   // rows per down block: lane t*16 + r holds (slot or token t, row r)
 constexpr int kMaxHidden = 8192;   // a stage (4H bytes) must leave room for kMinStages
 constexpr int kSmemBudget = 227 * 1024;
-constexpr uint64_t kWaitNs = 2000000000ull;
-// Every poll loop sleeps this long between polls, so a waiting warp (the
-// producer above all, which shares a scheduler with consumer warps) leaves
-// the issue slots to the warps doing the work.
-constexpr unsigned kBackoffNs = 32;
+constexpr int kMaxPend = 4;   // uncounted output rows per lane
 
 // Stream geometry, the same on host and device.
 struct Geo {
@@ -82,156 +71,23 @@ struct FusedSmem {
   // previous fill is still in flight, when its parity would read as the phase
   // the warp waits for; the tag shows which fill is pending.
   volatile uint32_t tag[kMaxStages];
-  uint64_t cand[kFusedMaxT][kConsumerWarps * kMaxSlots];  // per-slice survivors (64-bit keys)
-  uint32_t gkey[kFusedMaxT][32];                          // group score keys
-  uint32_t kept[kFusedMaxT];                              // kept-group masks
-  float red[kFusedMaxT][kConsumerWarps];
-  double sum[kFusedMaxT];
-  int32_t idx[kMaxSlots];  // slot -> expert
-  float w_raw[kMaxSlots];  // unbiased score of the slot's expert
-  float w[kMaxSlots];      // routing weight
-  int32_t act_e[kMaxSlots], act_a[kMaxSlots], act_b[kMaxSlots];  // distinct expert, first slot, second slot or -1
-  int n_act;
+  block_route::Smem<kConsumerWarps> rt;  // routing state and results
   int flag;
   volatile int abort;  // a consumer warp stopped before the grid barrier
   unsigned int next_unit;  // the next stream unit a consumer warp may claim
 };
 
-struct Range {
-  int lo, n;
-};
 
 // Dynamic shared memory after the ring: routing scratch ([T*E] fp32 scores,
 // [T*E] fp32 biased scores, [T*E] 64-bit keys), then the token rows (fp32,
 // converted once) and the expert bias (fp32).
-__host__ __device__ __forceinline__ size_t route_scratch_bytes(int T, int E) { return (size_t)T * E * 16; }
+__host__ __device__ __forceinline__ size_t route_scratch_bytes(int T, int E) { return block_route::scratch_bytes(T, E); }
 __host__ __device__ __forceinline__ size_t scratch_bytes(int T, int E, int H) {
   return route_scratch_bytes(T, E) + (size_t)T * H * 4 + (size_t)E * 4;
 }
 
-// Contiguous share b of G of `total` items.
-__host__ __device__ __forceinline__ Range split(int total, int b, int G) {
-  const int lo = (int)((int64_t)total * b / G), hi = (int)((int64_t)total * (b + 1) / G);
-  return {lo, hi - lo};
-}
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
-
-__device__ __forceinline__ int ld_acquire(const int32_t* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
-
-// Bounded wait for the phase of `bar` with the given parity, by every lane of
-// the warp; false (in every lane) after recording a timeout.
-__device__ bool warp_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
-  int ok = 1;
-  if (!mbar_try_wait(bar, parity)) {
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
-      if (globaltimer() - t0 > kWaitNs) {
-        ok = 0;
-        break;
-      }
-      __nanosleep(kBackoffNs);
-    }
-  }
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
-  return ok != 0;
-}
-
-// Bounded wait until the producer tagged slot `tag` with stream index v.
-__device__ bool warp_wait_tag(volatile uint32_t* tag, uint32_t v, WsHeader* hdr, int site) {
-  int ok = 1;
-  if (*tag != v) {
-    const uint64_t t0 = globaltimer();
-    while (*tag != v) {
-      if (globaltimer() - t0 > kWaitNs) {
-        ok = 0;
-        break;
-      }
-      __nanosleep(kBackoffNs);
-    }
-  }
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
-  return ok != 0;
-}
-
-// Single-thread bounded wait (producer side).
-__device__ bool thread_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitNs) {
-      if (hdr != nullptr) record_error(hdr, MOE_ERR_TIMEOUT, site);
-      return false;
-    }
-    __nanosleep(kBackoffNs);
-  }
-  return true;
-}
-
-// Lane 0 waits (bounded) until *ctr >= target; the whole warp then sees every
-// write released before the increments. False after recording a timeout.
-__device__ bool warp_wait_count(const int32_t* ctr, int target, WsHeader* hdr, int site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0 && ld_acquire(ctr) < target) {
-    const uint64_t t0 = globaltimer();
-    while (ld_acquire(ctr) < target) {
-      if (globaltimer() - t0 > kWaitNs) {
-        record_error(hdr, MOE_ERR_TIMEOUT, site);
-        ok = 0;
-        break;
-      }
-      __nanosleep(kBackoffNs);
-    }
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
-// Grid-wide barrier of the consumer threads of every CTA (sense by
-// generation). False if it timed out. Writes before it are visible to
-// ld.global.cg after it.
-__device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
-  consumer_sync();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    volatile uint32_t* gen = &hdr->bar_gen;
-    const uint32_t g = *gen;
-    __threadfence();
-    const uint32_t arrived = atomicAdd(&hdr->bar_count, 1u);
-    if (arrived == gridDim.x - 1) {
-      hdr->bar_count = 0u;
-      __threadfence();
-      atomicAdd(&hdr->bar_gen, 1u);
-    } else {
-      const uint64_t t0 = globaltimer();
-      while (*gen == g) {
-        if (globaltimer() - t0 > kWaitNs) {
-          record_error(hdr, MOE_ERR_TIMEOUT, 100 + site);
-          ok = 0;
-          break;
-        }
-        __nanosleep(kBackoffNs);
-      }
-    }
-    __threadfence();
-    *s_flag = ok;
-  }
-  consumer_sync();
-  return *s_flag != 0;
-}
 
 constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
 
@@ -395,291 +251,6 @@ __device__ __forceinline__ float down_unit(const uint16_t* w, int nrows, int K, 
   return reduce_scatter<2 * kMaxDownRows>(acc);
 }
 
-// Contributions to output rows a warp has stored but not yet counted (entry j
-// of lane l: the counter index tok*H + row of that lane's row in the warp's
-// j-th pending down block, or -1). They are counted whenever the warp is about
-// to block, when the list is full and at the warp's end: one fence covers
-// several blocks, and no warp waits while holding uncounted work.
-constexpr int kMaxPend = 4;
-struct Pending {
-  int pend[kMaxPend];
-  int np;  // warp-uniform number of pending down blocks
-};
-
-// y[tok, row] = bf16(sum of the k slot rows in slot order + the shared row).
-__device__ __forceinline__ void combine_row(const DecodeArgs& a, int idx) {
-  const int tok = idx / a.H, row = idx - tok * a.H;
-  float acc = 0.f;
-  for (int j = 0; j < a.k; ++j) acc += __ldcg(a.y_slots + (int64_t)(tok * a.k + j) * a.H + row);
-  if (a.ws_down != nullptr) acc += __ldcg(a.shared_out + (int64_t)tok * a.H + row);
-  a.y[idx] = f32_to_bf16(acc);
-}
-
-// Count the pending contributions: one fence, then the counter increments;
-// the lane that brings the last of an output row's k + 1 contributions
-// combines it.
-__device__ __forceinline__ void publish(const DecodeArgs& a, Pending& q, int target) {
-  __syncwarp();
-  __threadfence();
-  int32_t* rb_cnt = a.sync + kMaxSlots;
-  int last = 0;
-#pragma unroll
-  for (int j = 0; j < kMaxPend; ++j)
-    if (j < q.np && q.pend[j] >= 0 && atomicAdd(rb_cnt + q.pend[j], 1) == target - 1) last |= 1 << j;
-  if (last != 0) {
-    __threadfence();
-#pragma unroll
-    for (int j = 0; j < kMaxPend; ++j)
-      if ((last >> j) & 1) combine_row(a, q.pend[j]);
-  }
-  q.np = 0;
-}
-
-__device__ __forceinline__ void add_pending(Pending& q, int idx) {
-#pragma unroll
-  for (int j = 0; j < kMaxPend; ++j)
-    if (j == q.np) q.pend[j] = idx;
-  ++q.np;
-}
-
-// ---------------------------------------------------------------------------
-// Routing with the consumer warps
-// ---------------------------------------------------------------------------
-
-// Unique selection key: the order key of the biased score above the
-// complemented expert id, so that a larger key is a higher score or, on a tie,
-// a lower id. Real keys are > 0 (the order key of -inf is 0x007fffff).
-__device__ __forceinline__ uint64_t sel_key(float s, int e) {
-  return ((uint64_t)route_detail::order_key(s) << 32) | (uint64_t)(~(uint32_t)e);
-}
-
-// Level 1: this warp's slice [e0, e1) of token t's experts; lane l holds the
-// keys of experts e0 + l + 32 r. Each key's rank is the number of keys of the
-// slice above it; the ones ranked below k are stored at their rank.
-template <int R>
-__device__ __forceinline__ void rank_slice(const uint64_t* key, int e0, int e1, int k, uint64_t* out) {
-  const int lane = threadIdx.x & 31;
-  uint64_t mine[R];
-  int rank[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int e = e0 + lane + 32 * r;
-    mine[r] = e < e1 ? key[e] : 0ull;
-    rank[r] = 0;
-  }
-#pragma unroll 4
-  for (int j = e0; j < e1; ++j) {
-    const uint64_t kj = key[j];  // the same address in every lane: a broadcast
-#pragma unroll
-    for (int r = 0; r < R; ++r) rank[r] += kj > mine[r] ? 1 : 0;
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-    if (e0 + lane + 32 * r < e1 && rank[r] < k) out[rank[r]] = mine[r];
-}
-
-// Routes the T tokens with the consumer warps; results land in sm (slot
-// experts, weights, the distinct experts with their slots). Ends synchronised.
-// bias: the expert bias in shared memory, or null. Scratch: [T*E] fp32
-// scores, [T*E] fp32 biased scores, [T*E] 64-bit keys (first used for the
-// softmax exponentials).
-__device__ void route_block(const DecodeArgs& a, const float* logits, const float* bias, unsigned char* scratch,
-                            FusedSmem& sm) {
-  using namespace route_detail;
-  const int T = a.T, E = a.E, k = a.k;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* s_orig = reinterpret_cast<float*>(scratch);
-  float* s_sel = s_orig + T * E;
-  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_sel + T * E);
-  double* s_ex = reinterpret_cast<double*>(s_key);
-
-  // ---- scores: fp64 evaluation, one rounding to fp32; selection copy with the bias ----
-  if (a.score_fn != MOE_SCORE_SOFTMAX) {
-    for (int t = 0; t < T; ++t)
-      for (int e = threadIdx.x; e < E; e += kConsumers) {
-        const float L = __ldcg(logits + (int64_t)t * E + e);
-        const float o = __double2float_rn(1.0 / (1.0 + exp(-(double)L)));
-        s_orig[t * E + e] = o;
-        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
-      }
-  } else {
-    float m[kFusedMaxT] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int t = 0; t < kFusedMaxT; ++t)
-      if (t < T)
-        for (int e = threadIdx.x; e < E; e += kConsumers) {
-          const float L = __ldcg(logits + (int64_t)t * E + e);
-          s_orig[t * E + e] = L;
-          m[t] = fmaxf(m[t], L);
-        }
-#pragma unroll
-    for (int t = 0; t < kFusedMaxT; ++t) {
-      const float mt = warp_max_f32(m[t]);
-      if (lane == 0 && t < T) sm.red[t][warp] = mt;
-    }
-    consumer_sync();
-    for (int t = 0; t < T; ++t) {
-      float mt = sm.red[t][0];
-      for (int w = 1; w < kConsumerWarps; ++w) mt = fmaxf(mt, sm.red[t][w]);
-      const double md = (double)mt;
-      for (int e = threadIdx.x; e < E; e += kConsumers) s_ex[t * E + e] = exp((double)s_orig[t * E + e] - md);
-    }
-    consumer_sync();
-    if (warp < T) {
-      // the per-token router's association: lane l sums experts l*P .. l*P+P-1
-      int P = 1;
-      while (P * 32 < E) P <<= 1;
-      double sum = 0.0;
-      for (int i = 0; i < P; ++i) {
-        const int e = lane * P + i;
-        if (e < E) sum += s_ex[warp * E + e];
-      }
-      sum = warp_sum_f64(sum);
-      if (lane == 0) sm.sum[warp] = sum;
-    }
-    consumer_sync();
-    for (int t = 0; t < T; ++t)
-      for (int e = threadIdx.x; e < E; e += kConsumers) {
-        const float o = __double2float_rn(s_ex[t * E + e] / sm.sum[t]);
-        s_orig[t * E + e] = o;
-        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
-      }
-  }
-  consumer_sync();
-
-  // ---- groups: score = top1 + top2 of the group's biased scores; keep topk_group ----
-  const bool grouped = a.n_group > 1 && a.topk_group < a.n_group;
-  const int gsz = E / a.n_group;
-  if (grouped) {
-    for (int p = warp; p < T * a.n_group; p += kConsumerWarps) {
-      const int t = p / a.n_group, g = p - t * a.n_group;
-      const float* gv = s_sel + t * E + g * gsz;
-      float top1 = -INFINITY, top2 = -INFINITY;  // NaN never enters: it fails both comparisons
-      for (int i = lane; i < gsz; i += 32) {
-        const float v = gv[i];
-        if (v > top1) {
-          top2 = top1;
-          top1 = v;
-        } else if (v > top2) {
-          top2 = v;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {  // multiset top-2 of two lanes' pairs
-        const float b1 = __shfl_xor_sync(0xffffffffu, top1, o), b2 = __shfl_xor_sync(0xffffffffu, top2, o);
-        if (b1 > top1) {
-          top2 = fmaxf(top1, b2);
-          top1 = b1;
-        } else {
-          top2 = fmaxf(top2, b1);
-        }
-      }
-      if (lane == 0) sm.gkey[t][g] = order_key(gsz == 1 ? top1 : __fadd_rn(top1, top2));
-    }
-    consumer_sync();
-    if (warp < T) {
-      const uint32_t gk = lane < a.n_group ? sm.gkey[warp][lane] : 0u;
-      uint32_t kept = 0;
-      for (int r = 0; r < a.topk_group; ++r) {
-        const uint32_t key = ((kept >> lane) & 1u) ? 0u : gk;
-        const uint32_t mx = __reduce_max_sync(0xffffffffu, key);
-        const uint32_t win = __reduce_min_sync(0xffffffffu, key == mx ? (uint32_t)lane : 0xffffffffu);
-        kept |= 1u << win;
-      }
-      if (lane == 0) sm.kept[warp] = kept;
-    }
-    consumer_sync();
-  }
-
-  // ---- selection keys (experts of dropped groups select as -inf) ----
-  for (int t = 0; t < T; ++t) {
-    const uint32_t kept = grouped ? sm.kept[t] : 0xffffffffu;
-    for (int e = threadIdx.x; e < E; e += kConsumers) {
-      const bool live = !grouped || ((kept >> (e / gsz)) & 1u);
-      s_key[t * E + e] = sel_key(live ? s_sel[t * E + e] : -INFINITY, e);
-    }
-  }
-  consumer_sync();
-
-  // ---- level 1: the k best of each warp's slice of its token's experts ----
-  const int wpt = kConsumerWarps / T;
-  {
-    const int t = warp / wpt, wl = warp - t * wpt;
-    const int chunk = (E + wpt - 1) / wpt;
-    const int e0 = min(E, wl * chunk), e1 = min(E, e0 + chunk);
-    uint64_t* out = sm.cand[t] + wl * k;
-    const int per = (e1 - e0 + 31) / 32;
-    if (per <= 2) rank_slice<2>(s_key + t * E, e0, e1, k, out);
-    else if (per <= 4) rank_slice<4>(s_key + t * E, e0, e1, k, out);
-    else rank_slice<kMaxChunk>(s_key + t * E, e0, e1, k, out);
-    for (int j = min(k, e1 - e0) + lane; j < k; j += 32) out[j] = 0ull;  // fewer experts than k: padding
-  }
-  consumer_sync();
-
-  // ---- level 2: rank the survivors of the token's slices; rank j is slot j ----
-  {
-    const int per_tok = kConsumers / T;
-    const int t = threadIdx.x / per_tok, c = threadIdx.x - t * per_tok;
-    const int nc = wpt * k;
-    if (c < nc) {
-      const uint64_t mine = sm.cand[t][c];
-      if (mine != 0ull) {
-        int rank = 0;
-#pragma unroll 8
-        for (int j = 0; j < nc; ++j) rank += sm.cand[t][j] > mine ? 1 : 0;
-        if (rank < k) {
-          const int e = (int)(~(uint32_t)mine);
-          sm.idx[t * k + rank] = e;
-          sm.w_raw[t * k + rank] = s_orig[t * E + e];
-        }
-      }
-    }
-  }
-  consumer_sync();
-
-  // ---- weights: renormalise (k > 1) with the 1e-20 epsilon, then scale; fp32, slot order ----
-  if (warp < T) {
-    const int t = warp;
-    const bool do_norm = a.norm && k > 1;
-    float den = 0.f;
-    if (do_norm) {
-      if (lane == 0) {
-        den = sm.w_raw[t * k];
-        for (int j = 1; j < k; ++j) den = __fadd_rn(den, sm.w_raw[t * k + j]);
-        den = __fadd_rn(den, 1e-20f);
-      }
-      den = __shfl_sync(0xffffffffu, den, 0);
-    }
-    for (int j = lane; j < k; j += 32) {
-      float w = sm.w_raw[t * k + j];
-      if (do_norm) w = __fdiv_rn(w, den);
-      sm.w[t * k + j] = __fmul_rn(w, a.scale);
-    }
-  }
-  consumer_sync();
-
-  // ---- distinct experts, in order of first slot, with the slot(s) holding each ----
-  if (warp == 0) {
-    const int ns = T * k;
-    const int e = lane < ns ? sm.idx[lane] : (int)(0x40000000u | (uint32_t)lane);  // unique dummies
-    const uint32_t same = __match_any_sync(0xffffffffu, e);
-    const bool first = lane < ns && (__ffs(same) - 1) == lane;
-    const uint32_t firsts = __ballot_sync(0xffffffffu, first);
-    if (first) {
-      const int pos = __popc(firsts & ((1u << lane) - 1u));
-      const uint32_t other = same & ~(1u << lane);  // the other token's slot (ids are distinct per token)
-      sm.act_e[pos] = e;
-      sm.act_a[pos] = lane;
-      sm.act_b[pos] = other != 0u ? __ffs(other) - 1 : -1;
-    }
-    if (lane == 0) sm.n_act = __popc(firsts);
-    if (blockIdx.x == 0 && lane < ns) {
-      if (a.topk_idx_out != nullptr) a.topk_idx_out[lane] = e;
-      if (a.topk_w_out != nullptr) a.topk_w_out[lane] = sm.w[lane];
-    }
-  }
-  consumer_sync();
-}
 
 // ---------------------------------------------------------------------------
 // The stream of one CTA: a sequence of segments, each a contiguous share of
@@ -749,13 +320,13 @@ __device__ __forceinline__ UnitSrc unit_src(const DecodeArgs& a, const Geo& g, c
     u.p0 = a.ws_down + (int64_t)n0 * Is;
     u.n0 = 2u * rows * Is;
   } else if (sg.kind == kSegC) {
-    const uint16_t* gate = a.w_gate_up + ((int64_t)sm.act_e[sg.ai] * 2 * I + i) * H;
+    const uint16_t* gate = a.w_gate_up + ((int64_t)sm.rt.act_e[sg.ai] * 2 * I + i) * H;
     u.p0 = gate;
     u.p1 = gate + (int64_t)I * H;
     u.n0 = u.n1 = 2u * H;
   } else {
     const int n0 = i * g.rd, rows = min(g.rd, H - n0);
-    u.p0 = a.w_down + ((int64_t)sm.act_e[sg.ai] * H + n0) * I;
+    u.p0 = a.w_down + ((int64_t)sm.rt.act_e[sg.ai] * H + n0) * I;
     u.n0 = 2u * rows * I;
   }
   return u;
@@ -796,7 +367,7 @@ __device__ void producer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
       // end of S: wait for the routing, then continue with the selected experts
       ok = thread_wait_phase(&sm.route_ready, 0, a.hdr, 500);
       if (!ok) break;
-      n_act = sm.n_act;
+      n_act = sm.rt.n_act;
       nseg = num_segments(n_act);
       continue;
     }
@@ -860,7 +431,7 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
   const int n_router = a.logits_override == nullptr ? E : 0;
   const float* logits = a.logits_override != nullptr ? a.logits_override : a.logits;
   const int target = k + (a.ws_down != nullptr ? 1 : 0);
-  Pending q;
+  Pending<kMaxPend> q;
   q.np = 0;
   auto flush_if_pending = [&]() {
     if (q.np > 0) publish(a, q, target);
@@ -910,12 +481,12 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
       }
     }
   }
-  if (!grid_barrier(a.hdr, 1, &sm.flag) || sm.abort != 0) return;
+  if (!grid_barrier<kConsumers>(a.hdr, 1, &sm.flag) || sm.abort != 0) return;
 
   // ---- routing; then the producer may issue the selected experts' rows ----
-  route_block(a, logits, bias_s, scratch, sm);
+  block_route::route_block(a, logits, bias_s, scratch, sm.rt);
   if (threadIdx.x == 0) mbar_arrive(&sm.route_ready);
-  const int n_act = sm.n_act;
+  const int n_act = sm.rt.n_act;
   const int tq = lane >> 4, rr = lane & 15;  // down blocks: lane t*16 + r holds (slot or token t, row r)
 
   const int nseg = num_segments(n_act);
@@ -945,7 +516,7 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
         }
         add_pending(q, idx);
       } else if (sg.kind == kSegC) {  // ---- gate/up pair of a selected expert ----
-        const int slA = sm.act_a[sg.ai], slB = sm.act_b[sg.ai];
+        const int slA = sm.rt.act_a[sg.ai], slB = sm.rt.act_b[sg.ai];
         if (!stage(u, &st, &empty)) return;
         const uint16_t* w = reinterpret_cast<const uint16_t*>(st);
         const float v = gate_up_unit(w, w + H, H, xs + (slA / k) * H, slB >= 0 ? xs + (slB / k) * H : nullptr, empty);
@@ -956,7 +527,7 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
           red_release_add(done + sg.ai, 1);
         }
       } else {  // ---- down block of a selected expert ----
-        const int ai = sg.ai, slA = sm.act_a[ai], slB = sm.act_b[ai];
+        const int ai = sg.ai, slA = sm.rt.act_a[ai], slB = sm.rt.act_b[ai];
         const int n0 = i * g.rd, rows = min(g.rd, H - n0);
         const int need = slB >= 0 ? 2 * I : I;
         int complete = lane == 0 ? ld_acquire(done + ai) >= need : 0;
@@ -973,7 +544,7 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
         const int sl = tq == 0 ? slA : slB;
         int idx = -1;
         if (rr < rows && sl >= 0) {
-          a.y_slots[(int64_t)sl * H + n0 + rr] = sm.w[sl] * v;
+          a.y_slots[(int64_t)sl * H + n0 + rr] = sm.rt.w[sl] * v;
           idx = (sl / k) * H + n0 + rr;
         }
         add_pending(q, idx);
@@ -1027,7 +598,7 @@ Geo make_geo(int T, int E, int H, int I, int Is) {
 
 }  // namespace
 
-size_t decode_fused_sync_ints(int H) { return (size_t)kMaxSlots + (size_t)kFusedMaxT * H; }
+size_t decode_fused_sync_ints(int H) { return (size_t)kMaxSlots + (size_t)kFusedMaxT * H + 1; }
 
 bool decode_fused_supported(int64_t T, int k, int E, int H, int I, int Is) {
   // at most two tokens and one warp lane per slot; a stage must hold a router row

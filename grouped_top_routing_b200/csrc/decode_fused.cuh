@@ -1,4 +1,5 @@
-// Arguments and host entry points of the fused decode kernel (decode_fused.cu).
+// Arguments and host entry points of the fused decode kernels (decode_fused.cu,
+// decode_tc.cu).
 #pragma once
 
 #include "common.cuh"
@@ -28,11 +29,18 @@ struct DecodeArgs {
   WsHeader* hdr;
 };
 
-// Completion counters the kernel needs in the workspace (zeroed by the kernel).
+// Completion counters the kernels need in the workspace (zeroed by the kernels):
+// kMaxSlots per-expert counters, 2H per-row counters, one shared-MLP counter.
 size_t decode_fused_sync_ints(int H);
 // Whether the fused kernel handles this batch and shape (1-2 tokens, at most 32
 // slots, hidden size up to 8192, expert widths up to twice the hidden size).
 bool decode_fused_supported(int64_t T, int k, int E, int H, int I, int Is);
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s);
+
+// The tensor-core variant (decode_tc.cu): hidden size a multiple of 512 up to
+// 4096, expert and shared widths multiples of 16 up to 512. It uses the same
+// workspace (h and h_shared hold bf16 there) and the same sync counters.
+bool decode_tc_supported(int64_t T, int k, int E, int H, int I, int Is);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace moe

@@ -1,0 +1,200 @@
+// Helpers shared by the fused decode kernels (decode_fused.cu on the CUDA
+// cores, decode_tc.cu on the tensor cores): bounded waits, the grid barrier,
+// even splits of a phase over the CTAs, and the counting of output rows.
+// Every wait is bounded (globaltimer, ~2 s): one that runs out records
+// MOE_ERR_TIMEOUT in the workspace and returns false.
+#pragma once
+
+#include "decode_fused.cuh"
+#include "mbarrier.cuh"
+
+namespace moe {
+namespace fused {
+
+constexpr int kMaxSlots = 32;  // T * k; also the number of expert counters at the start of DecodeArgs::sync
+constexpr uint64_t kWaitNs = 2000000000ull;
+// Every poll loop sleeps this long between polls, so a waiting warp (a
+// producer above all, which shares a scheduler with consumer warps) leaves
+// the issue slots to the warps doing the work.
+constexpr unsigned kBackoffNs = 32;
+
+struct Range {
+  int lo, n;
+};
+
+// Contiguous share b of G of `total` items.
+__host__ __device__ __forceinline__ Range split(int total, int b, int G) {
+  const int lo = (int)((int64_t)total * b / G), hi = (int)((int64_t)total * (b + 1) / G);
+  return {lo, hi - lo};
+}
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+// Bounded wait for the phase of `bar` with the given parity, by every lane of
+// the warp; false (in every lane) after recording a timeout.
+__device__ inline bool warp_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+  int ok = 1;
+  if (!mbar_try_wait(bar, parity)) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+      if (globaltimer() - t0 > kWaitNs) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(kBackoffNs);
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
+  return ok != 0;
+}
+
+// Bounded wait until the producer tagged slot `tag` with stream index v.
+__device__ inline bool warp_wait_tag(volatile uint32_t* tag, uint32_t v, WsHeader* hdr, int site) {
+  int ok = 1;
+  if (*tag != v) {
+    const uint64_t t0 = globaltimer();
+    while (*tag != v) {
+      if (globaltimer() - t0 > kWaitNs) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(kBackoffNs);
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) record_error(hdr, MOE_ERR_TIMEOUT, site);
+  return ok != 0;
+}
+
+// Single-thread bounded wait (producer side).
+__device__ inline bool thread_wait_phase(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitNs) {
+      if (hdr != nullptr) record_error(hdr, MOE_ERR_TIMEOUT, site);
+      return false;
+    }
+    __nanosleep(kBackoffNs);
+  }
+  return true;
+}
+
+// Lane 0 waits (bounded) until *ctr >= target; the whole warp then sees every
+// write released before the increments. False after recording a timeout.
+__device__ inline bool warp_wait_count(const int32_t* ctr, int target, WsHeader* hdr, int site) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && ld_acquire(ctr) < target) {
+    const uint64_t t0 = globaltimer();
+    while (ld_acquire(ctr) < target) {
+      if (globaltimer() - t0 > kWaitNs) {
+        record_error(hdr, MOE_ERR_TIMEOUT, site);
+        ok = 0;
+        break;
+      }
+      __nanosleep(kBackoffNs);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// Grid-wide barrier of the NT consumer threads (threads 0 .. NT-1, named
+// barrier 1) of every CTA, sense by generation. False if it timed out. Writes
+// before it are visible to ld.global.cg after it.
+template <int NT>
+__device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
+  auto consumer_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); };
+  consumer_sync();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    volatile uint32_t* gen = &hdr->bar_gen;
+    const uint32_t g = *gen;
+    __threadfence();
+    const uint32_t arrived = atomicAdd(&hdr->bar_count, 1u);
+    if (arrived == gridDim.x - 1) {
+      hdr->bar_count = 0u;
+      __threadfence();
+      atomicAdd(&hdr->bar_gen, 1u);
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (*gen == g) {
+        if (globaltimer() - t0 > kWaitNs) {
+          record_error(hdr, MOE_ERR_TIMEOUT, 100 + site);
+          ok = 0;
+          break;
+        }
+        __nanosleep(kBackoffNs);
+      }
+    }
+    __threadfence();
+    *s_flag = ok;
+  }
+  consumer_sync();
+  return *s_flag != 0;
+}
+
+// Contributions to output rows a warp has stored but not yet counted (entry j
+// of lane l: the counter index tok*H + row of a row that lane stored, or -1).
+// Each output row y[t, n] counts its k + 1 contributions (k slot rows and the
+// shared row) in DecodeArgs::sync after the kMaxSlots expert counters; the
+// lane that brings the last one sums them in slot order and rounds once to
+// bf16. A warp counts its list in one go (one fence for many rows).
+template <int P>
+struct Pending {
+  int pend[P];
+  int np;  // warp-uniform number of entries
+};
+
+// y[tok, row] = bf16(sum of the k slot rows in slot order + the shared row).
+__device__ __forceinline__ void combine_row(const DecodeArgs& a, int idx) {
+  const int tok = idx / a.H, row = idx - tok * a.H;
+  float acc = 0.f;
+  for (int j = 0; j < a.k; ++j) acc += __ldcg(a.y_slots + (int64_t)(tok * a.k + j) * a.H + row);
+  if (a.ws_down != nullptr) acc += __ldcg(a.shared_out + (int64_t)tok * a.H + row);
+  a.y[idx] = f32_to_bf16(acc);
+}
+
+// Count the pending contributions: one fence, then the counter increments;
+// the lane that brings the last of an output row's k + 1 contributions
+// combines it.
+template <int P>
+__device__ __forceinline__ void publish(const DecodeArgs& a, Pending<P>& q, int target) {
+  __syncwarp();
+  __threadfence();
+  int32_t* rb_cnt = a.sync + kMaxSlots;
+  int last = 0;
+#pragma unroll
+  for (int j = 0; j < P; ++j)
+    if (j < q.np && q.pend[j] >= 0 && atomicAdd(rb_cnt + q.pend[j], 1) == target - 1) last |= 1 << j;
+  if (last != 0) {
+    __threadfence();
+#pragma unroll
+    for (int j = 0; j < P; ++j)
+      if ((last >> j) & 1) combine_row(a, q.pend[j]);
+  }
+  q.np = 0;
+}
+
+template <int P>
+__device__ __forceinline__ void add_pending(Pending<P>& q, int idx) {
+#pragma unroll
+  for (int j = 0; j < P; ++j)
+    if (j == q.np) q.pend[j] = idx;
+  ++q.np;
+}
+
+}  // namespace fused
+}  // namespace moe

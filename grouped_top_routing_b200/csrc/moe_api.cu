@@ -47,6 +47,7 @@ void* g_ev_start[MOE_KERNEL_COUNT] = {};
 void* g_ev_stop[MOE_KERNEL_COUNT] = {};
 int g_sm_count[64] = {};
 int g_ffn_path = 0;  // 0 auto, 1 streaming GEMV, 2 tensor cores
+int g_decode_kernel = 0;  // 0 auto (the CUDA-core fused decode), 1 CUDA cores, 2 tensor cores where the shapes fit
 
 moe_status fail(moe_status st, const char* fmt, ...) {
   va_list ap;
@@ -232,7 +233,9 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 4);
   L.y_slots = take((size_t)R * H * 4);
   L.shared_out = take((size_t)T * H * 4);
-  L.decode_sync = take(decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is) ? decode_fused_sync_ints((int)H) * 4 : 0);
+  const bool fused = decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is) ||
+                     decode_tc_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
+  L.decode_sync = take(fused ? decode_fused_sync_ints((int)H) * 4 : 0);
   L.total = off;
   return L;
 }
@@ -567,8 +570,10 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
-  if (g_ffn_path == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size, c.moe_intermediate_size,
-                                                    shared_width(c))) {
+  const bool tc_ok = g_decode_kernel == 2 && decode_tc_supported(T, c.num_experts_per_tok, c.num_experts,
+                                                                  c.hidden_size, c.moe_intermediate_size, shared_width(c));
+  if (g_ffn_path == 0 && (tc_ok || decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size,
+                                                         c.moe_intermediate_size, shared_width(c)))) {
     DecodeArgs d{};
     d.x = x;
     d.T = (int)T;
@@ -599,7 +604,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
     d.sync = at<int32_t>(ws, L.decode_sync);
     d.y = y;
     d.hdr = hdr;
-    cudaError_t e = launch_decode_fused(d, s);
+    cudaError_t e = tc_ok ? launch_decode_tc(d, s) : launch_decode_fused(d, s);
     if (e != cudaSuccess) return cuda_fail(e, "fused decode");
     return MOE_OK;
   }
@@ -659,6 +664,13 @@ uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relax
 moe_status moe_set_ffn_path(int32_t path) {
   if (path < 0 || path > 2) return fail(MOE_ERR_INVALID_ARG, "path = %d is not 0 (auto), 1 (streaming) or 2 (tensor cores)", path);
   g_ffn_path = path;
+  return MOE_OK;
+}
+
+moe_status moe_set_decode_kernel(int32_t which) {
+  if (which < 0 || which > 2)
+    return fail(MOE_ERR_INVALID_ARG, "which = %d is not 0 (auto), 1 (CUDA cores) or 2 (tensor cores)", which);
+  g_decode_kernel = which;
   return MOE_OK;
 }
 

@@ -1,0 +1,285 @@
+// Routing of 1-2 tokens by a whole thread block, for the fused decode kernels.
+//
+// Takes the same decisions as the per-token router kernel (route.cuh): the
+// same fp64 score evaluation rounded once to fp32, the same softmax sum
+// association, group scores from the multiset top-2 of each group, and the
+// top-k by (biased score descending, expert id ascending) found by ranking
+// unique 64-bit keys, first within each warp's slice of experts, then among
+// the slices' survivors, which is exact for a total order. Pages: mlxcel issue
+// #838 "add Ant Group Ling / Bailing MoE", section "Router: selection uses
+// biased scores, weights come from unbiased scores", and the model card
+// "Ling-2.6-flash-JANGTQ", paragraph "MoE routing".
+#pragma once
+
+#include "decode_fused.cuh"
+#include "route.cuh"
+
+namespace moe {
+namespace block_route {
+
+constexpr int kMaxT = 2;      // tokens
+constexpr int kMaxSlots = 32;  // T * k: one warp lane per slot
+
+// Shared-memory state of the routing of a block of W warps (the routing runs
+// on the W warps that share named barrier 1); the results are idx .. n_act.
+template <int W>
+struct Smem {
+  uint64_t cand[kMaxT][W * kMaxSlots];  // per-slice survivors (64-bit keys)
+  uint32_t gkey[kMaxT][32];             // group score keys
+  uint32_t kept[kMaxT];                 // kept-group masks
+  float red[kMaxT][W];
+  double sum[kMaxT];
+  int32_t idx[kMaxSlots];  // slot -> expert
+  float w_raw[kMaxSlots];  // unbiased score of the slot's expert
+  float w[kMaxSlots];      // routing weight
+  int32_t act_e[kMaxSlots], act_a[kMaxSlots], act_b[kMaxSlots];  // distinct expert, first slot, second slot or -1
+  int n_act;
+};
+
+// Dynamic shared memory the routing needs: [T*E] fp32 scores, [T*E] fp32
+// biased scores, [T*E] 64-bit keys.
+__host__ __device__ __forceinline__ size_t scratch_bytes(int T, int E) { return (size_t)T * E * 16; }
+
+// Unique selection key: the order key of the biased score above the
+// complemented expert id, so that a larger key is a higher score or, on a tie,
+// a lower id. Real keys are > 0 (the order key of -inf is 0x007fffff).
+__device__ __forceinline__ uint64_t sel_key(float s, int e) {
+  return ((uint64_t)route_detail::order_key(s) << 32) | (uint64_t)(~(uint32_t)e);
+}
+
+// Level 1: this warp's slice [e0, e1) of token t's experts; lane l holds the
+// keys of experts e0 + l + 32 r. Each key's rank is the number of keys of the
+// slice above it; the ones ranked below k are stored at their rank.
+template <int R>
+__device__ __forceinline__ void rank_slice(const uint64_t* key, int e0, int e1, int k, uint64_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint64_t mine[R];
+  int rank[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = e0 + lane + 32 * r;
+    mine[r] = e < e1 ? key[e] : 0ull;
+    rank[r] = 0;
+  }
+#pragma unroll 4
+  for (int j = e0; j < e1; ++j) {
+    const uint64_t kj = key[j];  // the same address in every lane: a broadcast
+#pragma unroll
+    for (int r = 0; r < R; ++r) rank[r] += kj > mine[r] ? 1 : 0;
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (e0 + lane + 32 * r < e1 && rank[r] < k) out[rank[r]] = mine[r];
+}
+
+// Routes the T tokens with the consumer warps; results land in sm (slot
+// experts, weights, the distinct experts with their slots). Ends synchronised.
+// bias: the expert bias in shared memory, or null. Scratch: [T*E] fp32
+// scores, [T*E] fp32 biased scores, [T*E] 64-bit keys (first used for the
+// softmax exponentials).
+template <int W>
+__device__ void route_block(const DecodeArgs& a, const float* logits, const float* bias, unsigned char* scratch,
+                            Smem<W>& sm) {
+  // up to 1024 experts: with at least four warps per token a warp's slice is
+  // at most 8 experts per lane (rank_slice<8>)
+  static_assert(W >= 8 && W % 2 == 0, "route_block needs an even number of at least 8 warps");
+  constexpr int kConsumerWarps = W, kConsumers = W * 32;
+  auto consumer_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); };
+  using namespace route_detail;
+  const int T = a.T, E = a.E, k = a.k;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* s_orig = reinterpret_cast<float*>(scratch);
+  float* s_sel = s_orig + T * E;
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(s_sel + T * E);
+  double* s_ex = reinterpret_cast<double*>(s_key);
+
+  // ---- scores: fp64 evaluation, one rounding to fp32; selection copy with the bias ----
+  if (a.score_fn != MOE_SCORE_SOFTMAX) {
+    for (int t = 0; t < T; ++t)
+      for (int e = threadIdx.x; e < E; e += kConsumers) {
+        const float L = __ldcg(logits + (int64_t)t * E + e);
+        const float o = __double2float_rn(1.0 / (1.0 + exp(-(double)L)));
+        s_orig[t * E + e] = o;
+        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
+      }
+  } else {
+    float m[kMaxT] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int t = 0; t < kMaxT; ++t)
+      if (t < T)
+        for (int e = threadIdx.x; e < E; e += kConsumers) {
+          const float L = __ldcg(logits + (int64_t)t * E + e);
+          s_orig[t * E + e] = L;
+          m[t] = fmaxf(m[t], L);
+        }
+#pragma unroll
+    for (int t = 0; t < kMaxT; ++t) {
+      const float mt = warp_max_f32(m[t]);
+      if (lane == 0 && t < T) sm.red[t][warp] = mt;
+    }
+    consumer_sync();
+    for (int t = 0; t < T; ++t) {
+      float mt = sm.red[t][0];
+      for (int w = 1; w < kConsumerWarps; ++w) mt = fmaxf(mt, sm.red[t][w]);
+      const double md = (double)mt;
+      for (int e = threadIdx.x; e < E; e += kConsumers) s_ex[t * E + e] = exp((double)s_orig[t * E + e] - md);
+    }
+    consumer_sync();
+    if (warp < T) {
+      // the per-token router's association: lane l sums experts l*P .. l*P+P-1
+      int P = 1;
+      while (P * 32 < E) P <<= 1;
+      double sum = 0.0;
+      for (int i = 0; i < P; ++i) {
+        const int e = lane * P + i;
+        if (e < E) sum += s_ex[warp * E + e];
+      }
+      sum = warp_sum_f64(sum);
+      if (lane == 0) sm.sum[warp] = sum;
+    }
+    consumer_sync();
+    for (int t = 0; t < T; ++t)
+      for (int e = threadIdx.x; e < E; e += kConsumers) {
+        const float o = __double2float_rn(s_ex[t * E + e] / sm.sum[t]);
+        s_orig[t * E + e] = o;
+        s_sel[t * E + e] = bias != nullptr ? __fadd_rn(o, bias[e]) : o;
+      }
+  }
+  consumer_sync();
+
+  // ---- groups: score = top1 + top2 of the group's biased scores; keep topk_group ----
+  const bool grouped = a.n_group > 1 && a.topk_group < a.n_group;
+  const int gsz = E / a.n_group;
+  if (grouped) {
+    for (int p = warp; p < T * a.n_group; p += kConsumerWarps) {
+      const int t = p / a.n_group, g = p - t * a.n_group;
+      const float* gv = s_sel + t * E + g * gsz;
+      float top1 = -INFINITY, top2 = -INFINITY;  // NaN never enters: it fails both comparisons
+      for (int i = lane; i < gsz; i += 32) {
+        const float v = gv[i];
+        if (v > top1) {
+          top2 = top1;
+          top1 = v;
+        } else if (v > top2) {
+          top2 = v;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {  // multiset top-2 of two lanes' pairs
+        const float b1 = __shfl_xor_sync(0xffffffffu, top1, o), b2 = __shfl_xor_sync(0xffffffffu, top2, o);
+        if (b1 > top1) {
+          top2 = fmaxf(top1, b2);
+          top1 = b1;
+        } else {
+          top2 = fmaxf(top2, b1);
+        }
+      }
+      if (lane == 0) sm.gkey[t][g] = order_key(gsz == 1 ? top1 : __fadd_rn(top1, top2));
+    }
+    consumer_sync();
+    if (warp < T) {
+      const uint32_t gk = lane < a.n_group ? sm.gkey[warp][lane] : 0u;
+      uint32_t kept = 0;
+      for (int r = 0; r < a.topk_group; ++r) {
+        const uint32_t key = ((kept >> lane) & 1u) ? 0u : gk;
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, key);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, key == mx ? (uint32_t)lane : 0xffffffffu);
+        kept |= 1u << win;
+      }
+      if (lane == 0) sm.kept[warp] = kept;
+    }
+    consumer_sync();
+  }
+
+  // ---- selection keys (experts of dropped groups select as -inf) ----
+  for (int t = 0; t < T; ++t) {
+    const uint32_t kept = grouped ? sm.kept[t] : 0xffffffffu;
+    for (int e = threadIdx.x; e < E; e += kConsumers) {
+      const bool live = !grouped || ((kept >> (e / gsz)) & 1u);
+      s_key[t * E + e] = sel_key(live ? s_sel[t * E + e] : -INFINITY, e);
+    }
+  }
+  consumer_sync();
+
+  // ---- level 1: the k best of each warp's slice of its token's experts ----
+  const int wpt = kConsumerWarps / T;
+  {
+    const int t = warp / wpt, wl = warp - t * wpt;
+    const int chunk = (E + wpt - 1) / wpt;
+    const int e0 = min(E, wl * chunk), e1 = min(E, e0 + chunk);
+    uint64_t* out = sm.cand[t] + wl * k;
+    const int per = (e1 - e0 + 31) / 32;
+    if (per <= 2) rank_slice<2>(s_key + t * E, e0, e1, k, out);
+    else if (per <= 4) rank_slice<4>(s_key + t * E, e0, e1, k, out);
+    else rank_slice<8>(s_key + t * E, e0, e1, k, out);
+    for (int j = min(k, e1 - e0) + lane; j < k; j += 32) out[j] = 0ull;  // fewer experts than k: padding
+  }
+  consumer_sync();
+
+  // ---- level 2: rank the survivors of the token's slices; rank j is slot j ----
+  {
+    const int per_tok = kConsumers / T;
+    const int t = threadIdx.x / per_tok, c = threadIdx.x - t * per_tok;
+    const int nc = wpt * k;
+    if (c < nc) {
+      const uint64_t mine = sm.cand[t][c];
+      if (mine != 0ull) {
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < nc; ++j) rank += sm.cand[t][j] > mine ? 1 : 0;
+        if (rank < k) {
+          const int e = (int)(~(uint32_t)mine);
+          sm.idx[t * k + rank] = e;
+          sm.w_raw[t * k + rank] = s_orig[t * E + e];
+        }
+      }
+    }
+  }
+  consumer_sync();
+
+  // ---- weights: renormalise (k > 1) with the 1e-20 epsilon, then scale; fp32, slot order ----
+  if (warp < T) {
+    const int t = warp;
+    const bool do_norm = a.norm && k > 1;
+    float den = 0.f;
+    if (do_norm) {
+      if (lane == 0) {
+        den = sm.w_raw[t * k];
+        for (int j = 1; j < k; ++j) den = __fadd_rn(den, sm.w_raw[t * k + j]);
+        den = __fadd_rn(den, 1e-20f);
+      }
+      den = __shfl_sync(0xffffffffu, den, 0);
+    }
+    for (int j = lane; j < k; j += 32) {
+      float w = sm.w_raw[t * k + j];
+      if (do_norm) w = __fdiv_rn(w, den);
+      sm.w[t * k + j] = __fmul_rn(w, a.scale);
+    }
+  }
+  consumer_sync();
+
+  // ---- distinct experts, in order of first slot, with the slot(s) holding each ----
+  if (warp == 0) {
+    const int ns = T * k;
+    const int e = lane < ns ? sm.idx[lane] : (int)(0x40000000u | (uint32_t)lane);  // unique dummies
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    const bool first = lane < ns && (__ffs(same) - 1) == lane;
+    const uint32_t firsts = __ballot_sync(0xffffffffu, first);
+    if (first) {
+      const int pos = __popc(firsts & ((1u << lane) - 1u));
+      const uint32_t other = same & ~(1u << lane);  // the other token's slot (ids are distinct per token)
+      sm.act_e[pos] = e;
+      sm.act_a[pos] = lane;
+      sm.act_b[pos] = other != 0u ? __ffs(other) - 1 : -1;
+    }
+    if (lane == 0) sm.n_act = __popc(firsts);
+    if (blockIdx.x == 0 && lane < ns) {
+      if (a.topk_idx_out != nullptr) a.topk_idx_out[lane] = e;
+      if (a.topk_w_out != nullptr) a.topk_w_out[lane] = sm.w[lane];
+    }
+  }
+  consumer_sync();
+}
+
+}  // namespace block_route
+}  // namespace moe

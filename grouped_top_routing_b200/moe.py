@@ -26,7 +26,7 @@ FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch at
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
-           "moe_set_ffn_path", "moe_launch_count", "moe_last_error", "moe_permute_static",
+           "moe_set_ffn_path", "moe_set_decode_kernel", "moe_launch_count", "moe_last_error", "moe_permute_static",
            "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 
@@ -104,6 +104,7 @@ def _load():
         "moe_check_device": (st, [vp, sz, vp]),
         "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
         "moe_set_ffn_path": (st, [ctypes.c_int32]),
+        "moe_set_decode_kernel": (st, [ctypes.c_int32]),
         "moe_permute_static": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp]),
         "moe_dense_mlp_workspace_size": (sz, [ctypes.c_int32, ctypes.c_int32, i64]),
         "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp]),
@@ -237,11 +238,43 @@ def moe_combine(cfg, y_slots, shared_out, T: int, y=None, stream=None):
     return y
 
 
+def shared_width(c: MoeConfig) -> int:
+    """Width of the shared MLP as the library derives it from the config."""
+    if c.num_shared_experts <= 0:
+        return 0
+    per = c.moe_shared_expert_intermediate_size or c.moe_intermediate_size
+    return per * c.num_shared_experts
+
+
+def _require(t, name: str, numel: int, dtype):
+    """The C ABI sees raw pointers only: a tensor smaller than the config says
+    would be read past its end on the device, so check sizes here."""
+    if t is None:
+        return
+    if t.numel() != numel or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected {numel} contiguous {dtype} elements for this config, got "
+                         f"{tuple(t.shape)} {t.dtype}{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _check_block_tensors(c: MoeConfig, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down,
+                         ws_gate_up, ws_down):
+    E, H, I, Is = c.num_experts, c.hidden_size, c.moe_intermediate_size, shared_width(c)
+    _require(x, "x", T * H, torch.bfloat16)
+    _require(router_w, "router_w", E * H, torch.float32)
+    _require(expert_bias, "expert_bias", E, torch.float32)
+    _require(logits_override, "logits_override", T * E, torch.float32)
+    _require(w_gate_up, "w_gate_up", E * 2 * I * H, torch.bfloat16)
+    _require(w_down, "w_down", E * H * I, torch.bfloat16)
+    _require(ws_gate_up, "ws_gate_up", 2 * Is * H, torch.bfloat16)
+    _require(ws_down, "ws_down", H * Is, torch.bfloat16)
+
+
 def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws_down, ws: Workspace,
                 logits_override=None, y=None, return_routing=False, stream=None):
     c = _as_cfg(cfg)
     T = x.shape[0]
     k = c.num_experts_per_tok
+    _check_block_tensors(c, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down, ws_gate_up, ws_down)
     if y is None:
         y = torch.empty_like(x)
     idx = w = None
@@ -259,6 +292,15 @@ def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws
 def set_ffn_path(path: str = "auto"):
     """Expert-FFN kernels for later calls: "auto", "streaming" or "tensor_cores"."""
     _check(lib.moe_set_ffn_path(FFN_PATHS[path]))
+
+
+DECODE_KERNELS = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
+
+
+def set_decode_kernel(which: str = "auto"):
+    """Fused decode kernel for later calls: "auto" (the CUDA-core kernel),
+    "cuda_cores", or "tensor_cores" (where its shapes fit)."""
+    _check(lib.moe_set_decode_kernel(DECODE_KERNELS[which]))
 
 
 def set_kernel_timer(kernel: str, ev_start=None, ev_stop=None):

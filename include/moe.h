@@ -197,9 +197,15 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
  * 32 slots (T*k), E <= 1024 and H <= 8192, the block runs as one cooperative
  * launch (MOE_KERNEL_DECODE_FUSED): a weight-streaming kernel, one CTA per SM,
  * with one bounded grid barrier and bounded per-expert and per-row counters.
+ * The kernel multiplies on the CUDA cores (fp32 sums throughout). A variant
+ * on the tensor cores (mma.sync, bf16 in, fp32 sums, h kept as two bf16
+ * planes as on the tensor-core expert path) takes H a multiple of 512 up to
+ * 4096 and expert and shared widths multiples of 64 up to 512 ([GGUF]
+ * shapes); moe_set_decode_kernel selects it.
  * Its routing (indices and weights) is bit-identical to moe_route on the same
  * logits; its logits and output equal those of the separate kernels up to the
- * fp32 summation order of the dot products.
+ * fp32 summation order of the dot products (and the 16-bit h planes of the
+ * tensor-core variant).
  *   logits_override [T,E] fp32 or NULL: when given, replaces the router
  *   projection (router_w may then be NULL).
  *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
@@ -270,6 +276,13 @@ moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop);
  * 1 = always the streaming GEMV, 2 = always the tensor-core grouped GEMM.
  * Both compute the same block. */
 moe_status moe_set_ffn_path(int32_t path);
+
+/* Selects the fused decode kernel of moe_forward for every later call in this
+ * process: 0 = automatic (the CUDA-core kernel, measured the faster of the two
+ * at Ling-3.0-flash decode shapes), 1 = the CUDA-core kernel, 2 = the
+ * tensor-core kernel where its shapes fit (else the CUDA-core one). Both
+ * compute the same block. Any other value: MOE_ERR_INVALID_ARG. */
+moe_status moe_set_decode_kernel(int32_t which);
 
 /* Number of this library's kernel launches since load (host-side counter). */
 uint64_t moe_launch_count(void);

@@ -175,6 +175,15 @@ def test_kernel_timer_arguments(M):
     assert M.lib.moe_set_kernel_timer(0, None, None) == 0
 
 
+def test_path_selectors_reject_unknown_values(M):
+    assert M.lib.moe_set_ffn_path(3) == 1 and M.lib.moe_set_ffn_path(-1) == 1
+    assert M.lib.moe_set_decode_kernel(3) == 1 and "not 0 (auto), 1 (CUDA cores) or 2" in M.last_error()
+    assert M.lib.moe_set_decode_kernel(-1) == 1
+    for which in (1, 2, 0):
+        assert M.lib.moe_set_decode_kernel(which) == 0
+    assert M.lib.moe_set_ffn_path(0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # The binding has no fallback: a missing library is an import error.
     import importlib.util

@@ -6,6 +6,7 @@ fp64 oracle, near-tie tokens reported separately. Inputs are seeded and
 synthetic (grouped_top_routing_b200.inputs); the oracle never sees a value the
 CUDA path produced except where a test compares them.
 """
+import contextlib
 import math
 
 import numpy as np
@@ -338,23 +339,44 @@ FUSED_CASES = [
 ]
 
 
-@pytest.mark.parametrize("name,over,T", FUSED_CASES, ids=[f"{n}-T{T}-{i}" for i, (n, _, T) in enumerate(FUSED_CASES)])
-def test_fused_decode(M, name, over, T):
+# The fused decode runs on the CUDA-core kernel by default; "tensor_cores"
+# selects the tensor-core variant, which takes the Ling-3.0-flash shapes
+# (H = 4096, I = Is = 512); the other shapes stay on the CUDA-core kernel.
+FUSED_KERNEL_CASES = [(c, "auto") for c in FUSED_CASES] + [(c, "tensor_cores") for c in FUSED_CASES
+                                                           if c[0].startswith("ling30")]
+
+
+@contextlib.contextmanager
+def decode_kernel(M, which):
+    M.set_decode_kernel(which)
+    try:
+        yield
+    finally:
+        M.set_decode_kernel("auto")
+
+
+@pytest.mark.parametrize("case,kernel", FUSED_KERNEL_CASES,
+                         ids=[f"{c[0]}-T{c[2]}-{i}-{kn}" for i, (c, kn) in enumerate(FUSED_KERNEL_CASES)])
+def test_fused_decode(M, case, kernel):
     # one launch for 1-2 tokens: routing bit-exact on given logits, output
     # against the oracle, and the same routing when it computes the logits
+    name, over, T = case
     wl, inp = _inputs(name)
     wl = dict(wl, **over, name=f"fused-{name}")
     sub = dict(inp, x=inp["x"][7:7 + T].contiguous(), tokens=T)
     L = G.random_logits(T, wl["num_experts"], S.logit_std(wl), seed=11).numpy()
-    n0 = M.launch_count()
-    _forward_and_compare(M, wl, sub, logits=L)
-    assert M.launch_count() - n0 == 1, "the fused decode is a single launch"
-    _forward_and_compare(M, wl, sub)
+    with decode_kernel(M, kernel):
+        n0 = M.launch_count()
+        _forward_and_compare(M, wl, sub, logits=L)
+        assert M.launch_count() - n0 == 1, "the fused decode is a single launch"
+        _forward_and_compare(M, wl, sub)
 
 
-@pytest.mark.parametrize("name,T", [("ling26_flash_t512", 2), ("ling30_flash_decode_t64", 1),
-                                    ("ling30_flash_decode_t64", 2)])
-def test_fused_decode_repeatable(M, name, T):
+@pytest.mark.parametrize("name,T,kernel", [("ling26_flash_t512", 2, "auto"), ("ling30_flash_decode_t64", 1, "auto"),
+                                           ("ling30_flash_decode_t64", 2, "auto"),
+                                           ("ling30_flash_decode_t64", 1, "tensor_cores"),
+                                           ("ling30_flash_decode_t64", 2, "tensor_cores")])
+def test_fused_decode_repeatable(M, name, T, kernel):
     # Every sum in the fused kernel has a fixed order, so repeated launches
     # must agree bit for bit. Its consumer warps, producer and counters run
     # unsynchronised across SMs; a missed wait shows up here as a changed bit
@@ -365,21 +387,24 @@ def test_fused_decode_repeatable(M, name, T):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=DEV)
     args = (wl, x, inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"],
             inp["ws_down"], ws)
-    first = M.moe_forward(*args).clone()
-    for i in range(40):
-        if i % 3 == 0:
-            flush.zero_()
-        y = M.moe_forward(*args)
-        assert torch.equal(y.view(torch.int16), first.view(torch.int16)), f"launch {i} differs"
+    with decode_kernel(M, kernel):
+        first = M.moe_forward(*args).clone()
+        for i in range(40):
+            if i % 3 == 0:
+                flush.zero_()
+            y = M.moe_forward(*args)
+            assert torch.equal(y.view(torch.int16), first.view(torch.int16)), f"launch {i} differs"
     ws.check()
 
 
-# The fused kernel routes with a whole thread block (per-warp top-k lists
+# The fused kernels route with a whole thread block (per-warp top-k lists
 # merged by one warp); the router kernel routes each token with one warp. Both
 # must take the same decisions bit for bit, ties included: logits on a 1/4
 # grid tie often, zipf biases have bitwise twins, E not a multiple of 32 leaves
 # padding lanes, and the cases reach the limits (32 slots, 1024 experts, 32
-# groups, every expert selected, k = 1).
+# groups, every expert selected, k = 1). They run on the CUDA-core kernel (12
+# routing warps) and, at hidden size 512, on the tensor-core one (8 routing
+# warps).
 FUSED_ROUTE_CASES = [
     # experts, k, n_group, topk_group, score, bias, tokens, shared MLP
     (64, 6, 1, 1, "softmax", "none", 1, True),
@@ -394,14 +419,17 @@ FUSED_ROUTE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("hidden,kernel", [(64, "auto"), (512, "tensor_cores")])
 @pytest.mark.parametrize("case", FUSED_ROUTE_CASES,
                          ids=[f"E{c[0]}-k{c[1]}-g{c[2]}_{c[3]}-{c[4]}-T{c[6]}" for c in FUSED_ROUTE_CASES])
-def test_fused_routing_matches_router_kernel(M, case):
+def test_fused_routing_matches_router_kernel(M, case, hidden, kernel):
     E, k, ng, tg, score, bias, T, shared = case
-    wl = G.tiny_workload(tokens=T, num_experts=E, num_experts_per_tok=k, n_group=ng, topk_group=tg,
-                         score_function=score, bias=bias, routed_scaling_factor=2.5,
-                         num_shared_experts=1 if shared else 0, shared_width=32 if shared else 0,
-                         name=f"fused-route-E{E}")
+    wl = G.tiny_workload(tokens=T, hidden_size=hidden, num_experts=E, num_experts_per_tok=k, n_group=ng,
+                         topk_group=tg, score_function=score, bias=bias, routed_scaling_factor=2.5,
+                         moe_intermediate_size=32 if hidden == 64 else 64,
+                         num_shared_experts=1 if shared else 0,
+                         shared_width=(32 if hidden == 64 else 64) if shared else 0,
+                         name=f"fused-route-E{E}-H{hidden}")
     inp = G.make_inputs(wl, seed=5, device=DEV)
     b = _np_bias(inp)
     rng = np.random.default_rng(1000 * E + 10 * k + T)
@@ -413,11 +441,12 @@ def test_fused_routing_matches_router_kernel(M, case):
             x = torch.stack([x[0], x[0]])
         Ld = torch.from_numpy(L).to(DEV)
         ws = M.Workspace(wl, T)
-        n0 = M.launch_count()
-        y, idx, w = M.moe_forward(wl, x, inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
-                                  inp["ws_gate_up"], inp["ws_down"], ws, logits_override=Ld, return_routing=True)
-        ws.check()
-        assert M.launch_count() - n0 == 1
+        with decode_kernel(M, kernel):
+            n0 = M.launch_count()
+            y, idx, w = M.moe_forward(wl, x, inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                                      inp["ws_gate_up"], inp["ws_down"], ws, logits_override=Ld, return_routing=True)
+            ws.check()
+            assert M.launch_count() - n0 == 1
         r_idx, r_w = M.moe_route(wl, Ld, inp["expert_bias"])
         assert torch.equal(idx, r_idx), (idx, r_idx)
         assert torch.equal(w.view(torch.int32), r_w.view(torch.int32))
