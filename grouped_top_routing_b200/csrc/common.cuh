@@ -21,9 +21,9 @@ struct WsHeader {
   int32_t error;        // first moe_status recorded on the device (0 = none)
   int32_t error_info;   // kernel-specific detail (offending index, wait site)
   int32_t num_active;   // number of experts with rows (written by permute)
-  uint32_t bar_count;   // grid barrier of the fused decode kernel: arrivals
-  uint32_t bar_gen;     //   and generation (both zero between launches)
-  int32_t pad[59];
+  int32_t pad0[3];
+  uint64_t bar_arrivals;  // grid barrier of the fused decode kernels: arrivals, only ever growing
+  int32_t pad[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

@@ -111,26 +111,33 @@ __device__ inline bool warp_wait_count(const int32_t* ctr, int target, WsHeader*
   return ok != 0;
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Grid-wide barrier of the NT consumer threads (threads 0 .. NT-1, named
-// barrier 1) of every CTA, sense by generation. False if it timed out. Writes
-// before it are visible to ld.global.cg after it.
+// barrier 1) of every CTA. The arrival counter only grows: a launch's G CTAs
+// take arrivals nG .. nG + G - 1 and each waits until the counter reaches
+// (n + 1) G, so nothing is reset between barriers or launches (after a timeout
+// the workspace must be initialised again). One release per CTA (fence and
+// add), one acquire load that sees the last arrival. False if it timed out.
+// Writes before it are visible to ld.global.cg after it.
 template <int NT>
 __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
   auto consumer_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); };
   consumer_sync();
   if (threadIdx.x == 0) {
     int ok = 1;
-    volatile uint32_t* gen = &hdr->bar_gen;
-    const uint32_t g = *gen;
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(&hdr->bar_arrivals);
+    const unsigned long long G = gridDim.x;
     __threadfence();
-    const uint32_t arrived = atomicAdd(&hdr->bar_count, 1u);
-    if (arrived == gridDim.x - 1) {
-      hdr->bar_count = 0u;
-      __threadfence();
-      atomicAdd(&hdr->bar_gen, 1u);
-    } else {
+    const unsigned long long arrival = atomicAdd(ctr, 1ull);
+    const unsigned long long target = (arrival / G + 1) * G;
+    if (arrival + 1 < target) {
       const uint64_t t0 = globaltimer();
-      while (*gen == g) {
+      while (ld_acquire_u64(ctr) < target) {
         if (globaltimer() - t0 > kWaitNs) {
           record_error(hdr, MOE_ERR_TIMEOUT, 100 + site);
           ok = 0;
@@ -138,8 +145,9 @@ __device__ bool grid_barrier(WsHeader* hdr, int site, int* s_flag) {
         }
         __nanosleep(kBackoffNs);
       }
+    } else {
+      (void)ld_acquire_u64(ctr);  // the last arrival: acquire the others' writes
     }
-    __threadfence();
     *s_flag = ok;
   }
   consumer_sync();
