@@ -77,7 +77,7 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     ("expert_gate_up", "ling26_flash_t512"): (2887062656, "9f13a7c16c1856c3"),
     ("expert_down", "ling26_flash_t512"): (1491627008, "9f13a7c16c1856c3"),
-    ("decode_fused", "ling30_flash_decode_t1"): (123498240, "71a362315a9d03f1"),
+    ("decode_fused", "ling30_flash_decode_t1"): (121980928, "2285db6e03f385e6"),
 }
 
 

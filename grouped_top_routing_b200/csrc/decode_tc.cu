@@ -2,9 +2,10 @@
 // launch, for hidden sizes that are a multiple of 512 (up to 4096) and expert
 // widths up to 512 (Ling-3.0-flash: H = 4096, I = Is = 512).
 //
-// Decode streams the router weight, the shared MLP and only the selected
-// experts (page "Ling-3.0-flash-GGUF", section "Measured performance"), so it
-// is bound by HBM bandwidth, and the arithmetic must cost little per byte.
+// Decode streams the router weight, the shared MLP and just the experts the
+// router chose (page "Ling-3.0-flash-GGUF", section "Measured performance"),
+// so it is bound by HBM bandwidth, and the arithmetic must cost little per
+// byte.
 // On the CUDA cores a bf16 weight costs about two instructions (unpack and
 // FMA); here the consumers multiply with mma.sync (m16n8k16, bf16 inputs, fp32
 // accumulation), one ldmatrix, one 8-byte shared load and one mma per 512

@@ -1,7 +1,8 @@
 // Decode expert FFN: weight-streaming GEMV over the selected experts only.
 //
 // The page "Ling-3.0-flash-GGUF" (section "Measured performance") bounds
-// decode by memory bandwidth: only the selected experts' weights are read.
+// decode by memory bandwidth, since a decode step touches just the weights of
+// the experts the router chose.
 // The expert is the SwiGLU MLP of mlxcel issue #838 ("Architecture notes";
 // "Shared experts are one wide MLP, not N separate experts"):
 //   h = silu(gate x) * (up x),  y = down h.

@@ -21,8 +21,8 @@
  *             instead of terminating, take gather bounds from real shapes).
  *   [LING26]  model card "Ling-2.6-flash-JANGTQ", "Architecture
  *             (bailing_hybrid)", paragraph "MoE routing".
- *   [GGUF]    page "Ling-3.0-flash-GGUF", "Measured performance": decode reads
- *             only the selected experts' weights.
+ *   [GGUF]    page "Ling-3.0-flash-GGUF", "Measured performance": a decode
+ *             step touches just the chosen experts' weights.
  *   [Q8]      model card "Ling-3.0-tiny-8bit-XL-mlx", "XL Quantization Recipe"
  *             (routed experts and the dense MLP 8-bit; router and shared
  *             experts bf16); model card "Ling-2.6-flash-JANGTQ", quantization
