@@ -75,8 +75,8 @@ KERNEL_SOURCES = {
                      "route.cuh", "mbarrier.cuh", "common.cuh"],
 }
 MEASURED_TRAFFIC = {
-    ("expert_gate_up", "ling26_flash_t512"): (2887062656, "9f13a7c16c1856c3"),
-    ("expert_down", "ling26_flash_t512"): (1491627008, "9f13a7c16c1856c3"),
+    ("expert_gate_up", "ling26_flash_t512"): (2884745856, "a5d1e9a9b5d9b50a"),
+    ("expert_down", "ling26_flash_t512"): (1491174528, "a5d1e9a9b5d9b50a"),
     ("decode_fused", "ling30_flash_decode_t1"): (121980928, "2285db6e03f385e6"),
 }
 
