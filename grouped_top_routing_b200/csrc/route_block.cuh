@@ -3,9 +3,11 @@
 // Takes the same decisions as the per-token router kernel (route.cuh): the
 // same fp64 score evaluation rounded once to fp32, the same softmax sum
 // association, group scores from the multiset top-2 of each group, and the
-// top-k by (biased score descending, expert id ascending) found by ranking
-// unique 64-bit keys, first within each warp's slice of experts, then among
-// the slices' survivors, which is exact for a total order. Pages: mlxcel issue
+// top-k by (biased score descending, expert id ascending), taken by one warp
+// per token in k rounds of warp arg-max over unique 64-bit keys (order key of
+// the biased score above the complemented id), which is exact for a total
+// order. The block's warps share the per-expert passes (scores, groups, keys);
+// the selection itself needs no block barrier. Pages: mlxcel issue
 // #838 "add Ant Group Ling / Bailing MoE", section "Router: selection uses
 // biased scores, weights come from unbiased scores", and the model card
 // "Ling-2.6-flash-JANGTQ", paragraph "MoE routing".
@@ -24,7 +26,6 @@ constexpr int kMaxSlots = 32;  // T * k: one warp lane per slot
 // on the W warps that share named barrier 1); the results are idx .. n_act.
 template <int W>
 struct Smem {
-  uint64_t cand[kMaxT][W * kMaxSlots];  // per-slice survivors (64-bit keys)
   uint32_t gkey[kMaxT][32];             // group score keys
   uint32_t kept[kMaxT];                 // kept-group masks
   float red[kMaxT][W];
@@ -47,42 +48,45 @@ __device__ __forceinline__ uint64_t sel_key(float s, int e) {
   return ((uint64_t)route_detail::order_key(s) << 32) | (uint64_t)(~(uint32_t)e);
 }
 
-// Level 1: this warp's slice [e0, e1) of token t's experts; lane l holds the
-// keys of experts e0 + l + 32 r. Each key's rank is the number of keys of the
-// slice above it; the ones ranked below k are stored at their rank.
+// The k best of one token's E experts by one warp: lane l holds the keys of
+// experts l + 32 r; each of k rounds takes the warp's largest key (the high
+// words first, then the low words among the lanes holding the largest high
+// word: keys are unique, so the pair is the maximum) and its owner drops it.
+// Round j yields slot j: biased score descending, expert id ascending. Lane 0
+// writes the slot's expert and its unbiased score.
 template <int R>
-__device__ __forceinline__ void rank_slice(const uint64_t* key, int e0, int e1, int k, uint64_t* out) {
+__device__ __forceinline__ void topk_warp(const uint64_t* key, const float* orig, int E, int k, int32_t* idx,
+                                          float* w_raw) {
   const int lane = threadIdx.x & 31;
   uint64_t mine[R];
-  int rank[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const int e = e0 + lane + 32 * r;
-    mine[r] = e < e1 ? key[e] : 0ull;
-    rank[r] = 0;
+    const int e = lane + 32 * r;
+    mine[r] = e < E ? key[e] : 0ull;  // 0 is below every real key
   }
-#pragma unroll 4
-  for (int j = e0; j < e1; ++j) {
-    const uint64_t kj = key[j];  // the same address in every lane: a broadcast
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = mine[0];
 #pragma unroll
-    for (int r = 0; r < R; ++r) rank[r] += kj > mine[r] ? 1 : 0;
+    for (int r = 1; r < R; ++r) best = mine[r] > best ? mine[r] : best;
+    const uint32_t hi = (uint32_t)(best >> 32);
+    const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t ml = __reduce_max_sync(0xffffffffu, hi == mh ? (uint32_t)best : 0u);
+    const uint64_t win = ((uint64_t)mh << 32) | ml;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (mine[r] == win) mine[r] = 0ull;
+    if (lane == 0) {
+      const int e = (int)(~ml);
+      idx[j] = e;
+      w_raw[j] = orig[e];
+    }
   }
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-    if (e0 + lane + 32 * r < e1 && rank[r] < k) out[rank[r]] = mine[r];
 }
 
-// Routes the T tokens with the consumer warps; results land in sm (slot
-// experts, weights, the distinct experts with their slots). Ends synchronised.
-// bias: the expert bias in shared memory, or null. Scratch: [T*E] fp32
-// scores, [T*E] fp32 biased scores, [T*E] 64-bit keys (first used for the
-// softmax exponentials).
 template <int W>
 __device__ void route_block(const DecodeArgs& a, const float* logits, const float* bias, unsigned char* scratch,
                             Smem<W>& sm) {
-  // up to 1024 experts: with at least four warps per token a warp's slice is
-  // at most 8 experts per lane (rank_slice<8>)
-  static_assert(W >= 8 && W % 2 == 0, "route_block needs an even number of at least 8 warps");
+  static_assert(W >= kMaxT, "route_block needs a warp per token");
   constexpr int kConsumerWarps = W, kConsumers = W * 32;
   auto consumer_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); };
   using namespace route_detail;
@@ -201,41 +205,19 @@ __device__ void route_block(const DecodeArgs& a, const float* logits, const floa
   }
   consumer_sync();
 
-  // ---- level 1: the k best of each warp's slice of its token's experts ----
-  const int wpt = kConsumerWarps / T;
-  {
-    const int t = warp / wpt, wl = warp - t * wpt;
-    const int chunk = (E + wpt - 1) / wpt;
-    const int e0 = min(E, wl * chunk), e1 = min(E, e0 + chunk);
-    uint64_t* out = sm.cand[t] + wl * k;
-    const int per = (e1 - e0 + 31) / 32;
-    if (per <= 2) rank_slice<2>(s_key + t * E, e0, e1, k, out);
-    else if (per <= 4) rank_slice<4>(s_key + t * E, e0, e1, k, out);
-    else rank_slice<8>(s_key + t * E, e0, e1, k, out);
-    for (int j = min(k, e1 - e0) + lane; j < k; j += 32) out[j] = 0ull;  // fewer experts than k: padding
+  // ---- top-k of token t by warp t (E <= 1024: at most 32 keys per lane) ----
+  if (warp < T) {
+    const int t = warp;
+    const uint64_t* key = s_key + t * E;
+    const float* orig = s_orig + t * E;
+    const int R = (E + 31) / 32;
+    if (R <= 2) topk_warp<2>(key, orig, E, k, sm.idx + t * k, sm.w_raw + t * k);
+    else if (R <= 4) topk_warp<4>(key, orig, E, k, sm.idx + t * k, sm.w_raw + t * k);
+    else if (R <= 8) topk_warp<8>(key, orig, E, k, sm.idx + t * k, sm.w_raw + t * k);
+    else if (R <= 16) topk_warp<16>(key, orig, E, k, sm.idx + t * k, sm.w_raw + t * k);
+    else topk_warp<32>(key, orig, E, k, sm.idx + t * k, sm.w_raw + t * k);
+    __syncwarp();
   }
-  consumer_sync();
-
-  // ---- level 2: rank the survivors of the token's slices; rank j is slot j ----
-  {
-    const int per_tok = kConsumers / T;
-    const int t = threadIdx.x / per_tok, c = threadIdx.x - t * per_tok;
-    const int nc = wpt * k;
-    if (c < nc) {
-      const uint64_t mine = sm.cand[t][c];
-      if (mine != 0ull) {
-        int rank = 0;
-#pragma unroll 8
-        for (int j = 0; j < nc; ++j) rank += sm.cand[t][j] > mine ? 1 : 0;
-        if (rank < k) {
-          const int e = (int)(~(uint32_t)mine);
-          sm.idx[t * k + rank] = e;
-          sm.w_raw[t * k + rank] = s_orig[t * E + e];
-        }
-      }
-    }
-  }
-  consumer_sync();
 
   // ---- weights: renormalise (k > 1) with the 1e-20 epsilon, then scale; fp32, slot order ----
   if (warp < T) {
