@@ -430,6 +430,7 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
 
   const int n_router = a.logits_override == nullptr ? E : 0;
   const float* logits = a.logits_override != nullptr ? a.logits_override : a.logits;
+  const bool pre_scores = block_route::scores_with_logits(a);
   const int target = k + (a.ws_down != nullptr ? 1 : 0);
   Pending<kMaxPend> q;
   q.np = 0;
@@ -470,8 +471,11 @@ __device__ void consumer(const DecodeArgs& a, const Geo& g, unsigned char* ring,
       const int i = sg.r.lo + (int)u;
       if (i < n_router) {
         const float v = router_unit(reinterpret_cast<const float*>(st), H, xs, T, empty);
-        if (lane == 0) a.logits[i] = v;
-        if (lane == 16 && T > 1) a.logits[E + i] = v;
+        if (lane == 0 || (lane == 16 && T > 1)) {
+          const int t = lane >> 4;
+          a.logits[t * E + i] = v;
+          if (pre_scores) block_route::store_score(a, t, i, v, bias_s);
+        }
       } else {
         const int j = i - n_router;
         const uint16_t* gate = reinterpret_cast<const uint16_t*>(st);

@@ -25,6 +25,11 @@ struct DecodeArgs {
   float* y_slots;                // [T*k, H] workspace
   float* shared_out;             // [T, H] workspace
   int32_t* sync;                 // decode_fused_sync_ints(H) counters, workspace
+  // Sigmoid scores and selection keys computed with each router logit (null:
+  // the routing computes them from the logits): [T, E] fp32 unbiased scores and
+  // [T, E] 64-bit keys, workspace.
+  float* pre_orig;
+  unsigned long long* pre_key;
   uint16_t* y;                   // [T, H] output
   WsHeader* hdr;
 };

@@ -506,6 +506,7 @@ __device__ void consumer(const DecodeArgs& a, const unsigned char* ring, int dep
   consumer_sync();
 
   const float* logits = a.logits_override != nullptr ? a.logits_override : a.logits;
+  const bool pre_scores = block_route::scores_with_logits(a);
   const int target = k + (a.ws_down != nullptr ? 1 : 0);
   Pending<kMaxPend> q;
   q.np = 0;
@@ -541,9 +542,10 @@ __device__ void consumer(const DecodeArgs& a, const unsigned char* ring, int dep
       break;
     }
     const float2 lg = router_row(st, H, xs, T, empty);
-    if (lane == 0) {
-      a.logits[i] = lg.x;
-      if (T > 1) a.logits[E + i] = lg.y;
+    if (lane < T) {  // lane t: token t
+      const float v = lane == 0 ? lg.x : lg.y;
+      a.logits[lane * E + i] = v;
+      if (pre_scores) block_route::store_score(a, lane, i, v, bias_s);
     }
   }
   if (!grid_barrier<kConsumers>(a.hdr, 1, &sm.flag) || sm.abort != 0) return;

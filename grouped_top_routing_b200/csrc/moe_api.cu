@@ -179,7 +179,7 @@ constexpr int64_t kLogitsGemvMaxT = 16;  // larger batches: router logits on the
 
 struct Layout {
   size_t hdr, logits, wr_planes, logit_parts, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
-  size_t x_perm, h_perm, h_shared, y_slots, shared_out, decode_sync, total;
+  size_t x_perm, h_perm, h_shared, y_slots, shared_out, decode_sync, decode_pre, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -236,6 +236,7 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   const bool fused = decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is) ||
                      decode_tc_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
   L.decode_sync = take(fused ? decode_fused_sync_ints((int)H) * 4 : 0);
+  L.decode_pre = take(fused ? (size_t)2 * E * 12 : 0);  // up to 2 tokens: scores then keys
   L.total = off;
   return L;
 }
@@ -602,6 +603,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
     d.y_slots = at<float>(ws, L.y_slots);
     d.shared_out = at<float>(ws, L.shared_out);
     d.sync = at<int32_t>(ws, L.decode_sync);
+    d.pre_orig = at<float>(ws, L.decode_pre);
+    d.pre_key = reinterpret_cast<unsigned long long*>(at<char>(ws, L.decode_pre) + (size_t)2 * c.num_experts * 4);
     d.y = y;
     d.hdr = hdr;
     cudaError_t e = tc_ok ? launch_decode_tc(d, s) : launch_decode_fused(d, s);
