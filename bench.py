@@ -77,7 +77,7 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     ("expert_gate_up", "ling26_flash_t512"): (2884745856, "a5d1e9a9b5d9b50a"),
     ("expert_down", "ling26_flash_t512"): (1491174528, "a5d1e9a9b5d9b50a"),
-    ("decode_fused", "ling30_flash_decode_t1"): (121981952, "51948401c494c085"),
+    ("decode_fused", "ling30_flash_decode_t1"): (121844992, "482c39e62c1e6fa6"),
 }
 
 
