@@ -269,3 +269,25 @@ def test_forward_q8_rejects_null_weights(M):
     st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, None, None, None, fake, None, None,
                               fake, 1 << 40, None)
     assert st == 1 and "NULL" in M.last_error()
+
+
+def test_binding_checks_tensor_sizes_against_the_config(M):
+    # The C ABI sees raw pointers only; the binding refuses tensors whose size
+    # disagrees with the config before anything reaches the device.
+    from grouped_top_routing_b200 import inputs as G
+    wl = G.tiny_workload(tokens=2, hidden_size=64, moe_intermediate_size=32, shared_width=32)
+    inp = G.make_inputs(wl, seed=0, device="cpu")
+    args = dict(x=inp["x"], router_w=inp["router_w"], expert_bias=inp["expert_bias"], w_gate_up=inp["w_gate_up"],
+                w_down=inp["w_down"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"])
+    for name in ("router_w", "w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+        bad = dict(args, **{name: args[name].reshape(-1)[:-8]})
+        with pytest.raises(ValueError, match=name):
+            M.moe_forward(wl, ws=None, **bad)
+    # a shared MLP wider than the config says (the width the library derives is
+    # moe_intermediate_size x num_shared_experts)
+    wide = G.make_inputs(dict(wl, shared_width=64), seed=0, device="cpu")
+    with pytest.raises(ValueError, match="ws_gate_up"):
+        M.moe_forward(wl, ws=None, **dict(args, ws_gate_up=wide["ws_gate_up"], ws_down=wide["ws_down"]))
+    assert M.shared_width(M.config_from_workload(wl)) == 32
+    assert M.shared_width(M.config_from_workload(dict(wl, num_shared_experts=2))) == 64
+    assert M.shared_width(M.config_from_workload(dict(wl, num_shared_experts=0))) == 0
