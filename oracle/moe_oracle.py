@@ -82,6 +82,9 @@ MUTATIONS = (
     "group_top1",           # group score from the top-1 only
     "shared_routed_weight",  # shared MLP weighted like a routed expert
     "bias_not_in_selection",  # bias ignored by the selection
+    "logits_layout",        # router weight [E, H] read as if it were stored [H, E]
+    "gap_next_pair",        # selection gap taken one rank too deep ((k+1)-th minus (k+2)-th)
+    "group_gap_unbiased",   # group gaps ranked on the unbiased scores
 )
 
 
@@ -139,12 +142,14 @@ def shared_width(moe_intermediate_size: int, num_shared_experts: int,
 # Router
 # --------------------------------------------------------------------------
 
-def router_logits(x, router_w) -> np.ndarray:
+def router_logits(x, router_w, mutate=None) -> np.ndarray:
     """gates = x . W_r^T for the router projection (mlp.gate, weight [E, H]),
     accumulated in fp64 and rounded once to the fp32 the router works in
     [ROUTER]: the gates are cast to float32 before the score function."""
     X = as_f64(x)
     W = as_f64(router_w)
+    if mutate == "logits_layout":
+        W = W.reshape(W.shape[1], W.shape[0]).T
     return (X @ W.T).astype(np.float32)
 
 
@@ -249,25 +254,30 @@ def route(logits, expert_bias, cfg: dict, mutate=None, return_keys=False):
     return idx, w
 
 
-def selection_gaps(sel: np.ndarray, k: int) -> np.ndarray:
+def selection_gaps(sel: np.ndarray, k: int, mutate=None) -> np.ndarray:
     """Per token, sel[k-th] - sel[(k+1)-th] of the masked biased scores
-    (inf when k == E). Tokens with a gap under 1e-6 are near-ties."""
+    (inf when k == E, and when the (k+1)-th is a masked -inf). Tokens with a
+    gap under 1e-6 are near-ties."""
     srt = -np.sort(-sel, axis=1)
-    if k >= sel.shape[1]:
+    d = 1 if mutate == "gap_next_pair" else 0
+    if k + d >= sel.shape[1]:
         return np.full(sel.shape[0], np.inf)
-    a = srt[:, k - 1].astype(np.float64)
-    b = srt[:, k].astype(np.float64)
+    a = srt[:, k - 1 + d].astype(np.float64)
+    b = srt[:, k + d].astype(np.float64)
     with np.errstate(invalid="ignore"):
         g = a - b
     return np.where(np.isfinite(b), g, np.inf)
 
 
-def group_gaps(s: np.ndarray, expert_bias, n_group: int, topk_group: int) -> np.ndarray:
-    """Per token, the gap between the topk_group-th and next group score."""
+def group_gaps(s: np.ndarray, expert_bias, n_group: int, topk_group: int, mutate=None) -> np.ndarray:
+    """Per token, the gap between the topk_group-th and next group score, the
+    group scores taken on the biased selection copy as the selection does
+    (inf when every group is kept)."""
     T, E = s.shape
     if n_group <= 1 or topk_group >= n_group:
         return np.full(T, np.inf)
-    sel = s if expert_bias is None else (s + as_f32(expert_bias)[None, :]).astype(np.float32)
+    unbiased = expert_bias is None or mutate == "group_gap_unbiased"
+    sel = s if unbiased else (s + as_f32(expert_bias)[None, :]).astype(np.float32)
     gs = group_scores(sel, n_group)
     srt = -np.sort(-gs, axis=1)
     return srt[:, topk_group - 1].astype(np.float64) - srt[:, topk_group].astype(np.float64)
@@ -389,7 +399,10 @@ def moe_block(inp: dict, cfg: dict, logits=None, idx=None, w=None, mutate=None,
         Wg, Wu, Wd = expert_weights_f64(inp["w_gate_up"], inp["w_down"], int(e), I)
         Ye = swiglu_mlp(X[t_sel], Wg, Wu, Wd)
         wt = np.asarray(w, dtype=np.float32)[t_sel, j_sel].astype(np.float64)
-        np.add.at(y, t_sel, wt[:, None] * Ye)
+        # a token holds an expert in at most one slot, so the rows of t_sel are
+        # distinct and a plain indexed add is the per-row sum
+        assert np.unique(t_sel).size == t_sel.size, "a token selected one expert twice"
+        y[t_sel] += wt[:, None] * Ye
     if cfg.get("num_shared_experts", 0) > 0 and inp.get("ws_gate_up") is not None:
         Wg, Wu, Wd = shared_weights_f64(inp["ws_gate_up"], inp["ws_down"])
         ys = swiglu_mlp(X, Wg, Wu, Wd)

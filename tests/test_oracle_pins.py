@@ -428,13 +428,93 @@ def test_zero_mask_reading_agrees_on_workload(name):
 
 
 # --------------------------------------------------------------------------
+# Router projection and the tie-band helpers
+# --------------------------------------------------------------------------
+
+def check_router_logits_exact(mutate=None):
+    # logits[t, e] = sum_h x[t, h] * W[e, h], on non-square shapes (E != H)
+    # whose inputs are small dyadic numbers: every product and partial sum is
+    # exact in fp64, so the oracle must equal a plain Python double loop bit
+    # for bit (mlxcel issue #838, section "Router: ...": gates = gate_proj(x)).
+    rng = np.random.default_rng(7)
+    for T, H, E in ((3, 5, 4), (2, 8, 3), (4, 6, 9)):
+        x = (rng.integers(-8, 9, (T, H)) / 8.0).astype(np.float32)
+        W = (rng.integers(-16, 17, (E, H)) / 16.0).astype(np.float32)
+        got = O.router_logits(x, W, mutate=mutate)
+        assert got.shape == (T, E) and got.dtype == np.float32
+        for t in range(T):
+            for e in range(E):
+                acc = 0.0
+                for h in range(H):
+                    acc += float(x[t, h]) * float(W[e, h])
+                assert got[t, e] == np.float32(acc), (T, H, E, t, e, got[t, e], acc)
+
+
+def test_router_logits_exact():
+    check_router_logits_exact()
+
+
+def _f64(v):
+    return np.float64(np.float32(v))
+
+
+def check_selection_gaps(mutate=None):
+    # Hand-worked gaps between the k-th and (k+1)-th biased keys.
+    ninf = -np.inf
+    sel = np.array([[0.9, 0.5, 0.5, 0.1],
+                    [0.7, ninf, 0.3, ninf],
+                    [0.2, 0.6, 0.4, 0.8]], dtype=np.float32)
+    g1 = O.selection_gaps(sel, 1, mutate=mutate)
+    assert g1[0] == _f64(0.9) - _f64(0.5) and g1[1] == _f64(0.7) - _f64(0.3)
+    assert g1[2] == _f64(0.8) - _f64(0.6)
+    g2 = O.selection_gaps(sel, 2, mutate=mutate)
+    assert g2[0] == 0.0, g2          # an exact tie at the boundary: gap 0
+    assert g2[1] == np.inf, g2        # the (k+1)-th is a masked expert
+    assert g2[2] == _f64(0.6) - _f64(0.4)
+    g3 = O.selection_gaps(sel, 3, mutate=mutate)
+    assert g3[0] == _f64(0.5) - _f64(0.1) and g3[1] == np.inf
+    assert np.all(O.selection_gaps(sel, 4, mutate=mutate) == np.inf)  # k == E: nothing left out
+
+
+def test_selection_gaps():
+    check_selection_gaps()
+
+
+def check_group_gaps(mutate=None):
+    # Four groups of two experts, top-2 groups kept. Group scores are top-1 +
+    # top-2 of the BIASED keys, each an fp32 add; the gap is between the 2nd
+    # and 3rd best group.
+    s = np.array([[0.1, 0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8]], dtype=np.float32)
+    b = np.array([0.5, 0.5, 0, 0, 0, 0, 0, 0], dtype=np.float32)
+    sel = (s + b).astype(np.float32)
+    gs = [np.float32(sel[0, 2 * q] + sel[0, 2 * q + 1]) for q in range(4)]  # 1.3, 0.7, 1.1, 1.5
+    g = O.group_gaps(s, b, 4, 2, mutate=mutate)
+    assert g[0] == np.float64(gs[0]) - np.float64(gs[2]), (g, gs)
+    # without a bias the order changes: 1.5, 1.1, 0.7, 0.3
+    g = O.group_gaps(s, None, 4, 2, mutate=mutate)
+    assert g[0] == np.float64(np.float32(np.float32(0.5) + np.float32(0.6))) - \
+        np.float64(np.float32(np.float32(0.3) + np.float32(0.4)))
+    # two groups with bitwise-equal scores at the boundary: gap 0
+    t = np.array([[0.2, 0.3, 0.3, 0.2, 0.9, 0.9, 0.0, 0.1]], dtype=np.float32)
+    assert O.group_gaps(t, None, 4, 2, mutate=mutate)[0] == 0.0
+    # every group kept, or no groups: no group boundary
+    assert O.group_gaps(s, b, 4, 4, mutate=mutate)[0] == np.inf
+    assert O.group_gaps(s, b, 1, 1, mutate=mutate)[0] == np.inf
+
+
+def test_group_gaps():
+    check_group_gaps()
+
+
+# --------------------------------------------------------------------------
 # Mutation checks: every planted bug must be caught by at least one pin.
 # --------------------------------------------------------------------------
 
 CHECKS = [check_worked_examples, check_score_closed_forms, check_selection_brute_force,
           check_selected_inside_groups_negative_keys, check_topk_is_argsort_of_logits,
           check_bias_selection_only, check_normalisation, check_topk_all_is_dense_softmax,
-          check_sparse_equals_dense, check_scale_zero_leaves_shared_only]
+          check_sparse_equals_dense, check_scale_zero_leaves_shared_only, check_router_logits_exact,
+          check_selection_gaps, check_group_gaps]
 
 
 @pytest.mark.parametrize("mutation", O.MUTATIONS)
