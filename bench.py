@@ -33,7 +33,7 @@ from grouped_top_routing_b200 import inputs as G  # noqa: E402
 
 METRIC = "MoE-block tokens/s at 1 B200; HBM GB/s (decode) & TFLOPS (prefill) vs roofline"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "ling26_flash_t512"
+DEFAULT_WORKLOAD = "ling26_flash_prefill_t32768"
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20  # B200 L2
 FALLBACK_HBM_GBS = 6650.0
@@ -92,10 +92,10 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decode_kernel: str = "auto"):
+def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decode: str = "auto"):
     """Bytes per launch from the capture, or None when it no longer applies."""
     entry = MEASURED_TRAFFIC.get((kernel, workload))
-    if entry is None or overrides or ffn_path != "auto" or decode_kernel != "auto":
+    if entry is None or overrides or ffn_path != "auto" or decode != "auto":
         return None
     return entry[0] if kernel_source_hash(kernel) == entry[1] else None
 
@@ -290,15 +290,17 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    M.set_ffn_path(args.ffn_path)
-    M.set_decode_kernel(args.decode_kernel)
     wl = workload_from_args(args)
     inp = G.make_inputs(wl, seed=0, device=dev)
     T = inp["tokens"]
     q8 = G.make_q8_weights(wl, seed=0, device=dev, group_size=args.q8) if args.q8 else None
-    if args.kernel == "auto":
-        fused = args.ffn_path == "auto" and T <= M.FUSED_DECODE_MAX_TOKENS and q8 is None
-        args.kernel = "decode_fused" if fused else "expert_gate_up"
+    fused = args.decode == "auto" and T <= M.FUSED_DECODE_MAX_TOKENS and q8 is None
+    # kernels timed live inside the steps (steps alternate between them when
+    # there are two); the roofline line reports the one that takes longer
+    if args.kernel != "auto":
+        timed = [args.kernel]
+    else:
+        timed = ["decode_fused"] if fused else ["expert_gate_up", "expert_down"]
     if rank > 0:  # each rank its own batch (weak scaling), same weights
         g = torch.Generator(device=dev)
         g.manual_seed(rank_activation_seed(rank))
@@ -308,13 +310,17 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(x=None, out=None):
+    base_opts = dict(ffn_path=args.ffn_path, decode=args.decode)
+
+    def step(x=None, out=None, timer=None):
         out = y if out is None else out
+        opts = M.options(timer=timer, **base_opts)
         if q8 is not None:
             return M.moe_forward_q8(wl, inp["x"] if x is None else x, inp["router_w"], inp["expert_bias"], q8, ws,
-                                    y=out)
+                                    y=out, opts=opts)
         return M.moe_forward(wl, inp["x"] if x is None else x, inp["router_w"], inp["expert_bias"],
-                             inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"], inp["ws_down"], ws, y=out)
+                             inp["w_gate_up"], inp["w_down"], inp["ws_gate_up"], inp["ws_down"], ws, y=out,
+                             opts=opts)
 
     warm = max(args.warmup, 3)
     for _ in range(warm):
@@ -324,7 +330,8 @@ def run_ours(args):
 
     # routing of this batch: distinct experts touched (algorithmic bytes)
     _, idx, _ = M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
-                              inp["ws_gate_up"], inp["ws_down"], ws, return_routing=True)
+                              inp["ws_gate_up"], inp["ws_down"], ws, return_routing=True,
+                              opts=M.options(**base_opts))
     n_unique = int(torch.unique(idx).numel())
     work = algorithmic(wl, T, n_unique, 1.0 + 4.0 / args.q8 if q8 is not None else 2.0)
 
@@ -341,11 +348,9 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         for i in range(K):
             flush.zero_()  # L2 flush, outside the timed events
-            M.set_kernel_timer(args.kernel, kev[i][0], kev[i][1])
             ev[i][0].record(stream)
-            step()
+            step(timer=(timed[i % len(timed)], kev[i][0], kev[i][1]))
             ev[i][1].record(stream)
-        M.set_kernel_timer(args.kernel)
         torch.cuda.synchronize(dev)
     launches = M.launch_count() - launches0
     if world > 1:
@@ -353,7 +358,9 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     ws.check()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_ms = [a.elapsed_time(b) for a, b in kev]
+    kern_ms = {name: [kev[i][0].elapsed_time(kev[i][1]) for i in range(K) if timed[i % len(timed)] == name]
+               for name in timed}
+    kernel = max(timed, key=lambda n: statistics.mean(kern_ms[n]))  # the dominant one
     total_ms = sum(step_ms)
 
     # e2e: host pinned x in, host y out, through the same public call. When a
@@ -429,28 +436,33 @@ def run_ours(args):
     e2e_value = whole_job_rate(T, world, e2e_ms / K)
 
     pk = peaks()
-    kms = statistics.mean(kern_ms)
-    if args.kernel == "decode_fused":  # the whole block in one kernel
+    kms = statistics.mean(kern_ms[kernel])
+    if kernel == "decode_fused":  # the whole block in one kernel
         kbytes, kflops = work["step_bytes"], work["flops"]
     else:
-        kbytes = work["gate_up_bytes"] if args.kernel == "expert_gate_up" else work["down_bytes"]
-        kflops = work["gate_up_flops"] if args.kernel == "expert_gate_up" else work["down_flops"]
-    traffic = None if q8 is not None else measured_traffic(args.kernel, args.workload, args.set, args.ffn_path, args.decode_kernel)
+        kbytes = work["gate_up_bytes"] if kernel == "expert_gate_up" else work["down_bytes"]
+        kflops = work["gate_up_flops"] if kernel == "expert_gate_up" else work["down_flops"]
+    traffic = None if q8 is not None else measured_traffic(kernel, args.workload, args.set, args.ffn_path, args.decode)
+    others = {n: statistics.mean(v) for n, v in kern_ms.items() if n != kernel}
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if kflops / kbytes > ridge:
+        # The kernel runs inside long back-to-back steps (power-capped), so the
+        # denominator is the sustained bf16 figure; the burst fraction is kept
+        # beside it.
         achieved = kflops / (kms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "kernel": args.kernel, "achieved": achieved, "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
-                    "peak_source": pk["source"] + " (bf16 burst)", "algorithmic_flops": kflops,
-                    "algorithmic_bytes": kbytes, "kernel_ms": kms,
-                    "hbm_gbs": kbytes / (kms / 1e3) / 1e9}
+        peak = pk["bf16_tflops_sustained"]
+        roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": pk["source"] + " (bf16 sustained)", "frac_of_burst": achieved / pk["bf16_tflops"],
+                    "algorithmic_flops": kflops, "algorithmic_bytes": kbytes, "kernel_ms": kms,
+                    "hbm_gbs": kbytes / (kms / 1e3) / 1e9, "other_kernels_ms": others}
     else:
         achieved = kbytes / (kms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": args.kernel, "achieved": achieved, "peak": pk["hbm_gbs"],
+        roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"],
                     "algorithmic_bytes": kbytes, "algorithmic_flops": kflops, "kernel_ms": kms,
-                    "tflops": kflops / (kms / 1e3) / 1e12}
+                    "tflops": kflops / (kms / 1e3) / 1e12, "other_kernels_ms": others}
     step_gbs = work["step_bytes"] / (ms_per_step / 1e3) / 1e9
     step_tflops = work["flops"] / (ms_per_step / 1e3) / 1e12
 
@@ -471,7 +483,7 @@ def run_ours(args):
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "overrides": args.set, "ffn_path": args.ffn_path,
-                   "decode_kernel": args.decode_kernel, "tokens": T, "hidden_size": wl["hidden_size"],
+                   "decode": args.decode, "tokens": T, "hidden_size": wl["hidden_size"],
                    "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
@@ -516,8 +528,9 @@ def run_dense(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(x=None):
-        return M.moe_dense_mlp(inp["x"] if x is None else x, inp["w_gate_up"], inp["w_down"], ws, y=y)
+    def step(x=None, timer=None):
+        return M.moe_dense_mlp(inp["x"] if x is None else x, inp["w_gate_up"], inp["w_down"], ws, y=y,
+                               opts=M.options(timer=timer))
 
     warm = max(args.warmup, 3)
     for _ in range(warm):
@@ -535,11 +548,9 @@ def run_dense(args):
     with ClockSampler(0) as clk:
         for i in range(K):
             flush.zero_()  # L2 flush, outside the timed events
-            M.set_kernel_timer("expert_gate_up", kev[i][0], kev[i][1])
             ev[i][0].record(stream)
-            step()
+            step(timer=("expert_gate_up", kev[i][0], kev[i][1]))
             ev[i][1].record(stream)
-        M.set_kernel_timer("expert_gate_up")
         torch.cuda.synchronize(dev)
     launches = M.launch_count() - launches0
     ws.check()
@@ -609,14 +620,14 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(G.WORKLOADS))
     ap.add_argument("--kernel", default="auto", choices=["auto", "expert_gate_up", "expert_down", "decode_fused"],
                     help="kernel whose live timing gives the roofline (auto: the fused decode kernel when the "
-                         "library runs the block as one launch, else the gate/up expert pass)")
+                         "library runs the block as one launch, else whichever expert pass takes longer)")
     ap.add_argument("--cpu-sample", type=int, default=64)
     ap.add_argument("--ref-sample", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "streaming", "tensor_cores"],
                     help="expert-FFN kernels (default: the library's automatic choice)")
-    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "cuda_cores", "tensor_cores"],
-                    help="fused decode kernel for 1-2 tokens (default: the library's choice, the CUDA-core kernel)")
+    ap.add_argument("--decode", default="auto", choices=["auto", "unfused"],
+                    help="a few tokens as one fused launch (auto, the library's choice) or as separate kernels")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (e.g. num_experts=64 for a small profiling case)")
     ap.add_argument("--q8", type=int, default=0, metavar="GROUP",

@@ -121,5 +121,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 void before_launch(int kernel_id, cudaStream_t s);
 void after_launch(int kernel_id, cudaStream_t s, int nkernels = 1);
 int sm_count();
+// Options of the entry point running on this thread (moe_options; defaults
+// outside a call): the bound on device waits and the test aid.
+uint64_t opt_wait_ns();
+int opt_withhold();
 
 }  // namespace moe

@@ -32,6 +32,7 @@ struct DecodeArgs {
   unsigned long long* pre_key;
   uint16_t* y;                   // [T, H] output
   WsHeader* hdr;
+  uint64_t wait_ns;  // bound on every device-side wait
 };
 
 // Completion counters the kernels need in the workspace (zeroed by the kernels):
@@ -41,11 +42,5 @@ size_t decode_fused_sync_ints(int H);
 // slots, hidden size up to 8192, expert widths up to twice the hidden size).
 bool decode_fused_supported(int64_t T, int k, int E, int H, int I, int Is);
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t s);
-
-// The tensor-core variant (decode_tc.cu): hidden size a multiple of 512 up to
-// 4096, expert and shared widths multiples of 16 up to 512. It uses the same
-// workspace (h and h_shared hold bf16 there) and the same sync counters.
-bool decode_tc_supported(int64_t T, int k, int E, int H, int I, int Is);
-cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace moe

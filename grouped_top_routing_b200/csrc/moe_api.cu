@@ -42,12 +42,12 @@ cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok
 namespace {
 
 thread_local char g_err[512] = "";
-std::atomic<uint64_t> g_launches{0};
-void* g_ev_start[MOE_KERNEL_COUNT] = {};
-void* g_ev_stop[MOE_KERNEL_COUNT] = {};
+thread_local uint64_t t_launches = 0;
+// The options of the entry point running on this thread (set for the
+// duration of one call by CallScope, null otherwise): kernel choices, the
+// wait limit and the timing hook. Nothing outlives the call.
+thread_local const moe_options* t_opts = nullptr;
 int g_sm_count[64] = {};
-int g_ffn_path = 0;  // 0 auto, 1 streaming GEMV, 2 tensor cores
-int g_decode_kernel = 0;  // 0 auto (the CUDA-core fused decode), 1 CUDA cores, 2 tensor cores where the shapes fit
 
 moe_status fail(moe_status st, const char* fmt, ...) {
   va_list ap;
@@ -61,17 +61,50 @@ moe_status cuda_fail(cudaError_t e, const char* where) {
   return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+// Installs a call's options on this thread for the duration of the call.
+struct CallScope {
+  explicit CallScope(const moe_options* o) { t_opts = o; }
+  ~CallScope() { t_opts = nullptr; }
+  CallScope(const CallScope&) = delete;
+  CallScope& operator=(const CallScope&) = delete;
+};
+
+moe_status validate_options(const moe_options* o) {
+  if (o == nullptr) return MOE_OK;
+  if (o->ffn_path < 0 || o->ffn_path > 2)
+    return fail(MOE_ERR_INVALID_ARG, "opts->ffn_path = %d is not 0 (auto), 1 (streaming) or 2 (tensor cores)",
+                o->ffn_path);
+  if (o->decode_kernel < 0 || o->decode_kernel > 1)
+    return fail(MOE_ERR_INVALID_ARG, "opts->decode_kernel = %d is not 0 (auto) or 1 (never fused)", o->decode_kernel);
+  if (o->timer_kernel < -1 || o->timer_kernel >= MOE_KERNEL_COUNT)
+    return fail(MOE_ERR_INVALID_ARG, "opts->timer_kernel = %d is not a kernel id or -1", o->timer_kernel);
+  if (o->timer_kernel >= 0 && (o->timer_start == nullptr || o->timer_stop == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "opts->timer_kernel = %d needs both timer events", o->timer_kernel);
+  if (o->test_withhold < 0 || o->test_withhold > 2)
+    return fail(MOE_ERR_INVALID_ARG, "opts->test_withhold = %d is not 0, 1 or 2", o->test_withhold);
+  return MOE_OK;
+}
+
 }  // namespace
 
+int opt_ffn_path() { return t_opts != nullptr ? t_opts->ffn_path : 0; }
+int opt_decode_kernel() { return t_opts != nullptr ? t_opts->decode_kernel : 0; }
+int opt_withhold() { return t_opts != nullptr ? t_opts->test_withhold : 0; }
+uint64_t opt_wait_ns() {
+  return (t_opts != nullptr && t_opts->wait_limit_ns != 0) ? t_opts->wait_limit_ns : kDefaultWaitNs;
+}
+
 void before_launch(int id, cudaStream_t s) {
-  if (id >= 0 && id < MOE_KERNEL_COUNT && g_ev_start[id] != nullptr)
-    cudaEventRecord(static_cast<cudaEvent_t>(g_ev_start[id]), s);
+  if (t_opts != nullptr && t_opts->timer_kernel == id && t_opts->timer_start != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(t_opts->timer_start), s);
 }
 
 void after_launch(int id, cudaStream_t s, int nkernels) {
-  g_launches.fetch_add((uint64_t)nkernels, std::memory_order_relaxed);
-  if (id >= 0 && id < MOE_KERNEL_COUNT && g_ev_stop[id] != nullptr)
-    cudaEventRecord(static_cast<cudaEvent_t>(g_ev_stop[id]), s);
+  t_launches += (uint64_t)nkernels;
+  if (t_opts != nullptr && t_opts->timer_kernel == id && t_opts->timer_stop != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(t_opts->timer_stop), s);
 }
 
 int sm_count() {
@@ -233,8 +266,7 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 4);
   L.y_slots = take((size_t)R * H * 4);
   L.shared_out = take((size_t)T * H * 4);
-  const bool fused = decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is) ||
-                     decode_tc_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
+  const bool fused = decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
   L.decode_sync = take(fused ? decode_fused_sync_ints((int)H) * 4 : 0);
   L.decode_pre = take(fused ? (size_t)2 * E * 12 : 0);  // up to 2 tokens: scores then keys
   L.total = off;
@@ -278,8 +310,8 @@ constexpr int64_t kStreamMaxT = 2;
 
 bool use_tensor_cores(const moe_config& c, int64_t T) {
   (void)c;
-  if (g_ffn_path == 1) return false;
-  if (g_ffn_path == 2) return true;
+  if (opt_ffn_path() == 1) return false;
+  if (opt_ffn_path() == 2) return true;
   return T > kStreamMaxT;
 }
 
@@ -506,7 +538,9 @@ moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, c
                           const int32_t* expert_offsets, const int32_t* tok_of, const float* topk_w,
                           const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* ws_gate_up,
                           const uint16_t* ws_down, float* y_slots, float* shared_out, void* ws,
-                          size_t ws_bytes, void* stream) {
+                          size_t ws_bytes, void* stream, const moe_options* opts) {
+  MOE_TRY(validate_options(opts));
+  CallScope scope(opts);
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
@@ -547,7 +581,10 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
 moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
                        const float* expert_bias, const float* logits_override, const uint16_t* w_gate_up,
                        const uint16_t* w_down, const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y,
-                       int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+                       int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream,
+                       const moe_options* opts) {
+  MOE_TRY(validate_options(opts));
+  CallScope scope(opts);
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
@@ -571,10 +608,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
-  const bool tc_ok = g_decode_kernel == 2 && decode_tc_supported(T, c.num_experts_per_tok, c.num_experts,
-                                                                  c.hidden_size, c.moe_intermediate_size, shared_width(c));
-  if (g_ffn_path == 0 && (tc_ok || decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size,
-                                                         c.moe_intermediate_size, shared_width(c)))) {
+  if (opt_decode_kernel() == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size,
+                                                         c.moe_intermediate_size, shared_width(c))) {
     DecodeArgs d{};
     d.x = x;
     d.T = (int)T;
@@ -607,7 +642,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
     d.pre_key = reinterpret_cast<unsigned long long*>(at<char>(ws, L.decode_pre) + (size_t)2 * c.num_experts * 4);
     d.y = y;
     d.hdr = hdr;
-    cudaError_t e = tc_ok ? launch_decode_tc(d, s) : launch_decode_fused(d, s);
+    d.wait_ns = opt_wait_ns();
+    cudaError_t e = launch_decode_fused(d, s);
     if (e != cudaSuccess) return cuda_fail(e, "fused decode");
     return MOE_OK;
   }
@@ -653,29 +689,7 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
   return fail(MOE_ERR_DEVICE_CHECK, "device index check failed (index %d)", word[1]);
 }
 
-moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop) {
-  if (which < 0 || which >= MOE_KERNEL_COUNT) return fail(MOE_ERR_INVALID_ARG, "which = %d is not a kernel id", which);
-  if ((ev_start == nullptr) != (ev_stop == nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "ev_start and ev_stop must both be set or both be NULL");
-  g_ev_start[which] = ev_start;
-  g_ev_stop[which] = ev_stop;
-  return MOE_OK;
-}
-
-uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
-
-moe_status moe_set_ffn_path(int32_t path) {
-  if (path < 0 || path > 2) return fail(MOE_ERR_INVALID_ARG, "path = %d is not 0 (auto), 1 (streaming) or 2 (tensor cores)", path);
-  g_ffn_path = path;
-  return MOE_OK;
-}
-
-moe_status moe_set_decode_kernel(int32_t which) {
-  if (which < 0 || which > 2)
-    return fail(MOE_ERR_INVALID_ARG, "which = %d is not 0 (auto), 1 (CUDA cores) or 2 (tensor cores)", which);
-  g_decode_kernel = which;
-  return MOE_OK;
-}
+uint64_t moe_launch_count(void) { return t_launches; }
 
 const char* moe_last_error(void) { return g_err; }
 
@@ -689,7 +703,9 @@ size_t moe_dense_mlp_workspace_size(int32_t hidden_size, int32_t intermediate_si
 
 moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const uint16_t* x, int64_t T,
                          const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* y, void* ws, size_t ws_bytes,
-                         void* stream) {
+                         void* stream, const moe_options* opts) {
+  MOE_TRY(validate_options(opts));
+  CallScope scope(opts);
   MOE_TRY(validate_dense(hidden_size, intermediate_size));
   const moe_config c = dense_config(hidden_size, intermediate_size);
   MOE_TRY(check_tokens(c, T));
@@ -717,7 +733,9 @@ moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const u
 moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
                           const float* expert_bias, const float* logits_override, const moe_q8_weights* w,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y, int32_t* topk_idx_out,
-                          float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+                          float* topk_w_out, void* ws, size_t ws_bytes, void* stream, const moe_options* opts) {
+  MOE_TRY(validate_options(opts));
+  CallScope scope(opts);
   MOE_TRY(validate_config(cfg));
   MOE_TRY(check_tokens(*cfg, T));
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));

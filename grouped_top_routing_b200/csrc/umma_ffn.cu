@@ -32,7 +32,8 @@
 // the m-block fastest, so CTAs that share a weight block run side by side and
 // the re-reads of that block hit L2.
 //
-// Every mbarrier wait is bounded (globaltimer, ~2 s). A wait that runs out sets
+// Every mbarrier wait is bounded (globaltimer; the call's moe_options.wait_limit_ns,
+// 2 s by default). A wait that runs out sets
 // MOE_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag, and all roles
 // wind down: the producer waits (bounded) for its copies in flight, the MMA lane
 // waits (bounded) for its MMAs, and TMEM is freed before the CTA exits.
@@ -50,7 +51,6 @@ constexpr int BM = 128;         // weight rows per A operand (MMA M)
 constexpr int BK = 64;          // K per stage: 64 bf16 = 128 bytes = one swizzle span
 constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1025;  // routed experts (<= 1024) + the shared MLP
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Modes. kGateUp / kDown: weight rows are the MMA's M side, the expert's
 // tokens its N side (skinny experts). kGateUpTM / kDownTM ("token-major", for
@@ -81,6 +81,8 @@ struct UmmaParams {
   // router-logits mode: A = the three bf16 planes of the router weight [3E, H]
   float* logits_out;  // [ksplit, T, E] partial sums (ksplit == 1: the logits)
   int ksplit, kper, kbH;
+  uint64_t wait_ns;  // bound on every mbarrier wait
+  int withhold;      // test aid: 1 = never hand the first accumulator to the epilogue
 };
 
 // ----------------------------------------------------------------------------
@@ -89,14 +91,14 @@ struct UmmaParams {
 // Bounded wait for the phase of `bar` with the given parity. Returns false when
 // the CTA is aborting or the wait ran out (which raises the abort).
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, WsHeader* hdr,
-                                         int site) {
+                                         int site, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         record_error(hdr, MOE_ERR_TIMEOUT, site);
         return false;
@@ -106,10 +108,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
-__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kTimeoutNs) return;
+    if (globaltimer() - t0 > limit_ns) return;
 }
 
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y) {
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < t.kblocks; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_bar(&empty[s], ph ^ 1u, abort_flag, p.hdr, 1)) {
+          if (!wait_bar(&empty[s], ph ^ 1u, abort_flag, p.hdr, 1, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -438,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: the copies of the last STAGES iterations must have landed
-      for (int j = max(0, it - STAGES); j < it; ++j) drain_bar(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u);
+      for (int j = max(0, it - STAGES); j < it; ++j) drain_bar(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u, p.wait_ns);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ok && ch < t.nchunks; ++ch, ++tcount) {
           const int a = tcount & 1;
           const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
-          if (!wait_bar(&tempty[a], tph ^ 1u, abort_flag, p.hdr, 2)) {
+          if (!wait_bar(&tempty[a], tph ^ 1u, abort_flag, p.hdr, 2, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-            if (!wait_bar(&full[s], ph, abort_flag, p.hdr, 3)) {
+            if (!wait_bar(&full[s], ph, abort_flag, p.hdr, 3, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -487,11 +489,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
           }
           if (!ok) break;
-          tc_commit(&tfull[a]);  // accumulators ready for the epilogue
+          if (!(p.withhold && tcount == 0)) tc_commit(&tfull[a]);  // accumulators ready for the epilogue
         }
       }
       tc_commit(done);
-      drain_bar(done, 0);
+      drain_bar(done, 0, p.wait_ns);
     }
   } else {
     // ======================= epilogue (warps 2..5) =======================
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one lane waits, the warp follows its verdict: the TMEM loads below are
         // .sync.aligned and need the whole warp converged
         int ok = 1;
-        if (lane == 0) ok = wait_bar(&tfull[a], tph, abort_flag, p.hdr, 4) ? 1 : 0;
+        if (lane == 0) ok = wait_bar(&tfull[a], tph, abort_flag, p.hdr, 4, p.wait_ns) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         __syncwarp();
         if (!ok) {
@@ -772,6 +774,8 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   p.h_shared = static_cast<uint16_t*>(a.h_shared);
   p.y_slots = a.y_slots;
   p.shared_out = a.shared_out;
+  p.wait_ns = opt_wait_ns();
+  p.withhold = opt_withhold() == 2 ? 1 : 0;
   // maps: A routed, B routed, B2 routed, A shared, B shared, B2 shared
   CUtensorMap m[6];
 
@@ -873,6 +877,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   p.ksplit = ksplit;
   p.kper = kper;
   p.kbH = (H + BK - 1) / BK;
+  p.wait_ns = opt_wait_ns();
   CUtensorMap m[6];
   if (!make_map(&m[0], planes, 3 * (int64_t)E, H, BM) || !make_map(&m[1], x, T, H, kLogitsBN))
     return cudaErrorInvalidValue;

@@ -21,14 +21,15 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 SCORE = {"softmax": 0, "sigmoid": 1}
 KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "expert_down": 4, "combine": 5,
            "decode_fused": 6}
-FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch at or below this batch
 
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
-           "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_set_kernel_timer",
-           "moe_set_ffn_path", "moe_set_decode_kernel", "moe_launch_count", "moe_last_error", "moe_permute_static",
-           "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
+           "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_launch_count", "moe_last_error",
+           "moe_permute_static", "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
+FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch at or below this batch
+DECODE = {"auto": 0, "unfused": 1}
+WITHHOLD = {None: 0, "decode_routing": 1, "expert_accumulator": 2}
 
 
 class MoeError(RuntimeError):
@@ -65,6 +66,37 @@ def config_from_workload(wl: dict) -> MoeConfig:
     )
 
 
+class Options(ctypes.Structure):
+    """moe_options: per-call kernel choices, wait limit and timing hook."""
+    _fields_ = [
+        ("ffn_path", ctypes.c_int32),
+        ("decode_kernel", ctypes.c_int32),
+        ("wait_limit_ns", ctypes.c_uint64),
+        ("timer_kernel", ctypes.c_int32),
+        ("timer_start", ctypes.c_void_p),
+        ("timer_stop", ctypes.c_void_p),
+        ("test_withhold", ctypes.c_int32),
+    ]
+
+
+def options(ffn_path: str = "auto", decode: str = "auto", timer=None, wait_limit_ns: int = 0,
+            withhold=None) -> Options:
+    """Build a moe_options: ffn_path in FFN_PATHS, decode in DECODE, timer =
+    (kernel name, start event, stop event) or None, withhold in WITHHOLD (a
+    test aid that makes one device wait run out)."""
+    o = Options(FFN_PATHS[ffn_path], DECODE[decode], int(wait_limit_ns), -1, None, None, WITHHOLD[withhold])
+    if timer is not None:
+        name, ev0, ev1 = timer
+        o.timer_kernel = KERNELS[name]
+        o.timer_start = ev0.cuda_event
+        o.timer_stop = ev1.cuda_event
+    return o
+
+
+def _opts(o):
+    return None if o is None else ctypes.byref(o)
+
+
 class Q8Matrix(ctypes.Structure):
     """moe_q8_matrix: codes [R, K] uint8, scale and bias [R, K / group_size] bf16."""
     _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
@@ -91,6 +123,7 @@ def _load():
         raise ImportError(f"{library_path} is not built; run `python -m grouped_top_routing_b200.build`")
     L = ctypes.CDLL(library_path)
     vp, i64, sz, cfgp = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.POINTER(MoeConfig)
+    op = ctypes.POINTER(Options)
     st = ctypes.c_int
     sig = {
         "moe_workspace_size": (sz, [cfgp, i64]),
@@ -98,17 +131,15 @@ def _load():
         "moe_router_logits": (st, [cfgp, vp, i64, vp, vp, vp, sz, vp]),
         "moe_route": (st, [cfgp, vp, vp, i64, vp, vp, vp]),
         "moe_permute": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp]),
-        "moe_expert_ffn": (st, [cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_expert_ffn": (st, [cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, op]),
         "moe_combine": (st, [cfgp, i64, vp, vp, vp, vp]),
-        "moe_forward": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_forward": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, op]),
         "moe_check_device": (st, [vp, sz, vp]),
-        "moe_set_kernel_timer": (st, [ctypes.c_int32, vp, vp]),
-        "moe_set_ffn_path": (st, [ctypes.c_int32]),
-        "moe_set_decode_kernel": (st, [ctypes.c_int32]),
         "moe_permute_static": (st, [cfgp, vp, i64, vp, vp, vp, vp, vp, vp]),
         "moe_dense_mlp_workspace_size": (sz, [ctypes.c_int32, ctypes.c_int32, i64]),
-        "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp]),
-        "moe_forward_q8": (st, [cfgp, vp, i64, vp, vp, vp, ctypes.POINTER(Q8Weights), vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp, op]),
+        "moe_forward_q8": (st, [cfgp, vp, i64, vp, vp, vp, ctypes.POINTER(Q8Weights), vp, vp, vp, vp, vp, vp, sz, vp,
+                                op]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -179,65 +210,6 @@ class Workspace:
         _check(lib.moe_check_device(self.cptr, self.nbytes, _stream(stream)))
 
 
-def moe_router_logits(cfg, x, router_w, ws: "Workspace", out=None, stream=None):
-    c = _as_cfg(cfg)
-    T = x.shape[0]
-    if out is None:
-        out = torch.empty((T, c.num_experts), dtype=torch.float32, device=x.device)
-    _check(lib.moe_router_logits(ctypes.byref(c), _p(x), T, _p(router_w), _p(out), ws.cptr, ws.nbytes,
-                                 _stream(stream)))
-    return out
-
-
-def moe_route(cfg, logits, expert_bias=None, topk_idx=None, topk_w=None, stream=None):
-    c = _as_cfg(cfg)
-    T = logits.shape[0]
-    k = c.num_experts_per_tok
-    if topk_idx is None:
-        topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
-    if topk_w is None:
-        topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    _check(lib.moe_route(ctypes.byref(c), _p(logits), _p(expert_bias), T, _p(topk_idx), _p(topk_w), _stream(stream)))
-    return topk_idx, topk_w
-
-
-def moe_permute(cfg, topk_idx, ws: Workspace, x=None, want_x_perm=False, stream=None):
-    c = _as_cfg(cfg)
-    T = topk_idx.shape[0]
-    k, E, H = c.num_experts_per_tok, c.num_experts, c.hidden_size
-    dev = topk_idx.device
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
-    tok_of = torch.empty(T * k, dtype=torch.int32, device=dev)
-    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev) if want_x_perm else None
-    _check(lib.moe_permute(ctypes.byref(c), _p(topk_idx), T, _p(x), _p(offsets), _p(row_of), _p(tok_of), _p(x_perm),
-                           ws.cptr, ws.nbytes, _stream(stream)))
-    return offsets, row_of, tok_of, x_perm
-
-
-def moe_expert_ffn(cfg, x, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws: Workspace, ws_gate_up=None,
-                   ws_down=None, x_perm=None, y_slots=None, shared_out=None, stream=None):
-    c = _as_cfg(cfg)
-    T = x.shape[0]
-    k, H = c.num_experts_per_tok, c.hidden_size
-    if y_slots is None:
-        y_slots = torch.empty((T * k, H), dtype=torch.float32, device=x.device)
-    if ws_gate_up is not None and shared_out is None:
-        shared_out = torch.empty((T, H), dtype=torch.float32, device=x.device)
-    _check(lib.moe_expert_ffn(ctypes.byref(c), T, _p(x), _p(x_perm), _p(expert_offsets), _p(tok_of), _p(topk_w),
-                              _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y_slots), _p(shared_out),
-                              ws.cptr, ws.nbytes, _stream(stream)))
-    return y_slots, shared_out
-
-
-def moe_combine(cfg, y_slots, shared_out, T: int, y=None, stream=None):
-    c = _as_cfg(cfg)
-    if y is None:
-        y = torch.empty((T, c.hidden_size), dtype=torch.bfloat16, device=y_slots.device)
-    _check(lib.moe_combine(ctypes.byref(c), T, _p(y_slots), _p(shared_out), _p(y), _stream(stream)))
-    return y
-
-
 def shared_width(c: MoeConfig) -> int:
     """Width of the shared MLP as the library derives it from the config."""
     if c.num_shared_experts <= 0:
@@ -248,17 +220,40 @@ def shared_width(c: MoeConfig) -> int:
 
 def _require(t, name: str, numel: int, dtype):
     """The C ABI sees raw pointers only: a tensor smaller than the config says
-    would be read past its end on the device, so check sizes here."""
+    would be read or written past its end on the device. Check size, dtype and
+    layout here, before any launch (the device is checked by _on_device once
+    every size has passed)."""
     if t is None:
         return
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name}: expected a torch tensor, got {type(t).__name__}")
     if t.numel() != numel or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name}: expected {numel} contiguous {dtype} elements for this config, got "
                          f"{tuple(t.shape)} {t.dtype}{'' if t.is_contiguous() else ' (not contiguous)'}")
 
 
+def _on_device(dev, **tensors):
+    """A host tensor, or one on another GPU, would be dereferenced as a device
+    address of the call's GPU: refuse it before any launch."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+        if t.device != dev:
+            raise ValueError(f"{name}: on {t.device}, but the call runs on {dev}")
+
+
+def _rows(t, name: str):
+    if not isinstance(t, torch.Tensor) or t.dim() < 1:
+        raise ValueError(f"{name}: expected a tensor with a leading token dimension")
+    return int(t.shape[0])
+
+
 def _check_block_tensors(c: MoeConfig, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down,
-                         ws_gate_up, ws_down):
+                         ws_gate_up, ws_down, y=None):
     E, H, I, Is = c.num_experts, c.hidden_size, c.moe_intermediate_size, shared_width(c)
+    dev = x.device
     _require(x, "x", T * H, torch.bfloat16)
     _require(router_w, "router_w", E * H, torch.float32)
     _require(expert_bias, "expert_bias", E, torch.float32)
@@ -267,14 +262,124 @@ def _check_block_tensors(c: MoeConfig, T, x, router_w, expert_bias, logits_overr
     _require(w_down, "w_down", E * H * I, torch.bfloat16)
     _require(ws_gate_up, "ws_gate_up", 2 * Is * H, torch.bfloat16)
     _require(ws_down, "ws_down", H * Is, torch.bfloat16)
+    _require(y, "y", T * H, torch.bfloat16)
+    _on_device(x.device, x=x, router_w=router_w, expert_bias=expert_bias, logits_override=logits_override,
+               w_gate_up=w_gate_up, w_down=w_down, ws_gate_up=ws_gate_up, ws_down=ws_down, y=y)
+
+
+def _check_ws(ws, dev):
+    if not isinstance(ws, Workspace):
+        raise ValueError("ws: expected a Workspace")
+    if ws.buf.device != dev:
+        raise ValueError(f"workspace: on {ws.buf.device}, but the call runs on {dev}")
+
+
+def moe_router_logits(cfg, x, router_w, ws: "Workspace", out=None, stream=None):
+    c = _as_cfg(cfg)
+    T = _rows(x, "x")
+    dev = x.device
+    _require(x, "x", T * c.hidden_size, torch.bfloat16)
+    _require(router_w, "router_w", c.num_experts * c.hidden_size, torch.float32)
+    _require(out, "logits", T * c.num_experts, torch.float32)
+    _on_device(dev, x=x, router_w=router_w, logits=out)
+    _check_ws(ws, dev)
+    if out is None:
+        out = torch.empty((T, c.num_experts), dtype=torch.float32, device=dev)
+    _check(lib.moe_router_logits(ctypes.byref(c), _p(x), T, _p(router_w), _p(out), ws.cptr, ws.nbytes,
+                                 _stream(stream)))
+    return out
+
+
+def moe_route(cfg, logits, expert_bias=None, topk_idx=None, topk_w=None, stream=None):
+    c = _as_cfg(cfg)
+    T = _rows(logits, "logits")
+    k, E = c.num_experts_per_tok, c.num_experts
+    dev = logits.device
+    _require(logits, "logits", T * E, torch.float32)
+    _require(expert_bias, "expert_bias", E, torch.float32)
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    _require(topk_idx, "topk_idx", T * k, torch.int32)
+    _require(topk_w, "topk_w", T * k, torch.float32)
+    _on_device(dev, logits=logits, expert_bias=expert_bias, topk_idx=topk_idx, topk_w=topk_w)
+    _check(lib.moe_route(ctypes.byref(c), _p(logits), _p(expert_bias), T, _p(topk_idx), _p(topk_w), _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_permute(cfg, topk_idx, ws: Workspace, x=None, want_x_perm=False, stream=None):
+    c = _as_cfg(cfg)
+    T = _rows(topk_idx, "topk_idx")
+    k, E, H = c.num_experts_per_tok, c.num_experts, c.hidden_size
+    dev = topk_idx.device
+    _require(topk_idx, "topk_idx", T * k, torch.int32)
+    _require(x, "x", T * H, torch.bfloat16)
+    if want_x_perm and x is None:
+        raise ValueError("x_perm needs x")
+    _on_device(dev, topk_idx=topk_idx, x=x)
+    _check_ws(ws, dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tok_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev) if want_x_perm else None
+    _check(lib.moe_permute(ctypes.byref(c), _p(topk_idx), T, _p(x), _p(offsets), _p(row_of), _p(tok_of), _p(x_perm),
+                           ws.cptr, ws.nbytes, _stream(stream)))
+    return offsets, row_of, tok_of, x_perm
+
+
+def moe_expert_ffn(cfg, x, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws: Workspace, ws_gate_up=None,
+                   ws_down=None, x_perm=None, y_slots=None, shared_out=None, stream=None, opts: Options | None = None):
+    c = _as_cfg(cfg)
+    T = _rows(x, "x")
+    k, H, E, I, Is = c.num_experts_per_tok, c.hidden_size, c.num_experts, c.moe_intermediate_size, shared_width(c)
+    dev = x.device
+    _require(x, "x", T * H, torch.bfloat16)
+    _require(x_perm, "x_perm", T * k * H, torch.bfloat16)
+    _require(expert_offsets, "expert_offsets", E + 1, torch.int32)
+    _require(tok_of, "tok_of", T * k, torch.int32)
+    _require(topk_w, "topk_w", T * k, torch.float32)
+    _require(w_gate_up, "w_gate_up", E * 2 * I * H, torch.bfloat16)
+    _require(w_down, "w_down", E * H * I, torch.bfloat16)
+    _require(ws_gate_up, "ws_gate_up", 2 * Is * H, torch.bfloat16)
+    _require(ws_down, "ws_down", H * Is, torch.bfloat16)
+    _require(y_slots, "y_slots", T * k * H, torch.float32)
+    _require(shared_out, "shared_out", T * H, torch.float32)
+    _on_device(dev, x=x, x_perm=x_perm, expert_offsets=expert_offsets, tok_of=tok_of, topk_w=topk_w,
+               w_gate_up=w_gate_up, w_down=w_down, ws_gate_up=ws_gate_up, ws_down=ws_down, y_slots=y_slots,
+               shared_out=shared_out)
+    _check_ws(ws, dev)
+    if y_slots is None:
+        y_slots = torch.empty((T * k, H), dtype=torch.float32, device=dev)
+    if ws_gate_up is not None and shared_out is None:
+        shared_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    _check(lib.moe_expert_ffn(ctypes.byref(c), T, _p(x), _p(x_perm), _p(expert_offsets), _p(tok_of), _p(topk_w),
+                              _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y_slots), _p(shared_out),
+                              ws.cptr, ws.nbytes, _stream(stream), _opts(opts)))
+    return y_slots, shared_out
+
+
+def moe_combine(cfg, y_slots, shared_out, T: int, y=None, stream=None):
+    c = _as_cfg(cfg)
+    k, H = c.num_experts_per_tok, c.hidden_size
+    dev = y_slots.device
+    _require(y_slots, "y_slots", T * k * H, torch.float32)
+    _require(shared_out, "shared_out", T * H, torch.float32)
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    _require(y, "y", T * H, torch.bfloat16)
+    _on_device(dev, y_slots=y_slots, shared_out=shared_out, y=y)
+    _check(lib.moe_combine(ctypes.byref(c), T, _p(y_slots), _p(shared_out), _p(y), _stream(stream)))
+    return y
 
 
 def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws_down, ws: Workspace,
-                logits_override=None, y=None, return_routing=False, stream=None):
+                logits_override=None, y=None, return_routing=False, stream=None, opts: Options | None = None):
     c = _as_cfg(cfg)
-    T = x.shape[0]
+    T = _rows(x, "x")
     k = c.num_experts_per_tok
-    _check_block_tensors(c, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down, ws_gate_up, ws_down)
+    _check_block_tensors(c, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down, ws_gate_up, ws_down, y)
+    _check_ws(ws, x.device)
     if y is None:
         y = torch.empty_like(x)
     idx = w = None
@@ -283,33 +388,14 @@ def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws
         w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     _check(lib.moe_forward(ctypes.byref(c), _p(x), T, _p(router_w), _p(expert_bias), _p(logits_override),
                            _p(w_gate_up), _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y), _p(idx), _p(w),
-                           ws.cptr, ws.nbytes, _stream(stream)))
+                           ws.cptr, ws.nbytes, _stream(stream), _opts(opts)))
     if return_routing:
         return y, idx, w
     return y
 
 
-def set_ffn_path(path: str = "auto"):
-    """Expert-FFN kernels for later calls: "auto", "streaming" or "tensor_cores"."""
-    _check(lib.moe_set_ffn_path(FFN_PATHS[path]))
-
-
-DECODE_KERNELS = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
-
-
-def set_decode_kernel(which: str = "auto"):
-    """Fused decode kernel for later calls: "auto" (the CUDA-core kernel),
-    "cuda_cores", or "tensor_cores" (where its shapes fit)."""
-    _check(lib.moe_set_decode_kernel(DECODE_KERNELS[which]))
-
-
-def set_kernel_timer(kernel: str, ev_start=None, ev_stop=None):
-    a = ctypes.c_void_p(ev_start.cuda_event) if ev_start is not None else None
-    b = ctypes.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
-    _check(lib.moe_set_kernel_timer(KERNELS[kernel], a, b))
-
-
 def launch_count() -> int:
+    """Kernel launches this library made from the calling thread."""
     return int(lib.moe_launch_count())
 
 
@@ -321,34 +407,83 @@ def dense_mlp_workspace(hidden_size: int, intermediate_size: int, max_tokens: in
     return Workspace(None, max_tokens, device=device, nbytes=n)
 
 
-def moe_dense_mlp(x, w_gate_up, w_down, ws: Workspace, y=None, stream=None):
+def moe_dense_mlp(x, w_gate_up, w_down, ws: Workspace, y=None, stream=None, opts: Options | None = None):
     """Dense-prefix SwiGLU MLP: w_gate_up [2*Id, H] (gate rows first), w_down [H, Id]."""
-    T, H = x.shape
-    Id = w_down.shape[1]
+    T = _rows(x, "x")
+    if x.dim() != 2 or w_down.dim() != 2:
+        raise ValueError("x [T, H] and w_down [H, Id] must be 2-D")
+    H = int(x.shape[1])
+    Id = int(w_down.shape[1])
+    dev = x.device
+    _require(x, "x", T * H, torch.bfloat16)
+    _require(w_gate_up, "w_gate_up", 2 * Id * H, torch.bfloat16)
+    _require(w_down, "w_down", H * Id, torch.bfloat16)
+    _require(y, "y", T * H, torch.bfloat16)
+    _on_device(dev, x=x, w_gate_up=w_gate_up, w_down=w_down, y=y)
+    _check_ws(ws, dev)
     if y is None:
         y = torch.empty_like(x)
     _check(lib.moe_dense_mlp(int(H), int(Id), _p(x), T, _p(w_gate_up), _p(w_down), _p(y), ws.cptr, ws.nbytes,
-                             _stream(stream)))
+                             _stream(stream), _opts(opts)))
     return y
 
 
+def _check_q8(c: MoeConfig, q8: dict, dev):
+    g = int(q8["group_size"])
+    E, H, I, Is = c.num_experts, c.hidden_size, c.moe_intermediate_size, shared_width(c)
+    if g <= 0 or H % g or I % g:
+        raise ValueError(f"group_size {g} must divide hidden_size {H} and moe_intermediate_size {I}")
+
+    def mat(t, name, R, K):
+        if t is None:
+            return
+        q, sc, bi = t
+        _require(q, f"{name}.q", R * K, torch.uint8)
+        _require(sc, f"{name}.scale", R * (K // g), torch.bfloat16)
+        _require(bi, f"{name}.bias", R * (K // g), torch.bfloat16)
+    mat(q8["gate_up"], "gate_up", E * 2 * I, H)
+    mat(q8["down"], "down", E * H, I)
+    if q8.get("shared_gate_up") is not None:
+        if Is % g:
+            raise ValueError(f"group_size {g} must divide the shared MLP width {Is}")
+        mat(q8["shared_gate_up"], "shared_gate_up", 2 * Is, H)
+        mat(q8.get("shared_down"), "shared_down", H, Is)
+
+
 def moe_forward_q8(cfg, x, router_w, expert_bias, q8: dict, ws: Workspace, ws_gate_up=None, ws_down=None,
-                   logits_override=None, y=None, return_routing=False, stream=None):
+                   logits_override=None, y=None, return_routing=False, stream=None, opts: Options | None = None):
     """The block with 8-bit affine expert weights (q8 as in inputs.make_q8_weights);
     the shared MLP is q8's when present, else the bf16 ws_gate_up / ws_down."""
     c = _as_cfg(cfg)
-    T = x.shape[0]
-    k = c.num_experts_per_tok
+    T = _rows(x, "x")
+    k, E, H = c.num_experts_per_tok, c.num_experts, c.hidden_size
+    Is = shared_width(c)
+    dev = x.device
+    _require(x, "x", T * H, torch.bfloat16)
+    _require(router_w, "router_w", E * H, torch.float32)
+    _require(expert_bias, "expert_bias", E, torch.float32)
+    _require(logits_override, "logits_override", T * E, torch.float32)
+    _require(ws_gate_up, "ws_gate_up", 2 * Is * H, torch.bfloat16)
+    _require(ws_down, "ws_down", H * Is, torch.bfloat16)
+    _check_q8(c, q8, dev)
+    _require(y, "y", T * H, torch.bfloat16)
+    _on_device(dev, x=x, router_w=router_w, expert_bias=expert_bias, logits_override=logits_override,
+               ws_gate_up=ws_gate_up, ws_down=ws_down, y=y)
+    for key in ("gate_up", "down", "shared_gate_up", "shared_down"):
+        if q8.get(key) is not None:
+            q, sc, bi = q8[key]
+            _on_device(dev, **{f"{key}.q": q, f"{key}.scale": sc, f"{key}.bias": bi})
+    _check_ws(ws, dev)
     if y is None:
         y = torch.empty_like(x)
     idx = w = None
     if return_routing:
-        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
-        w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
     qw = q8_weights(q8)
     _check(lib.moe_forward_q8(ctypes.byref(c), _p(x), T, _p(router_w), _p(expert_bias), _p(logits_override),
                               ctypes.byref(qw), _p(ws_gate_up), _p(ws_down), _p(y), _p(idx), _p(w), ws.cptr,
-                              ws.nbytes, _stream(stream)))
+                              ws.nbytes, _stream(stream), _opts(opts)))
     if return_routing:
         return y, idx, w
     return y

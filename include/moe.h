@@ -43,8 +43,10 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *     is the legacy default stream). They return once the work is enqueued.
  *   - The caller owns every buffer. The library allocates no device memory and
- *     keeps no state beyond a per-device attribute cache, per-thread error text
- *     and the measurement hooks of moe_set_kernel_timer.
+ *     keeps no state between calls beyond a per-device attribute cache (SM
+ *     count, the address of moe_permute_static's scratch array) and per-thread
+ *     error text and launch count. Kernel choices, wait limits and timing hooks
+ *     travel with each call in a moe_options struct (NULL: the defaults).
  *   - All arguments are validated on the host BEFORE any launch. A rejected call
  *     launches nothing and returns a status; the library never aborts or throws
  *     across this ABI ([DEFENSE]). moe_last_error() names the offending field.
@@ -103,7 +105,7 @@ typedef struct {
   int32_t moe_shared_expert_intermediate_size; /* 0 = use I ([SHARED]) */
 } moe_config;
 
-/* Kernels that moe_set_kernel_timer can bracket. */
+/* Kernels that moe_options.timer_kernel can bracket. */
 typedef enum {
   MOE_KERNEL_ROUTER_LOGITS = 0,
   MOE_KERNEL_ROUTE = 1,
@@ -111,9 +113,38 @@ typedef enum {
   MOE_KERNEL_EXPERT_GATE_UP = 3, /* routed + shared gate/up projections with SwiGLU */
   MOE_KERNEL_EXPERT_DOWN = 4,    /* routed + shared down projections, weighted */
   MOE_KERNEL_COMBINE = 5,
-  MOE_KERNEL_DECODE_FUSED = 6,   /* the whole block for 1-2 tokens in one launch (moe_forward) */
+  MOE_KERNEL_DECODE_FUSED = 6,   /* the whole block for a few tokens in one launch (moe_forward) */
   MOE_KERNEL_COUNT = 7
 } moe_kernel_id;
+
+/* Per-call options of moe_expert_ffn, moe_forward, moe_forward_q8 and
+ * moe_dense_mlp. Pass NULL for the defaults; a zero-initialised struct with
+ * timer_kernel = -1 is the same. The library reads the struct during the call
+ * only and keeps no pointer to it. */
+typedef struct {
+  int32_t ffn_path;       /* expert kernels: 0 automatic (the streaming GEMV for
+                             T <= 2 tokens when the block is not fused, the
+                             tensor-core grouped GEMM above), 1 always the
+                             streaming GEMV, 2 always the tensor-core GEMM */
+  int32_t decode_kernel;  /* moe_forward on a few tokens: 0 automatic (one fused
+                             launch where the shapes allow it), 1 never fused
+                             (the separate kernels of the larger batches) */
+  uint64_t wait_limit_ns; /* bound on every device-side wait of the call's
+                             kernels; 0 = the default of 2 s. A wait that runs
+                             out records MOE_ERR_TIMEOUT and the kernel returns. */
+  int32_t timer_kernel;   /* moe_kernel_id whose launches in this call are
+                             bracketed by the two events, or -1 for none */
+  void* timer_start;      /* cudaEvent_t recorded just before each such launch */
+  void* timer_stop;       /* cudaEvent_t recorded just after it */
+  int32_t test_withhold;  /* test aid, 0 in normal use. 1: the fused decode
+                             kernel withholds the release of its routing, so
+                             every wait for it runs out; 2: the tensor-core
+                             expert kernel withholds its first accumulator
+                             hand-over, so the epilogue's wait runs out. Both
+                             end in MOE_ERR_TIMEOUT after wait_limit_ns and
+                             leave the workspace usable once moe_check_device
+                             has reported. Any other value is rejected. */
+} moe_options;
 
 /* Workspace bytes moe_permute, moe_expert_ffn and moe_forward need for up to
  * max_tokens tokens. Returns 0 (and sets moe_last_error) on an invalid config.
@@ -182,7 +213,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, c
                           const uint16_t* w_gate_up, const uint16_t* w_down,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down,
                           float* y_slots, float* shared_out,
-                          void* ws, size_t ws_bytes, void* stream);
+                          void* ws, size_t ws_bytes, void* stream, const moe_options* opts);
 
 /* Weighted combine ([ROUTER], [SHARED]: out = routed mixture + shared(x)):
  *   y[t] = bf16( sum_{j<k} y_slots[t*k + j] + shared_out[t] ),
@@ -193,29 +224,25 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
                        uint16_t* y, void* stream);
 
 /* The whole block: router logits -> route -> permute -> experts -> combine.
- * With the automatic expert path (moe_set_ffn_path(0)), T <= 2 tokens, at most
- * 32 slots (T*k), E <= 1024 and H <= 8192, the block runs as one cooperative
- * launch (MOE_KERNEL_DECODE_FUSED): a weight-streaming kernel, one CTA per SM,
- * with one bounded grid barrier and bounded per-expert and per-row counters.
- * The kernel multiplies on the CUDA cores (fp32 sums throughout). A variant
- * on the tensor cores (mma.sync, bf16 in, fp32 sums, h kept as two bf16
- * planes as on the tensor-core expert path) takes H a multiple of 512 up to
- * 4096 and expert and shared widths multiples of 64 up to 512 ([GGUF]
- * shapes); moe_set_decode_kernel selects it.
+ * With opts->decode_kernel = 0 (the default), T <= 2 tokens, at most 32 slots
+ * (T*k), E <= 1024 and H <= 8192, the block runs as one cooperative launch
+ * (MOE_KERNEL_DECODE_FUSED): a weight-streaming kernel, one CTA per SM, with
+ * one bounded grid barrier and bounded per-expert and per-row counters, that
+ * multiplies on the CUDA cores (fp32 sums throughout).
  * Its routing (indices and weights) is bit-identical to moe_route on the same
  * logits; its logits and output equal those of the separate kernels up to the
- * fp32 summation order of the dot products (and the 16-bit h planes of the
- * tensor-core variant).
+ * fp32 summation order of the dot products.
  *   logits_override [T,E] fp32 or NULL: when given, replaces the router
  *   projection (router_w may then be NULL).
  *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
- *   routing. y [T,H] bf16 out. ws / ws_bytes >= moe_workspace_size(cfg, T). */
+ *   routing. y [T,H] bf16 out. ws / ws_bytes >= moe_workspace_size(cfg, T).
+ *   opts: per-call options or NULL. */
 moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
                        const float* expert_bias, const float* logits_override,
                        const uint16_t* w_gate_up, const uint16_t* w_down,
                        const uint16_t* ws_gate_up, const uint16_t* ws_down,
                        uint16_t* y, int32_t* topk_idx_out, float* topk_w_out,
-                       void* ws, size_t ws_bytes, void* stream);
+                       void* ws, size_t ws_bytes, void* stream, const moe_options* opts);
 
 /* The dense-prefix MLP ([DENSE]): y = W_down (silu(W_gate x) * (W_up x)), bf16
  * in and out, fp32 accumulation, on the expert kernels of moe_expert_ffn (the
@@ -227,7 +254,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
 size_t moe_dense_mlp_workspace_size(int32_t hidden_size, int32_t intermediate_size, int64_t max_tokens);
 moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const uint16_t* x, int64_t T,
                          const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* y,
-                         void* ws, size_t ws_bytes, void* stream);
+                         void* ws, size_t ws_bytes, void* stream, const moe_options* opts);
 
 /* 8-bit affine weights ([Q8]): for each row and each group of `group_size`
  * consecutive inputs, w = scale * q + bias, with q uint8 and scale, bias bf16
@@ -256,7 +283,8 @@ typedef struct {
 moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
                           const float* expert_bias, const float* logits_override, const moe_q8_weights* w,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y,
-                          int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+                          int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream,
+                          const moe_options* opts);
 
 /* Synchronises `stream`, reads and clears the workspace error word (after an
  * error the whole 256-byte header is cleared, barrier state included). Returns
@@ -264,27 +292,8 @@ moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, c
  * MOE_ERR_CUDA if the stream itself reports an error. Blocking. */
 moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
 
-/* Measurement aid. While set, every launch of kernel `which` is bracketed by
- * cudaEventRecord(ev_start) / cudaEventRecord(ev_stop) on its launch stream
- * (events are cudaEvent_t passed as void*; the caller owns them). Passing NULL
- * events clears the hook. Not thread-safe with concurrent launches. */
-moe_status moe_set_kernel_timer(int32_t which, void* ev_start, void* ev_stop);
-
-/* Selects the expert-FFN kernels for every later call in this process:
- * 0 = automatic (the streaming GEMV for T <= 2 tokens, where each expert's
- * weights are streamed once over all SMs; the tensor-core grouped GEMM above),
- * 1 = always the streaming GEMV, 2 = always the tensor-core grouped GEMM.
- * Both compute the same block. */
-moe_status moe_set_ffn_path(int32_t path);
-
-/* Selects the fused decode kernel of moe_forward for every later call in this
- * process: 0 = automatic (the CUDA-core kernel, measured the faster of the two
- * at Ling-3.0-flash decode shapes), 1 = the CUDA-core kernel, 2 = the
- * tensor-core kernel where its shapes fit (else the CUDA-core one). Both
- * compute the same block. Any other value: MOE_ERR_INVALID_ARG. */
-moe_status moe_set_decode_kernel(int32_t which);
-
-/* Number of this library's kernel launches since load (host-side counter). */
+/* Number of this library's kernel launches made by the calling thread since
+ * the library was loaded (a host-side counter). */
 uint64_t moe_launch_count(void);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
@@ -297,7 +306,10 @@ uint64_t moe_launch_count(void);
  *   MOE_ERR_UNSUPPORTED (about 65k tokens at E = 256, 16k at E = 1024; any T
  *   <= 128). The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture. The address is then cached for the life of
+ *   the process: it does not survive cudaDeviceReset (or the destruction of
+ *   the device's primary context), after which this function must not be
+ *   called on that device again.
  *   Calls share the array: two calls whose work overlaps on the GPU (other
  *   streams, other threads, other devices' calls are fine) race and corrupt
  *   each other's results. Each call clears what must start at zero.

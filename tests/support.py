@@ -64,6 +64,14 @@ def check_ties_constructed(L, bias, wl, toks, pairs):
     return idx
 
 
+def near_tie_bound(T: int, constructed: int = 0) -> int:
+    """Most near-tie tokens a workload of T random tokens may hold: the gap
+    between the k-th and (k+1)-th biased score falls under 1e-6 about once in
+    a few thousand tokens on these workloads (counted on the oracle: 2 of 8192
+    and 1 of 16384). ``constructed`` adds tokens built as exact ties."""
+    return 4 + T // 1000 + constructed
+
+
 def near_tie_tokens(L, bias, wl):
     s = O.scores(L, wl["score_function"])
     _, sel = O.select_experts(s, bias, wl["num_experts_per_tok"], wl.get("n_group", 1), wl.get("topk_group", 1),

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from grouped_top_routing_b200 import build as B
 
@@ -88,7 +89,7 @@ def test_invalid_config_rejected(M, field, over, status):
     for call in (
         lambda: M.lib.moe_route(ctypes.byref(c), fake, None, 4, fake, fake, None),
         lambda: M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None,
-                                  None, fake, 1 << 40, None),
+                                  None, fake, 1 << 40, None, None),
         lambda: M.lib.moe_combine(ctypes.byref(c), 4, fake, None, fake, None),
     ):
         st = call()
@@ -141,17 +142,17 @@ def test_null_and_misaligned_pointers_rejected(M):
     ws_need = M.lib.moe_workspace_size(ctypes.byref(c), 4)
     # forward: router weight required unless logits are given
     st = M.lib.moe_forward(ctypes.byref(c), fake, 4, None, None, None, fake, fake, fake, fake, fake, None, None, fake,
-                           ws_need, None)
+                           ws_need, None, None)
     assert st == 1 and "router_w" in M.last_error()
     # shared weights required when the config has a shared MLP
     st = M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, None, None, fake, None, None, fake,
-                           ws_need, None)
+                           ws_need, None, None)
     assert st == 1 and "ws_gate_up" in M.last_error()
     # and rejected when it has none
     c0 = _cfg(M, num_shared_experts=0)
     ws0 = M.lib.moe_workspace_size(ctypes.byref(c0), 4)
     st = M.lib.moe_forward(ctypes.byref(c0), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None, None, fake,
-                           ws0, None)
+                           ws0, None, None)
     assert st == 1 and "shared" in M.last_error()
 
 
@@ -169,19 +170,39 @@ def test_workspace_rejected(M):
     assert M.lib.moe_workspace_init(None, 0, None) == 3
 
 
-def test_kernel_timer_arguments(M):
-    assert M.lib.moe_set_kernel_timer(99, None, None) == 1
-    assert M.lib.moe_set_kernel_timer(0, ctypes.c_void_p(8), None) == 1
-    assert M.lib.moe_set_kernel_timer(0, None, None) == 0
+OPTION_BAD = [
+    # field, value, text in the message
+    ("ffn_path", 3, "ffn_path"),
+    ("ffn_path", -1, "ffn_path"),
+    ("decode_kernel", 2, "decode_kernel"),
+    ("timer_kernel", 99, "timer_kernel"),
+    ("timer_kernel", -2, "timer_kernel"),
+    ("timer_kernel", 0, "timer events"),   # a kernel id without its events
+    ("test_withhold", 3, "test_withhold"),
+]
 
 
-def test_path_selectors_reject_unknown_values(M):
-    assert M.lib.moe_set_ffn_path(3) == 1 and M.lib.moe_set_ffn_path(-1) == 1
-    assert M.lib.moe_set_decode_kernel(3) == 1 and "not 0 (auto), 1 (CUDA cores) or 2" in M.last_error()
-    assert M.lib.moe_set_decode_kernel(-1) == 1
-    for which in (1, 2, 0):
-        assert M.lib.moe_set_decode_kernel(which) == 0
-    assert M.lib.moe_set_ffn_path(0) == 0
+@pytest.mark.parametrize("field,value,text", OPTION_BAD, ids=[f"{f}={v}" for f, v, _ in OPTION_BAD])
+def test_options_rejected_before_launch(M, field, value, text):
+    # Per-call options are validated before anything else; a bad one launches nothing.
+    c = _cfg(M)
+    fake = ctypes.c_void_p(1 << 20)
+    o = M.options()
+    setattr(o, field, value)
+    n0 = M.lib.moe_launch_count()
+    st = M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None, None,
+                           fake, 1 << 40, None, ctypes.byref(o))
+    assert st == 1 and text in M.last_error(), (st, M.last_error())
+    st = M.lib.moe_dense_mlp(4096, 9216, fake, 4, fake, fake, fake, fake, 1 << 40, None, ctypes.byref(o))
+    assert st == 1 and text in M.last_error()
+    assert M.lib.moe_launch_count() == n0
+
+
+def test_options_defaults(M):
+    o = M.options()
+    assert (o.ffn_path, o.decode_kernel, o.wait_limit_ns, o.timer_kernel, o.test_withhold) == (0, 0, 0, -1, 0)
+    o = M.options("tensor_cores", "unfused", wait_limit_ns=1000, withhold="expert_accumulator")
+    assert (o.ffn_path, o.decode_kernel, o.wait_limit_ns, o.test_withhold) == (2, 1, 1000, 2)
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
@@ -215,7 +236,7 @@ def test_dense_mlp_rejects_before_launch(M, H, Id, T, with_ws, status, field):
     fake = ctypes.c_void_p(1 << 20)
     ws = fake if with_ws else None
     n0 = M.lib.moe_launch_count()
-    st = M.lib.moe_dense_mlp(H, Id, fake, T, fake, fake, fake, ws, 1 << 40, None)
+    st = M.lib.moe_dense_mlp(H, Id, fake, T, fake, fake, fake, ws, 1 << 40, None, None)
     assert st == status, (st, M.last_error())
     assert field in M.last_error()
     assert M.lib.moe_launch_count() == n0
@@ -257,7 +278,7 @@ def test_forward_q8_rejects_before_launch(M, what, wargs, bf16_shared, status, t
     n0 = M.lib.moe_launch_count()
     st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, ctypes.byref(w),
                               fake if bf16_shared else None, fake if bf16_shared else None, fake, None, None,
-                              fake, 1 << 40, None)
+                              fake, 1 << 40, None, None)
     assert st == status, (st, M.last_error())
     assert text in M.last_error(), M.last_error()
     assert M.lib.moe_launch_count() == n0
@@ -267,7 +288,7 @@ def test_forward_q8_rejects_null_weights(M):
     c = _cfg(M)
     fake = ctypes.c_void_p(1 << 20)
     st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, None, None, None, fake, None, None,
-                              fake, 1 << 40, None)
+                              fake, 1 << 40, None, None)
     assert st == 1 and "NULL" in M.last_error()
 
 
@@ -279,10 +300,13 @@ def test_binding_checks_tensor_sizes_against_the_config(M):
     inp = G.make_inputs(wl, seed=0, device="cpu")
     args = dict(x=inp["x"], router_w=inp["router_w"], expert_bias=inp["expert_bias"], w_gate_up=inp["w_gate_up"],
                 w_down=inp["w_down"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"])
-    for name in ("router_w", "w_gate_up", "w_down", "ws_gate_up", "ws_down"):
-        bad = dict(args, **{name: args[name].reshape(-1)[:-8]})
+    args["expert_bias"] = torch.zeros(wl["num_experts"])
+    for name in ("router_w", "w_gate_up", "w_down", "ws_gate_up", "ws_down", "expert_bias"):
+        bad = dict(args, **{name: args[name].reshape(-1)[:-1]})
         with pytest.raises(ValueError, match=name):
             M.moe_forward(wl, ws=None, **bad)
+    with pytest.raises(ValueError, match="y:"):  # a caller-supplied output is checked too
+        M.moe_forward(wl, ws=None, y=torch.empty(3, 64, dtype=torch.bfloat16), **args)
     # a shared MLP wider than the config says (the width the library derives is
     # moe_intermediate_size x num_shared_experts)
     wide = G.make_inputs(dict(wl, shared_width=64), seed=0, device="cpu")
@@ -291,3 +315,59 @@ def test_binding_checks_tensor_sizes_against_the_config(M):
     assert M.shared_width(M.config_from_workload(wl)) == 32
     assert M.shared_width(M.config_from_workload(dict(wl, num_shared_experts=2))) == 64
     assert M.shared_width(M.config_from_workload(dict(wl, num_shared_experts=0))) == 0
+
+
+def test_binding_rejects_host_tensors(M):
+    # Right sizes but host memory: the kernels would dereference a host address
+    # as a device one, so the binding refuses before any launch.
+    from grouped_top_routing_b200 import inputs as G
+    wl = G.tiny_workload(tokens=2, hidden_size=64, moe_intermediate_size=32, shared_width=32)
+    inp = G.make_inputs(wl, seed=0, device="cpu")
+    n0 = M.launch_count()
+    with pytest.raises(ValueError, match="CUDA"):
+        M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                      inp["ws_gate_up"], inp["ws_down"], ws=None)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.moe_route(wl, torch.zeros(2, wl["num_experts"]))
+    assert M.launch_count() == n0
+
+
+def test_component_wrappers_check_sizes(M):
+    # Every component wrapper checks what it hands the C ABI (size first, so
+    # these run on the host without a device).
+    from grouped_top_routing_b200 import inputs as G
+    wl = G.tiny_workload(tokens=4, hidden_size=64, num_experts=8, num_experts_per_tok=2, moe_intermediate_size=32,
+                         shared_width=32)
+    T, E, k, H = 4, 8, 2, 64
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    with pytest.raises(ValueError, match="logits"):
+        M.moe_route(wl, torch.zeros(T, E - 1))
+    with pytest.raises(ValueError, match="expert_bias"):
+        M.moe_route(wl, torch.zeros(T, E), torch.zeros(E + 1))
+    with pytest.raises(ValueError, match="topk_idx"):
+        M.moe_route(wl, torch.zeros(T, E), topk_idx=torch.zeros(T, k + 1, dtype=i32))
+    with pytest.raises(ValueError, match="topk_idx"):
+        M.moe_permute(wl, torch.zeros(T, k, dtype=torch.int64), ws=None)
+    with pytest.raises(ValueError, match="x:"):
+        M.moe_permute(wl, torch.zeros(T, k, dtype=i32), ws=None, x=torch.zeros(T, H - 8, dtype=bf))
+    with pytest.raises(ValueError, match="router_w"):
+        M.moe_router_logits(wl, torch.zeros(T, H, dtype=bf), torch.zeros(E, H - 8), ws=None)
+    good = dict(x=torch.zeros(T, H, dtype=bf), expert_offsets=torch.zeros(E + 1, dtype=i32),
+                tok_of=torch.zeros(T * k, dtype=i32), topk_w=torch.zeros(T * k),
+                w_gate_up=torch.zeros(E * 64 * H, dtype=bf), w_down=torch.zeros(E * H * 32, dtype=bf))
+    for name, bad in (("expert_offsets", torch.zeros(E, dtype=i32)), ("tok_of", torch.zeros(T * k - 1, dtype=i32)),
+                      ("topk_w", torch.zeros(T * k, dtype=torch.float64)), ("w_down", torch.zeros(7, dtype=bf))):
+        with pytest.raises(ValueError, match=name):
+            M.moe_expert_ffn(wl, ws=None, **dict(good, **{name: bad}))
+    with pytest.raises(ValueError, match="y_slots"):
+        M.moe_expert_ffn(wl, ws=None, y_slots=torch.zeros(T * k, H + 1), **good)
+    with pytest.raises(ValueError, match="y_slots"):
+        M.moe_combine(wl, torch.zeros(T * k - 1, H), None, T)
+    with pytest.raises(ValueError, match="shared_out"):
+        M.moe_combine(wl, torch.zeros(T * k, H), torch.zeros(T, H - 1), T)
+    q8 = G.make_q8_weights(wl, seed=0, device="cpu", group_size=32, shared=True)
+    bad_q8 = dict(q8, down=(q8["down"][0][:-16], q8["down"][1], q8["down"][2]))
+    with pytest.raises(ValueError, match="down.q"):
+        M.moe_forward_q8(wl, torch.zeros(T, H, dtype=bf), torch.zeros(E, H), None, bad_q8, ws=None)
+    with pytest.raises(ValueError, match="router_w"):
+        M.moe_forward_q8(wl, torch.zeros(T, H, dtype=bf), torch.zeros(E, H + 8), None, q8, ws=None)

@@ -65,6 +65,34 @@ def test_static_permute_matches_workspace_permute(M):
         assert torch.equal(tok_of, r_tok)
         assert torch.equal(x_perm.view(torch.int16), r_xp.view(torch.int16))
         assert int(off[-1]) == T * k  # no id was skipped
+        # and both equal the oracle's permutation (its definition: sorted by
+        # expert, then token)
+        o_off, o_row, o_tok = O.permutation(idx_np, E)
+        assert np.array_equal(off.cpu().numpy(), o_off)
+        assert np.array_equal(row_of.cpu().numpy(), o_row)
+        assert np.array_equal(tok_of.cpu().numpy(), o_tok)
+
+
+@pytest.mark.gpu
+def test_static_permute_signals_bad_ids(M):
+    # With no workspace error word, invalid or repeated ids show as a short
+    # total: expert_offsets[E] < T*k. The next call, with good ids, is whole.
+    T, E, k = 200, 16, 2
+    wl = G.tiny_workload(tokens=T, num_experts=E, num_experts_per_tok=k, hidden_size=64)
+    idx = torch.zeros((T, k), dtype=torch.int32)
+    idx[:, 0] = torch.arange(T) % E
+    idx[:, 1] = (torch.arange(T) + 1) % E
+    bad = idx.clone()
+    bad[17, 1] = E          # out of range
+    bad[30, 1] = bad[30, 0]  # repeated within a token
+    x = G.make_inputs(wl, seed=3, device="cpu", weights=False)["x"].cuda()
+    off, _, _, _ = _static_permute(M, wl, bad.cuda(), x)
+    assert int(off[-1]) == T * k - 2
+    off, row_of, tok_of, _ = _static_permute(M, wl, idx.cuda(), x)
+    o_off, o_row, o_tok = O.permutation(idx.numpy(), E)
+    assert np.array_equal(off.cpu().numpy(), o_off)
+    assert np.array_equal(row_of.cpu().numpy(), o_row)
+    assert np.array_equal(tok_of.cpu().numpy(), o_tok)
 
 
 def test_static_permute_rejects_sizes_beyond_its_scratch(M):
