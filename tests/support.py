@@ -2,7 +2,8 @@
 construction of the skewed workload, and the comparison rules.
 
 Tolerances (end-to-end, bf16 I/O with fp32 accumulation): max-abs <= 2e-2 and
-relative L2 <= 5e-3 against the fp64 oracle. Routing: indices bit-exact and
+relative L2 <= 5e-3 against the fp64 oracle; for bf16 outputs at |y| >= 8 the
+max-abs bar grows with bf16's half-ulp (see abs_tolerance). Routing: indices bit-exact and
 weights bitwise equal given identical fp32 logits. Tokens whose k-th and
 (k+1)-th biased scores (or topk_group-th and next group scores) lie within
 1e-6 are near-ties and are reported separately.
@@ -85,14 +86,37 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return O.as_f64(t)
 
 
-def compare(gpu: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, rel_l2=REL_L2):
-    d = gpu - ref
-    ma = float(np.max(np.abs(d))) if d.size else 0.0
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |v| (8 significant bits): the
+    largest error a correctly rounded bf16 output can have there."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 8.0)
+
+
+def abs_tolerance(ref: np.ndarray, max_abs=MAX_ABS, bf16_out=True) -> np.ndarray:
+    """Per-element max-abs bar. For bf16 outputs the 2e-2 bar leaves, below
+    |y| = 8, at least 2e-2 - 2^-6 for the arithmetic once the output's own
+    rounding (half an ulp, 2^-6 at 4 <= |y| < 8) is paid. From |y| = 8 on a
+    bf16 number alone can be 2^-5 away from the exact value, more than the bar,
+    so the bar grows with the half-ulp and keeps that same allowance for the
+    arithmetic (reading of "max-abs 2e-2 for bf16 I/O"). fp32 outputs keep 2e-2."""
+    if not bf16_out:
+        return np.full(np.shape(ref), max_abs)
+    return max_abs + np.maximum(0.0, bf16_half_ulp(ref) - 2.0 ** -6)
+
+
+def compare(gpu: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, rel_l2=REL_L2, bf16_out=True):
+    d = np.abs(gpu - ref)
+    ma = float(np.max(d)) if d.size else 0.0
+    tol = abs_tolerance(ref, max_abs, bf16_out)
+    over = float(np.max(d - tol)) if d.size else -1.0
+    wide = int(np.sum(tol > max_abs))
     den = float(np.linalg.norm(ref))
-    rl = float(np.linalg.norm(d) / den) if den > 0 else float(np.linalg.norm(d))
-    msg = f"{what}: max-abs {ma:.3e} (<= {max_abs}), rel-L2 {rl:.3e} (<= {rel_l2}), max|ref| {np.max(np.abs(ref)):.3f}"
+    rl = float(np.linalg.norm(gpu - ref) / den) if den > 0 else float(np.linalg.norm(gpu - ref))
+    msg = (f"{what}: max-abs {ma:.3e} (bar {max_abs}; {wide} elements at |y| >= 8 have the bar raised by the bf16 "
+           f"half-ulp), worst margin {-over:.3e}, rel-L2 {rl:.3e} (<= {rel_l2}), max|ref| {np.max(np.abs(ref)):.3f}")
     print(msg)
-    assert ma <= max_abs and rl <= rel_l2, msg
+    assert over <= 0.0 and rl <= rel_l2, msg
     return ma, rl
 
 

@@ -74,3 +74,17 @@ def test_expert_kernel_wait_runs_out_skinny_tiles(M):
                          moe_intermediate_size=64, shared_width=64, name="timeout-umma-bn64")
     inp = G.make_inputs(wl, seed=1, device=DEV)
     _expect_timeout_then_recover(M, wl, inp, "expert_accumulator", "tensor_cores")
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_fused_decode_wait_runs_out(M, T):
+    # The fused decode kernel's routing CTA withholds the release of the
+    # routing: every scheduler that needs it waits out its 1 ms, records the
+    # timeout and raises the abort word; every CTA leaves, the last one
+    # restoring the kernel's counters. Ling-3.0-flash shapes, 64 experts.
+    wl = G.workload("ling30_flash_decode_t8", num_experts=64, tokens=T)
+    wl = dict(wl, name="timeout-decode")
+    inp = G.make_inputs(wl, seed=2, device=DEV)
+    n0 = M.launch_count()
+    _expect_timeout_then_recover(M, wl, inp, "decode_routing", "auto")
+    assert M.launch_count() - n0 == 2, "both calls ran as one fused launch each"
