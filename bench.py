@@ -71,13 +71,12 @@ def peaks():
 KERNEL_SOURCES = {
     "expert_gate_up": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
     "expert_down": ["umma_ffn.cu", "ffn.cuh", "mbarrier.cuh", "common.cuh"],
-    "decode_fused": ["decode_fused.cu", "decode_tc.cu", "decode_fused.cuh", "fused_common.cuh", "route_block.cuh",
-                     "route.cuh", "mbarrier.cuh", "common.cuh"],
+    "decode_fused": ["decode_fused.cu", "decode_fused.cuh", "fused_common.cuh", "route_block.cuh", "route.cuh",
+                     "mbarrier.cuh", "common.cuh"],
 }
 MEASURED_TRAFFIC = {
     ("expert_gate_up", "ling26_flash_t512"): (2884745856, "a5d1e9a9b5d9b50a"),
     ("expert_down", "ling26_flash_t512"): (1491174528, "a5d1e9a9b5d9b50a"),
-    ("decode_fused", "ling30_flash_decode_t1"): (121844992, "482c39e62c1e6fa6"),
 }
 
 

@@ -27,12 +27,6 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
-// The header is followed by a block of counters the fused decode kernel needs
-// at zero when it starts (and leaves at zero when it ends). moe_workspace_init
-// zeroes both, and moe_check_device clears both after reporting an error.
-constexpr size_t kWsSyncBytes = 4096;
-constexpr size_t kWsZeroBytes = sizeof(WsHeader) + kWsSyncBytes;
-
 __device__ __forceinline__ void record_error(WsHeader* h, int status, int info) {
   if (h == nullptr) return;
   if (atomicCAS(&h->error, 0, status) == 0) h->error_info = info;

@@ -12,7 +12,7 @@
 #include <cstring>
 
 #include "common.cuh"
-#include "decode.cuh"
+#include "decode_fused.cuh"
 #include "ffn.cuh"
 
 namespace moe {
@@ -212,7 +212,7 @@ constexpr int64_t kLogitsGemvMaxT = 16;  // larger batches: router logits on the
 
 struct Layout {
   size_t hdr, logits, wr_planes, logit_parts, topk_idx, topk_w, offsets, row_of, tok_of, active, tile_cnt, tile_base;
-  size_t x_perm, h_perm, h_shared, y_slots, shared_out, sync, decode_h, decode_part, decode_route, total;
+  size_t x_perm, h_perm, h_shared, y_slots, shared_out, decode_sync, decode_pre, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -250,7 +250,6 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
     return at;
   };
   L.hdr = take(sizeof(WsHeader));
-  L.sync = take(kWsSyncBytes);  // directly after the header: both are zeroed by moe_workspace_init
   L.logits = take((size_t)T * E * 4);
   L.wr_planes = take(T > kLogitsGemvMaxT ? (size_t)3 * E * H * 2 : 0);
   L.logit_parts = take(logit_partial_bytes(c, T));
@@ -267,10 +266,9 @@ Layout layout(const moe_config& c, int64_t max_tokens) {
   L.h_shared = take((size_t)T * (Is > 0 ? Is : 8) * 4);
   L.y_slots = take((size_t)R * H * 4);
   L.shared_out = take((size_t)T * H * 4);
-  const bool fused = decode_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
-  L.decode_h = take(fused ? decode_hbuf_bytes((int)I, (int)Is) : 0);
-  L.decode_part = take(fused ? decode_part_bytes((int)H) : 0);
-  L.decode_route = take(fused ? sizeof(DecodeRoute) : 0);
+  const bool fused = decode_fused_supported(1, (int)k, (int)E, (int)H, (int)I, (int)Is);
+  L.decode_sync = take(fused ? decode_fused_sync_ints((int)H) * 4 : 0);
+  L.decode_pre = take(fused ? (size_t)2 * E * 12 : 0);  // up to 2 tokens: scores then keys
   L.total = off;
   return L;
 }
@@ -475,9 +473,9 @@ size_t moe_workspace_size(const moe_config* cfg, int64_t max_tokens) {
 }
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
-  if (ws == nullptr || ws_bytes < kWsZeroBytes) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
-  cudaError_t e = cudaMemsetAsync(ws, 0, kWsZeroBytes, as_stream(stream));
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "workspace init");
   return MOE_OK;
 }
@@ -610,8 +608,8 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
-  if (opt_decode_kernel() == 0 && decode_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size,
-                                                   c.moe_intermediate_size, shared_width(c))) {
+  if (opt_decode_kernel() == 0 && decode_fused_supported(T, c.num_experts_per_tok, c.num_experts, c.hidden_size,
+                                                         c.moe_intermediate_size, shared_width(c))) {
     DecodeArgs d{};
     d.x = x;
     d.T = (int)T;
@@ -632,18 +630,21 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
     d.w_down = w_down;
     d.ws_gate_up = has_shared ? ws_gate_up : nullptr;
     d.ws_down = has_shared ? ws_down : nullptr;
-    d.y = y;
+    d.logits = at<float>(ws, L.logits);
     d.topk_idx_out = topk_idx_out;
     d.topk_w_out = topk_w_out;
-    d.logits = at<float>(ws, L.logits);
-    d.hbuf = at<uint16_t>(ws, L.decode_h);
-    d.part = at<float>(ws, L.decode_part);
-    d.route = at<DecodeRoute>(ws, L.decode_route);
-    d.sync = at<int32_t>(ws, L.sync);
+    d.h = at<float>(ws, L.h_perm);
+    d.h_shared = at<float>(ws, L.h_shared);
+    d.y_slots = at<float>(ws, L.y_slots);
+    d.shared_out = at<float>(ws, L.shared_out);
+    d.sync = at<int32_t>(ws, L.decode_sync);
+    d.pre_orig = at<float>(ws, L.decode_pre);
+    d.pre_key = reinterpret_cast<unsigned long long*>(at<char>(ws, L.decode_pre) + (size_t)2 * c.num_experts * 4);
+    d.y = y;
     d.hdr = hdr;
     d.wait_ns = opt_wait_ns();
     d.withhold = opt_withhold() == 1 ? 1 : 0;
-    cudaError_t e = launch_decode(d, s);
+    cudaError_t e = launch_decode_fused(d, s);
     if (e != cudaSuccess) return cuda_fail(e, "fused decode");
     return MOE_OK;
   }
@@ -674,7 +675,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
 }
 
 moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
-  if (ws == nullptr || ws_bytes < kWsZeroBytes) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace is NULL or too small");
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "stream");
@@ -682,7 +683,7 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
   e = cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "read error word");
   if (word[0] == 0) return MOE_OK;
-  e = cudaMemsetAsync(ws, 0, kWsZeroBytes, s);
+  e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   if (word[0] == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "device wait timed out (site %d)", word[1]);

@@ -59,11 +59,8 @@ __device__ __forceinline__ float warp_max_f32(float v) {
 
 // Routes the token whose fp32 gates are Lrow[0..E): writes idx_out[0..k) (expert
 // ids, ordered by biased score descending then id ascending) and w_out[0..k)
-// (routing weights). buf: this warp's 32*P floats of shared memory. kLdg:
-// Lrow is read-only global memory for the whole launch (read through the
-// non-coherent cache); false for gates in shared memory or written earlier in
-// the same launch.
-template <int P, bool kLdg = true>
+// (routing weights). buf: this warp's 32*P floats of shared memory.
+template <int P>
 __device__ __forceinline__ void route_one_token(const float* __restrict__ Lrow, const float* __restrict__ bias, int E,
                                                 int k, int n_group, int topk_group, int score_fn, int norm,
                                                 float scale, float* buf, int32_t* idx_out, float* w_out) {
@@ -75,7 +72,7 @@ __device__ __forceinline__ void route_one_token(const float* __restrict__ Lrow, 
 #pragma unroll
   for (int i = 0; i < P; ++i) {
     const int e = lane * P + i;
-    L[i] = (e < E) ? (kLdg ? __ldg(Lrow + e) : Lrow[e]) : -INFINITY;
+    L[i] = (e < E) ? __ldg(Lrow + e) : -INFINITY;
   }
 
   // ---- score function: fp64 evaluation, one rounding to fp32 ----

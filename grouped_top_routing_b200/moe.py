@@ -27,7 +27,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_launch_count", "moe_last_error",
            "moe_permute_static", "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
-FUSED_DECODE_MAX_TOKENS = 8  # moe_forward runs the whole block as one launch up to this batch (shapes permitting)
+FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch up to this batch (shapes permitting)
 DECODE = {"auto": 0, "unfused": 1}
 WITHHOLD = {None: 0, "decode_routing": 1, "expert_accumulator": 2}
 

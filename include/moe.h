@@ -136,9 +136,9 @@ typedef struct {
                              bracketed by the two events, or -1 for none */
   void* timer_start;      /* cudaEvent_t recorded just before each such launch */
   void* timer_stop;       /* cudaEvent_t recorded just after it */
-  int32_t test_withhold;  /* test aid, 0 in normal use. 1: the fused decode
-                             kernel withholds the release of its routing, so
-                             every wait for it runs out; 2: the tensor-core
+  int32_t test_withhold;  /* test aid, 0 in normal use. 1: CTA 0 of the fused
+                             decode kernel never arrives at its grid barrier,
+                             so every other CTA's wait runs out; 2: the tensor-core
                              expert kernel withholds its first accumulator
                              hand-over, so the epilogue's wait runs out. Both
                              end in MOE_ERR_TIMEOUT after wait_limit_ns and

@@ -76,12 +76,14 @@ def test_expert_kernel_wait_runs_out_skinny_tiles(M):
     _expect_timeout_then_recover(M, wl, inp, "expert_accumulator", "tensor_cores")
 
 
-@pytest.mark.parametrize("T", [1, 8])
+@pytest.mark.parametrize("T", [1, 2])
 def test_fused_decode_wait_runs_out(M, T):
-    # The fused decode kernel's routing CTA withholds the release of the
-    # routing: every scheduler that needs it waits out its 1 ms, records the
-    # timeout and raises the abort word; every CTA leaves, the last one
-    # restoring the kernel's counters. Ling-3.0-flash shapes, 64 experts.
+    # CTA 0 of the fused decode kernel never arrives at the grid barrier that
+    # follows the router rows: every other CTA's wait there runs out after
+    # 1 ms, and every producer's wait for the routing after another; all CTAs
+    # leave with their copies drained. moe_check_device reports the timeout
+    # and resets the barrier's arrival count with the header. Ling-3.0-flash
+    # shapes, 64 experts.
     wl = G.workload("ling30_flash_decode_t8", num_experts=64, tokens=T)
     wl = dict(wl, name="timeout-decode")
     inp = G.make_inputs(wl, seed=2, device=DEV)
