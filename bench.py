@@ -99,21 +99,22 @@ def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decod
     return entry[0] if kernel_source_hash(kernel) == entry[1] else None
 
 
-def algorithmic(wl, T, n_unique, weight_bytes=2.0):
+def algorithmic(wl, T, n_unique, weight_bytes=2.0, h_bytes=4):
     """Bytes each expert pass must move, and the block's flops, given the
     number of distinct routed experts the batch touched. Expert weights count
-    weight_bytes per element (2 for bf16; 1 + 4 / group for 8-bit affine codes
-    with a bf16 scale and bias per group). Activations count at the width this
-    design stores them: token rows bf16 (2 B), the SwiGLU product as two bf16
-    planes or fp32 (4 B), expert slot rows and the shared MLP output fp32 (4 B)."""
+    weight_bytes per element (2 for bf16 or fp16; 1 + 4 / group for 8-bit
+    affine codes with a bf16 scale and bias per group). Activations count at
+    the width this design stores them: token rows bf16 (2 B), the SwiGLU
+    product h_bytes (two bf16 planes or fp32: 4 B; one fp16 plane: 2 B),
+    expert slot rows and the shared MLP output fp32 (4 B)."""
     H, E, k, I, Is = (wl["hidden_size"], wl["num_experts"], wl["num_experts_per_tok"],
                       wl["moe_intermediate_size"], wl["shared_width"])
     R = T * k
     w_gate_up = int((n_unique * 2 * I + 2 * Is) * H * weight_bytes)
     w_down = int((n_unique * I + Is) * H * weight_bytes)
     h_elems = R * I + T * Is
-    gate_up_bytes = w_gate_up + (R + T) * H * 2 + h_elems * 4   # weights + token rows in + h planes out
-    down_bytes = w_down + h_elems * 4 + (R + T) * H * 4          # weights + h planes in + fp32 rows out
+    gate_up_bytes = w_gate_up + (R + T) * H * 2 + h_elems * h_bytes   # weights + token rows in + h out
+    down_bytes = w_down + h_elems * h_bytes + (R + T) * H * 4          # weights + h in + fp32 rows out
     step_bytes = (w_gate_up + w_down + E * H * 4 + 2 * T * H * 2)  # weights + router + x in + y out
     gate_up_flops = 2 * H * 2 * h_elems          # gate and up projections of every routed and shared row
     down_flops = 2 * H * h_elems
@@ -310,6 +311,13 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     base_opts = dict(ffn_path=args.ffn_path, decode=args.decode)
+    # fp16 copies of the down weights, made once before anything is timed (a
+    # load-time conversion, exact for |w| >= 2^-14): the tensor-core down pass
+    # then multiplies fp16 operands, one MMA per k-step
+    f16 = q8 is None and args.down_weights == "f16"
+    if f16:
+        base_opts["w_down_f16"] = M.convert_bf16_to_f16(inp["w_down"])
+        base_opts["ws_down_f16"] = None if inp["ws_down"] is None else M.convert_bf16_to_f16(inp["ws_down"])
 
     def step(x=None, out=None, timer=None):
         out = y if out is None else out
@@ -332,7 +340,9 @@ def run_ours(args):
                               inp["ws_gate_up"], inp["ws_down"], ws, return_routing=True,
                               opts=M.options(**base_opts))
     n_unique = int(torch.unique(idx).numel())
-    work = algorithmic(wl, T, n_unique, 1.0 + 4.0 / args.q8 if q8 is not None else 2.0)
+    tc_path = not fused and (args.ffn_path == "tensor_cores" or (args.ffn_path == "auto" and T > M.STREAM_MAX_TOKENS))
+    work = algorithmic(wl, T, n_unique, 1.0 + 4.0 / args.q8 if q8 is not None else 2.0,
+                       h_bytes=2 if (f16 and tc_path) else 4)
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -482,12 +492,15 @@ def run_ours(args):
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "overrides": args.set, "ffn_path": args.ffn_path,
+                   "down_weights": None if q8 is not None else args.down_weights,
                    "decode": args.decode, "tokens": T, "hidden_size": wl["hidden_size"],
                    "num_experts": wl["num_experts"], "top_k": wl["num_experts_per_tok"],
                    "n_group": wl["n_group"], "topk_group": wl["topk_group"],
                    "moe_intermediate_size": wl["moe_intermediate_size"], "shared_width": wl["shared_width"],
                    "experts_touched": n_unique, "parallelism": f"replicas x{world} (token batches)",
-                   "expert_weights": f"8-bit affine, group {args.q8}" if q8 is not None else "bf16",
+                   "expert_weights": (f"8-bit affine, group {args.q8}" if q8 is not None else
+                                      "bf16; down_proj also as an fp16 copy made once before timing (exact for "
+                                      "|w| >= 2^-14), read by the tensor-core down pass" if f16 else "bf16"),
                    "l2": "256 MiB L2 flush between timed steps; expert weights >> 126 MB L2"},
         "step_hbm_gbs": step_gbs, "step_tflops": step_tflops,
         "roofline": roofline,
@@ -625,6 +638,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "streaming", "tensor_cores"],
                     help="expert-FFN kernels (default: the library's automatic choice)")
+    ap.add_argument("--down-weights", default="f16", choices=["f16", "bf16"],
+                    help="down_proj operands of the tensor-core pass: an fp16 copy made before timing, or the bf16 "
+                         "weights (h then kept as two bf16 planes)")
     ap.add_argument("--decode", default="auto", choices=["auto", "unfused"],
                     help="a few tokens as one fused launch (auto, the library's choice) or as separate kernels")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",

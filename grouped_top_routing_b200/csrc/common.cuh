@@ -60,6 +60,14 @@ __device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// fp32 -> fp16 bits, round to nearest even; and whether fp16 bits are finite.
+__device__ __forceinline__ uint16_t f32_to_f16(float f) {
+  uint16_t h;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(f));
+  return h;
+}
+__device__ __forceinline__ bool f16_finite(uint16_t h) { return (h & 0x7C00u) != 0x7C00u; }
+
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
 // Sum of the 8 products of one 16-byte bf16 weight chunk with 8 fp32 values.

@@ -26,7 +26,11 @@ struct FfnArgs {
   const uint16_t* w_down;     // [E, H, I]
   const uint16_t* ws_gate_up; // [2Is, H] or null
   const uint16_t* ws_down;    // [H, Is]
-  void* h_perm;               // [T*k, I]: fp32 (streaming path) or bf16 (tensor-core path)
+  // fp16 copies of the down weights, or null: the tensor-core path then keeps
+  // h as one fp16 plane and multiplies fp16 operands in the down pass
+  const uint16_t* w_down_f16;   // [E, H, I]
+  const uint16_t* ws_down_f16;  // [H, Is]; set whenever ws_gate_up is
+  void* h_perm;               // [T*k, I]: fp32 (streaming path), two bf16 planes or one fp16 plane (tensor cores)
   void* h_shared;             // [T, Is]: same element type as h_perm
   float* y_slots;             // [T*k, H]
   float* shared_out;          // [T, H]

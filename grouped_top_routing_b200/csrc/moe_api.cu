@@ -33,6 +33,8 @@ cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* a
 cudaError_t launch_identity_route(int64_t T, int32_t* offsets, int32_t* tok_of, float* w, cudaStream_t s);
 cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
                            cudaStream_t s);
+cudaError_t launch_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, int32_t* bad_count,
+                                       cudaStream_t s);
 cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
                                const uint16_t* x, int H, uint16_t* x_perm, cudaStream_t s);
 
@@ -205,6 +207,20 @@ moe_status check_ptr(const char* name, const void* p, size_t align, bool require
   return MOE_OK;
 }
 
+// opts->w_down_f16 / ws_down_f16 against the call: aligned, and the shared
+// MLP's copy present whenever the call runs a shared MLP.
+moe_status check_down_f16(bool shared_used) {
+  if (t_opts == nullptr) return MOE_OK;
+  if (t_opts->w_down_f16 == nullptr) {
+    if (t_opts->ws_down_f16 != nullptr)
+      return fail(MOE_ERR_INVALID_ARG, "opts->ws_down_f16 is set but opts->w_down_f16 is NULL");
+    return MOE_OK;
+  }
+  MOE_TRY(check_ptr("opts->w_down_f16", t_opts->w_down_f16, 16, true));
+  MOE_TRY(check_ptr("opts->ws_down_f16", t_opts->ws_down_f16, 16, shared_used));
+  return MOE_OK;
+}
+
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
@@ -367,6 +383,10 @@ moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint
     return MOE_OK;
   }
   if (use_tensor_cores(c, T)) {
+    if (t_opts != nullptr && t_opts->w_down_f16 != nullptr) {
+      a.w_down_f16 = t_opts->w_down_f16;
+      a.ws_down_f16 = a.ws_gate_up != nullptr ? t_opts->ws_down_f16 : nullptr;
+    }
     if (x_perm == nullptr) {  // the tensor-core path reads expert rows contiguously
       uint16_t* xp = at<uint16_t>(ws, L.x_perm);
       e = launch_gather_rows(offsets, c.num_experts, tok_of, c.num_experts_per_tok, T, x, c.hidden_size, xp, s);
@@ -559,6 +579,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int64_t T, const uint16_t* x, c
   MOE_TRY(check_ptr("shared_out", shared_out, 16, ws_gate_up != nullptr));
   if (ws_gate_up != nullptr && !has_shared)
     return fail(MOE_ERR_INVALID_ARG, "ws_gate_up given but the config has no shared MLP");
+  MOE_TRY(check_down_f16(ws_gate_up != nullptr));
   if (ws_gate_up == nullptr) shared_out = nullptr;
   return run_ffn(*cfg, T, x, x_perm, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws_gate_up, ws_down, y_slots,
                  shared_out, ws, false, as_stream(stream));
@@ -597,6 +618,7 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   MOE_TRY(check_ptr("expert_bias", expert_bias, 4, false));
   MOE_TRY(check_ptr("w_gate_up", w_gate_up, 16, true));
   MOE_TRY(check_ptr("w_down", w_down, 16, true));
+  MOE_TRY(check_down_f16(has_shared));
   MOE_TRY(check_ptr("ws_gate_up", ws_gate_up, 16, has_shared));
   MOE_TRY(check_ptr("ws_down", ws_down, 16, has_shared));
   MOE_TRY(check_ptr("y", y, 16, true));
@@ -687,7 +709,26 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   if (word[0] == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "device wait timed out (site %d)", word[1]);
+  if (word[0] == MOE_ERR_RANGE)
+    return fail(MOE_ERR_RANGE, "a SwiGLU product left fp16's range (expert row %d); use the bf16 down weights",
+                word[1]);
   return fail(MOE_ERR_DEVICE_CHECK, "device index check failed (index %d)", word[1]);
+}
+
+moe_status moe_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, int32_t* out_of_range,
+                                   void* stream) {
+  if (n < 0) return fail(MOE_ERR_INVALID_ARG, "n = %lld is negative", (long long)n);
+  MOE_TRY(check_ptr("src", src, 16, n > 0));
+  MOE_TRY(check_ptr("dst", dst, 16, n > 0));
+  MOE_TRY(check_ptr("out_of_range", out_of_range, 4, true));
+  if (n > 0) {
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+    const uintptr_t bytes = (uintptr_t)n * 2;
+    if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(MOE_ERR_INVALID_ARG, "src and dst overlap");
+  }
+  cudaError_t e = launch_convert_bf16_to_f16(src, dst, n, out_of_range, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bf16 -> fp16 conversion");
+  return MOE_OK;
 }
 
 uint64_t moe_launch_count(void) { return t_launches; }
@@ -716,6 +757,7 @@ moe_status moe_dense_mlp(int32_t hidden_size, int32_t intermediate_size, const u
   MOE_TRY(check_ptr("w_gate_up", w_gate_up, 16, true));
   MOE_TRY(check_ptr("w_down", w_down, 16, true));
   MOE_TRY(check_ptr("y", y, 16, true));
+  MOE_TRY(check_down_f16(false));
   const Layout L = layout(c, T);
   cudaStream_t s = as_stream(stream);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -742,6 +784,8 @@ moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, c
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   const moe_config& c = *cfg;
   MOE_TRY(validate_q8(c, w, ws_gate_up, ws_down));
+  if (opts != nullptr && (opts->w_down_f16 != nullptr || opts->ws_down_f16 != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "opts->w_down_f16 applies to bf16 weights, not to moe_forward_q8");
   if (T == 0) return MOE_OK;
   const bool has_shared = shared_width(c) > 0;
   MOE_TRY(check_ptr("x", x, 16, true));

@@ -16,12 +16,18 @@
 //                 y_slots[slot(token), n] = w_slot * (D_hi[n] + D_lo[n])
 //                 (fp32; shared MLP: weight 1)
 //
-// h is written as two bf16 planes, h_hi = bf16(h) and h_lo = bf16(h - h_hi).
-// The DOWN stage holds the token tile of each plane back to back, so the pair
-// is a single B operand of 2 BN rows: one MMA per weight tile yields both
-// W.h_hi and W.h_lo, which the epilogue adds. The SwiGLU product thus carries
-// ~16 significant bits into the down projection, with no extra weight bytes
-// and no extra MMA instructions.
+// With bf16 down weights, h is written as two bf16 planes, h_hi = bf16(h) and
+// h_lo = bf16(h - h_hi). The DOWN stage holds the token tile of each plane back
+// to back, so the pair is a single B operand of 2 BN rows: one MMA per weight
+// tile yields both W.h_hi and W.h_lo, which the epilogue adds. The SwiGLU
+// product thus carries ~16 significant bits into the down projection, at twice
+// the down pass's tensor work.
+//
+// With an fp16 copy of the down weights (exact for bf16 values of magnitude
+// 2^-14 or more), h is written as one fp16 plane (11 significant bits) and the
+// down pass runs kind::f16 MMAs on fp16 operands: one MMA per k-step and half
+// the h bytes. A SwiGLU product beyond fp16's range is recorded as
+// MOE_ERR_RANGE.
 //
 // Persistent, warp-specialised CTA (one per SM, 192 threads):
 //   warp 0      : TMA producer (one lane), STAGES-deep ring of weight and token tiles
@@ -140,7 +146,8 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 
-// D[tmem] (+)= A[smem] . B[smem]^T, bf16 inputs, fp32 accumulate, 128 x N x 16.
+// D[tmem] (+)= A[smem] . B[smem]^T, 16-bit inputs (bf16 or fp16, per the
+// instruction descriptor), fp32 accumulate, 128 x N x 16.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
   const uint32_t z = 0;
@@ -173,10 +180,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
+// Instruction descriptor, kind::f16: D fp32, A and B both bf16 (format 1) or
+// both fp16 (format 0), both K-major.
 template <int N>
 __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+template <int N>
+__device__ __forceinline__ constexpr uint32_t idesc_fp16() {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 // ----------------------------------------------------------------------------
@@ -184,20 +196,22 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
 // ----------------------------------------------------------------------------
 // Stage = NA weight tiles (128 x 64) then NB token tiles (BN x 64), all
 // 1024-byte aligned. GATE_UP / LOGITS: NA = 2, NB = 1 (gate and up rows, or
-// two blocks of router rows, share the token tile). DOWN: NB = 2 (the h_hi and
-// h_lo token tiles, one B operand of 2 BN rows) and NA = 2 while the TMEM
-// budget allows (BN <= 64), else 1. Each accumulator is NCOL columns.
+// two blocks of router rows, share the token tile). DOWN with two h planes:
+// NB = 2 (the h_hi and h_lo token tiles, one B operand of 2 BN rows) and
+// NA = 2 while the TMEM budget allows (BN <= 64), else 1; with one fp16 plane
+// (H16): NB = 1, NA = 2. Each accumulator is NCOL columns.
 //
 // Token-major modes (BN = 128 token rows): NA = token tiles per stage (1; the
-// h_hi and h_lo planes for kDownTM), NB = 2 weight boxes of 128 rows forming
-// one B operand of 256 rows, one accumulator of NCOL = 256 columns.
-template <int BN, int MODE>
+// h_hi and h_lo planes for kDownTM on bf16 weights), NB = 2 weight boxes of
+// 128 rows forming one B operand of 256 rows, one accumulator of NCOL = 256.
+template <int BN, int MODE, bool H16>
 struct Shape {
   static constexpr bool TM = token_major(MODE);
-  static constexpr int NA = TM ? (MODE == kDownTM ? 2 : 1)
-                               : ((MODE == kLogits || (MODE == kDown && BN > 64)) ? 1 : 2);
-  static constexpr int NB = TM ? 2 : (MODE == kDown ? 2 : 1);
-  static constexpr int NCOL = TM ? 256 : (MODE == kDown ? 2 * BN : BN);
+  static constexpr bool kTwoPlanes = (MODE == kDown || MODE == kDownTM) && !H16;  // h_hi and h_lo tiles
+  static constexpr int NA = TM ? (MODE == kDownTM && kTwoPlanes ? 2 : 1)
+                               : ((MODE == kLogits || (MODE == kDown && kTwoPlanes && BN > 64)) ? 1 : 2);
+  static constexpr int NB = TM ? 2 : (MODE == kDown && kTwoPlanes ? 2 : 1);
+  static constexpr int NCOL = TM ? 256 : (MODE == kDown && kTwoPlanes ? 2 * BN : BN);
   static constexpr int NACC = TM ? 1 : NA;                         // accumulators per buffer
   static constexpr int ROWS = TM ? (MODE == kDownTM ? 256 : BM) : NA * BM;  // weight rows per tile
   static constexpr uint32_t kTmemCols = 2 * NACC * NCOL;           // two buffers
@@ -211,8 +225,8 @@ struct TileInfo {
   int a0_row, a1_row, b_row, kb0, kblocks, nchunks;
 };
 
-template <int BN, int MODE>
-__device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const int* pre, const int* s_e, const int* s_m,
+template <int BN, int MODE, bool H16>
+__device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const int* pre, const int16_t* s_e, const int* s_m,
                                                 const int* s_r0, const UmmaParams& p) {
   int lo = 0, hi = n_groups - 1;
   while (lo < hi) {
@@ -266,7 +280,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
     }
   } else {
     K = t.shared ? p.Is : p.I;
-    t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * Shape<BN, MODE>::ROWS;
+    t.a0_row = (t.shared ? 0 : t.e * p.H) + t.nb * Shape<BN, MODE, H16>::ROWS;
     t.a1_row = t.a0_row + BM;  // used when the stage holds two weight tiles
   }
   t.b_row = (int)t.r0 + t.mb * BN;
@@ -276,36 +290,49 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, int n_groups, const in
 }
 
 // Shared-memory carve-up of one CTA.
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, bool H16>
 struct Smem {
-  static constexpr int NA = Shape<BN, MODE>::NA;
-  static constexpr int NB = Shape<BN, MODE>::NB;
+  static constexpr int NA = Shape<BN, MODE, H16>::NA;
+  static constexpr int NB = Shape<BN, MODE, H16>::NB;
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = BN * BK * 2;
   static constexpr int kStage = NA * kA + NB * kB;
   static constexpr int kBarriers = (2 * STAGES + 5) * 8;
-  static constexpr int kTables = 4 * (kMaxGroups + 1) * 4;
-  static constexpr size_t kTotal = 1024 + (size_t)STAGES * kStage + kBarriers + 16 + kTables;
+  static constexpr int kTables = 3 * (kMaxGroups + 1) * 4 + ((kMaxGroups + 1) * 2 + 15) / 16 * 16;
+  static constexpr size_t kBase = 1024 + (size_t)STAGES * kStage + kBarriers + 16 + kTables;
+  // Token-major DOWN epilogue: per epilogue warp, one tile of 32 rows x kCW
+  // fp32 columns, rows padded by 16 bytes so that both the row-per-thread
+  // writes and the row-per-lane-group reads are free of bank conflicts. The
+  // widest chunk that fits beside the ring.
+  static constexpr size_t kLimit = 232448;
+  static constexpr size_t stg_bytes(int cw) { return (size_t)4 * 32 * (cw * 4 + 16); }
+  static constexpr bool kStg = MODE == kDownTM;
+  static constexpr int kCW = (!kStg || kBase + stg_bytes(32) <= kLimit) ? 32 : 16;  // (unused without kStg)
+  static constexpr int kStgRow = kCW * 4 + 16;
+  static constexpr size_t kStaging = kStg ? stg_bytes(kCW) : 0;
+  static constexpr size_t kTotal = kBase + kStaging;
 };
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, bool H16>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_ffn_kernel(const __grid_constant__ CUtensorMap mapA_r, const __grid_constant__ CUtensorMap mapB_r,
                     const __grid_constant__ CUtensorMap mapB2_r, const __grid_constant__ CUtensorMap mapA_s,
                     const __grid_constant__ CUtensorMap mapB_s, const __grid_constant__ CUtensorMap mapB2_s,
                     const UmmaParams p) {
   pdl_launch_dependents();
-  using L = Smem<BN, STAGES, MODE>;
-  using SH = Shape<BN, MODE>;
+  using L = Smem<BN, STAGES, MODE, H16>;
+  using SH = Shape<BN, MODE, H16>;
   constexpr uint32_t kTmemCols = SH::kTmemCols;
+  constexpr bool kDownF16 = H16 && (MODE == kDown || MODE == kDownTM);  // fp16 operands
   constexpr uint32_t kIdesc = idesc_bf16<BN>();
-  constexpr uint32_t kIdescDown = idesc_bf16<(2 * BN <= 256 ? 2 * BN : 256)>();
-  constexpr uint32_t kIdescTM = idesc_bf16<256>();
-  static_assert(MODE != kDown || 2 * BN <= 256, "DOWN issues N = 2 BN <= 256");
+  constexpr uint32_t kIdescDown = kDownF16 ? idesc_fp16<BN>() : idesc_bf16<(2 * BN <= 256 ? 2 * BN : 256)>();
+  constexpr uint32_t kIdescTM = kDownF16 ? idesc_fp16<256>() : idesc_bf16<256>();
+  static_assert(MODE != kDown || !SH::kTwoPlanes || 2 * BN <= 256, "DOWN issues N = 2 BN <= 256");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * L::kStage);
+  uint8_t* staging = smem + (size_t)STAGES * L::kStage;  // L::kStaging bytes (token-major DOWN only)
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + L::kStaging);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -313,9 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* pre = reinterpret_cast<int*>(tmem_slot + 4);
-  int* s_e = pre + (kMaxGroups + 1);
-  int* s_m = s_e + (kMaxGroups + 1);
+  int* s_m = pre + (kMaxGroups + 1);
   int* s_r0 = s_m + (kMaxGroups + 1);
+  int16_t* s_e = reinterpret_cast<int16_t*>(s_r0 + (kMaxGroups + 1));  // expert ids < 1024 (-1: shared MLP)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -367,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       m = (int)p.T;
       tiles = nb_shared * ((m + BN - 1) / BN);
     }
-    s_e[g] = e;
+    s_e[g] = (int16_t)e;
     s_m[g] = m;
     s_r0[g] = (int)r0;
     pre[g + 1] = tiles;
@@ -404,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+        const TileInfo t = decode_tile<BN, MODE, H16>(tile, n_groups, pre, s_e, s_m, s_r0, p);
         const CUtensorMap* mA = t.shared ? &mapA_s : &mapA_r;
         const CUtensorMap* mB = t.shared ? &mapB_s : &mapB_r;
         const CUtensorMap* mB2 = t.shared ? &mapB2_s : &mapB2_r;
@@ -448,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+        const TileInfo t = decode_tile<BN, MODE, H16>(tile, n_groups, pre, s_e, s_m, s_r0, p);
         for (int ch = 0; ok && ch < t.nchunks; ++ch, ++tcount) {
           const int a = tcount & 1;
           const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
@@ -477,8 +504,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t bdesc = sw128_desc(sb + kk * 32);
               if (SH::TM) {  // D (128 tokens x 256 weight rows) += A_token . B_weights
                 umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdescTM, acc);
-                if (MODE == kDownTM) umma_bf16(d0, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescTM, 1u);  // h_lo
-              } else if (MODE == kDown) {  // B = [h_hi tile; h_lo tile]: 2 BN rows, each D spans 2 BN columns
+                if (MODE == kDownTM && SH::kTwoPlanes)
+                  umma_bf16(d0, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescTM, 1u);  // h_lo
+              } else if (MODE == kDown) {  // B = [h_hi tile; h_lo tile] (2 BN rows, D spans 2 BN columns) or the fp16 h tile
                 umma_bf16(d0, sw128_desc(sa0 + kk * 32), bdesc, kIdescDown, acc);
                 if (SH::NA == 2) umma_bf16(d1, sw128_desc(sa0 + L::kA + kk * 32), bdesc, kIdescDown, acc);
               } else {
@@ -504,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tcount = 0;
     bool alive = true;
     for (int tile = blockIdx.x; alive && tile < total_tiles; tile += gridDim.x) {
-      const TileInfo t = decode_tile<BN, MODE>(tile, n_groups, pre, s_e, s_m, s_r0, p);
+      const TileInfo t = decode_tile<BN, MODE, H16>(tile, n_groups, pre, s_e, s_m, s_r0, p);
       const int mvalid = min(BN, t.m - t.mb * BN);
       // DOWN: every token column's destination slot and routing weight, fetched
       // once per tile (column lane + 32 r in register r) before the accumulator
@@ -580,7 +608,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(taddr + c0, g);
             tmem_ld16(taddr + BM + c0, u);
             const int j0 = t.nb * BM + c0;
-            if (tm_valid && j0 < width) {
+            if (H16 && tm_valid && j0 < width) {
+              uint32_t h2[8];
+              bool fin = true;
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                const uint16_t a0 = f32_to_f16(silu_f32(g[i]) * u[i]), a1 = f32_to_f16(silu_f32(g[i + 1]) * u[i + 1]);
+                fin = fin && f16_finite(a0) && f16_finite(a1);
+                h2[i / 2] = (uint32_t)a0 | ((uint32_t)a1 << 16);
+              }
+              if (!fin) record_error(p.hdr, MOE_ERR_RANGE, (int)(t.r0 + tm_tok));
+              if (j0 + 16 <= width) {
+                uint4* dh = reinterpret_cast<uint4*>(hrow + j0);
+                dh[0] = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+                dh[1] = make_uint4(h2[4], h2[5], h2[6], h2[7]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (j0 + i < width) hrow[j0 + i] = (uint16_t)(h2[i / 2] >> (16 * (i & 1)));
+              }
+            } else if (tm_valid && j0 < width) {
               uint32_t hi2[8], lo2[8];
 #pragma unroll
               for (int i = 0; i < 16; i += 2) {
@@ -609,25 +656,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else if (MODE == kDownTM) {
-          // columns: 256 weight rows n0 .. n0+255 (h_hi and h_lo already summed by the MMA)
+          // columns: 256 weight rows n0 .. n0+255 (with two h planes, h_hi and h_lo
+          // are already summed by the MMA). Thread `lane` holds output row
+          // `lane` of the warp's 32; each chunk of kCW columns is turned around
+          // in shared memory so that every store instruction writes whole
+          // row segments: lane l stores 16 bytes of row (l / G) of a group of
+          // 32 / G rows, G = kCW / 4 lanes per row (row-per-thread 16-byte
+          // stores touched 32 lines per instruction and left the pass
+          // store-bound at twice its MMA time).
+          constexpr int kCW = L::kCW, G = kCW / 4, RPI = 32 / G;  // lanes per row, rows per instruction
           const int n0 = t.nb * 2 * BM;
-          float* orow = t.shared ? p.shared_out + tm_tok * p.H : p.y_slots + tm_slot * p.H;
+          // the destination row offset of this lane's row, or -1 when the row is absent
+          const long long my_dst = !(tm_valid && tm_slot >= 0)
+                                       ? -1ll
+                                       : (t.shared ? (long long)tm_tok : tm_slot) * (long long)p.H;
+          float* obase = t.shared ? p.shared_out : p.y_slots;
+          uint8_t* stg = staging + (size_t)q * 32 * L::kStgRow;
+          const int sub = lane / G, part = lane % G;  // this lane's row within a group, its 16-byte column part
 #pragma unroll 1
-          for (int c0 = 0; c0 < 2 * BM; c0 += 16) {
-            float v[16];
-            tmem_ld16(taddr + c0, v);
+          for (int c0 = 0; c0 < 2 * BM; c0 += kCW) {
+            float v[kCW];
+#pragma unroll
+            for (int j = 0; j < kCW; j += 16) tmem_ld16(taddr + c0 + j, v + j);
             const int n = n0 + c0;
-            if (tm_valid && tm_slot >= 0 && n < p.H) {
-              if (n + 16 <= p.H) {
-                float4* d = reinterpret_cast<float4*>(orow + n);
+            if (n >= p.H) continue;  // warp-uniform
+            if (n + kCW <= p.H) {
+              __syncwarp();  // the previous chunk's reads of the tile are done
+              float4* d = reinterpret_cast<float4*>(stg + lane * L::kStgRow);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  d[i] = make_float4(tm_w * v[4 * i], tm_w * v[4 * i + 1], tm_w * v[4 * i + 2], tm_w * v[4 * i + 3]);
-              } else {
+              for (int i = 0; i < G; ++i)
+                d[i] = make_float4(tm_w * v[4 * i], tm_w * v[4 * i + 1], tm_w * v[4 * i + 2], tm_w * v[4 * i + 3]);
+              __syncwarp();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  if (n + i < p.H) orow[n + i] = tm_w * v[i];
+              for (int r0 = 0; r0 < 32; r0 += RPI) {
+                const int r = r0 + sub;
+                const long long dst = __shfl_sync(0xffffffffu, my_dst, r);
+                const float4 val = *reinterpret_cast<const float4*>(stg + r * L::kStgRow + part * 16);
+                if (dst >= 0) *reinterpret_cast<float4*>(obase + dst + n + part * 4) = val;
               }
+            } else if (my_dst >= 0) {  // ragged last chunk of the hidden size: per element
+#pragma unroll
+              for (int i = 0; i < kCW; ++i)
+                if (n + i < p.H) obase[my_dst + n + i] = tm_w * v[i];
             }
           }
         }
@@ -654,11 +724,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = c0 + i;
                 if (c < mvalid) {
                   const float h = silu_f32(v0[i]) * v1[i];
-                  const uint16_t h_hi = f32_to_bf16(h);
-                  const uint16_t h_lo = f32_to_bf16(h - __uint_as_float((uint32_t)h_hi << 16));
                   const int64_t at = ((int64_t)t.mb * BN + c) * width + j;
-                  hi[at] = h_hi;
-                  hi[plane + at] = h_lo;
+                  if (H16) {
+                    const uint16_t hh = f32_to_f16(h);
+                    if (!f16_finite(hh)) record_error(p.hdr, MOE_ERR_RANGE, (int)(t.r0 + t.mb * BN + c));
+                    hi[at] = hh;
+                  } else {
+                    const uint16_t h_hi = f32_to_bf16(h);
+                    const uint16_t h_lo = f32_to_bf16(h - __uint_as_float((uint32_t)h_hi << 16));
+                    hi[at] = h_hi;
+                    hi[plane + at] = h_lo;
+                  }
                 }
               }
             }
@@ -668,15 +744,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int acc_i = 0; acc_i < SH::NA; ++acc_i) {  // accumulator acc_i: weight rows n + acc_i * 128
               const uint32_t ta = taddr + (uint32_t)(acc_i * SH::NCOL);
-              tmem_ld16(ta + c0, v0);       // W . h_hi
-              tmem_ld16(ta + BN + c0, v1);  // W . h_lo
+              tmem_ld16(ta + c0, v0);  // W . h_hi (or W . h, one fp16 plane)
+              if (SH::kTwoPlanes) tmem_ld16(ta + BN + c0, v1);  // W . h_lo
               const int nn = n + acc_i * BM;
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int c = c0 + i;  // compile-time after unrolling
                 const long long slot = __shfl_sync(0xffffffffu, col_slot[c / 32], c % 32);
                 const float w = __shfl_sync(0xffffffffu, col_w[c / 32], c % 32);
-                if (slot >= 0 && nn < p.H) base[slot * p.H + nn] = w * (v0[i] + v1[i]);
+                const float d = SH::kTwoPlanes ? v0[i] + v1[i] : v0[i];
+                if (slot >= 0 && nn < p.H) base[slot * p.H + nn] = w * d;
               }
             }
           }
@@ -724,35 +801,39 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (cols contiguous), box {64 cols, box_rows}, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+// 2-D 16-bit tensor [rows, cols] (cols contiguous; bf16, or fp16 when f16),
+// box {64 cols, box_rows}, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+            dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, bool H16>
 cudaError_t launch_pass(const CUtensorMap* maps, const UmmaParams& p, int kernel_id, cudaStream_t s) {
-  const size_t smem = Smem<BN, STAGES, MODE>::kTotal;
-  static_assert(Smem<BN, STAGES, MODE>::kTotal <= 232448, "shared memory over the 227 KB limit");
-  cudaError_t e = cudaFuncSetAttribute(umma_ffn_kernel<BN, STAGES, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = Smem<BN, STAGES, MODE, H16>::kTotal;
+  static_assert(Smem<BN, STAGES, MODE, H16>::kTotal <= 232448, "shared memory over the 227 KB limit");
+  cudaError_t e = cudaFuncSetAttribute(umma_ffn_kernel<BN, STAGES, MODE, H16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   before_launch(kernel_id, s);
-  launch_pdl(umma_ffn_kernel<BN, STAGES, MODE>, dim3(sm_count()), dim3(kThreads), smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  launch_pdl(umma_ffn_kernel<BN, STAGES, MODE, H16>, dim3(sm_count()), dim3(kThreads), smem, s, maps[0], maps[1],
+             maps[2], maps[3], maps[4], maps[5], p);
   after_launch(kernel_id, s);
   return cudaGetLastError();
 }
 
 // Stage counts: gate/up stages hold two weight tiles and one token tile; down
-// stages one weight tile and the token tiles of both h planes.
-template <int BN, int ST_GU, int ST_DN, bool TM>
+// stages the weight tile(s) and the token tiles of both h planes, or of the
+// one fp16 plane (H16: the down weights' fp16 copy, a.w_down_f16).
+template <int BN, int ST_GU, int ST_DN, bool TM, bool H16>
 cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   static_assert(!TM || BN == BM, "token-major tiles hold 128 token rows");
   const int64_t R = a.T * a.k;
@@ -789,22 +870,34 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   }
   m[5] = m[4];
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = launch_pass<BN, ST_GU, TM ? kGateUpTM : kGateUp>(m, p, MOE_KERNEL_EXPERT_GATE_UP, s);
+  cudaError_t e = launch_pass<BN, ST_GU, TM ? kGateUpTM : kGateUp, H16>(m, p, MOE_KERNEL_EXPERT_GATE_UP, s);
   if (e != cudaSuccess) return e;
 
-  // pass 2: down projection of h_hi + h_lo, weighted scatter into slot order
-  ok = make_map(&m[0], a.w_down, (int64_t)a.E * a.H, a.I, BM) && make_map(&m[1], p.h_perm, R, a.I, BN) &&
-       make_map(&m[2], p.h_perm + R * a.I, R, a.I, BN);
-  if (shared)
-    ok = ok && make_map(&m[3], a.ws_down, a.H, a.Is, BM) && make_map(&m[4], p.h_shared, a.T, a.Is, BN) &&
-         make_map(&m[5], p.h_shared + a.T * a.Is, a.T, a.Is, BN);
-  else {
+  // pass 2: down projection of h (h_hi + h_lo, or the fp16 plane), weighted
+  // scatter into slot order
+  if (H16) {
+    ok = make_map(&m[0], a.w_down_f16, (int64_t)a.E * a.H, a.I, BM, true) &&
+         make_map(&m[1], p.h_perm, R, a.I, BN, true);
+    m[2] = m[1];
+    if (shared) {
+      ok = ok && make_map(&m[3], a.ws_down_f16, a.H, a.Is, BM, true) &&
+           make_map(&m[4], p.h_shared, a.T, a.Is, BN, true);
+      m[5] = m[4];
+    }
+  } else {
+    ok = make_map(&m[0], a.w_down, (int64_t)a.E * a.H, a.I, BM) && make_map(&m[1], p.h_perm, R, a.I, BN) &&
+         make_map(&m[2], p.h_perm + R * a.I, R, a.I, BN);
+    if (shared)
+      ok = ok && make_map(&m[3], a.ws_down, a.H, a.Is, BM) && make_map(&m[4], p.h_shared, a.T, a.Is, BN) &&
+           make_map(&m[5], p.h_shared + a.T * a.Is, a.T, a.Is, BN);
+  }
+  if (!shared) {
     m[3] = m[0];
     m[4] = m[1];
     m[5] = m[2];
   }
   if (!ok) return cudaErrorInvalidValue;
-  return launch_pass<BN, ST_DN, TM ? kDownTM : kDown>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
+  return launch_pass<BN, ST_DN, TM ? kDownTM : kDown, H16>(m, p, MOE_KERNEL_EXPERT_DOWN, s);
 }
 
 // Splits the fp32 router weight into three bf16 planes whose sum is the weight
@@ -886,11 +979,11 @@ cudaError_t launch_router_logits_tc(const moe_config& c, const uint16_t* x, int6
   m[4] = m[1];
   m[5] = m[1];
   constexpr int kStages = 8;
-  const size_t smem = Smem<kLogitsBN, kStages, kLogits>::kTotal;
-  e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  const size_t smem = Smem<kLogitsBN, kStages, kLogits, false>::kTotal;
+  e = cudaFuncSetAttribute(umma_ffn_kernel<kLogitsBN, kStages, kLogits, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  launch_pdl(umma_ffn_kernel<kLogitsBN, kStages, kLogits>, dim3(sm_count()), dim3(kThreads), smem, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
+  launch_pdl(umma_ffn_kernel<kLogitsBN, kStages, kLogits, false>, dim3(sm_count()), dim3(kThreads), smem, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int nk = 2;
@@ -920,11 +1013,19 @@ int umma_pick_bn(int64_t T, int k, int E) {
 
 cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cudaStream_t s) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  if (a.w_down_f16 != nullptr) {  // one fp16 h plane: smaller down stages, one more of them where it fits
+    switch (bn) {
+      case 32: return run_bn<32, 5, 5, false, true>(a, x_perm, s);
+      case 64: return run_bn<64, 5, 5, false, true>(a, x_perm, s);
+      case 128: return run_bn<128, 4, 4, false, true>(a, x_perm, s);
+      default: return run_bn<128, 4, 4, true, true>(a, x_perm, s);  // token-major
+    }
+  }
   switch (bn) {
-    case 32: return run_bn<32, 5, 5, false>(a, x_perm, s);
-    case 64: return run_bn<64, 5, 4, false>(a, x_perm, s);
-    case 128: return run_bn<128, 4, 4, false>(a, x_perm, s);
-    default: return run_bn<128, 4, 3, true>(a, x_perm, s);  // token-major
+    case 32: return run_bn<32, 5, 5, false, false>(a, x_perm, s);
+    case 64: return run_bn<64, 5, 4, false, false>(a, x_perm, s);
+    case 128: return run_bn<128, 4, 4, false, false>(a, x_perm, s);
+    default: return run_bn<128, 4, 3, true, false>(a, x_perm, s);  // token-major
   }
 }
 

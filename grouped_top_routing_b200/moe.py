@@ -17,7 +17,7 @@ library_path = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
-                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_RANGE"}
 SCORE = {"softmax": 0, "sigmoid": 1}
 KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "expert_down": 4, "combine": 5,
            "decode_fused": 6}
@@ -25,9 +25,11 @@ KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "e
 # Every entry point include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_launch_count", "moe_last_error",
-           "moe_permute_static", "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8")
+           "moe_permute_static", "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8",
+           "moe_convert_bf16_to_f16")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch up to this batch (shapes permitting)
+STREAM_MAX_TOKENS = 2  # ffn_path "auto": the streaming expert kernels up to this batch, the tensor cores above
 DECODE = {"auto": 0, "unfused": 1}
 WITHHOLD = {None: 0, "decode_routing": 1, "expert_accumulator": 2}
 
@@ -67,7 +69,8 @@ def config_from_workload(wl: dict) -> MoeConfig:
 
 
 class Options(ctypes.Structure):
-    """moe_options: per-call kernel choices, wait limit and timing hook."""
+    """moe_options: per-call kernel choices, wait limit, timing hook and the
+    optional fp16 copies of the down weights."""
     _fields_ = [
         ("ffn_path", ctypes.c_int32),
         ("decode_kernel", ctypes.c_int32),
@@ -76,21 +79,58 @@ class Options(ctypes.Structure):
         ("timer_start", ctypes.c_void_p),
         ("timer_stop", ctypes.c_void_p),
         ("test_withhold", ctypes.c_int32),
+        ("w_down_f16", ctypes.c_void_p),
+        ("ws_down_f16", ctypes.c_void_p),
     ]
 
 
 def options(ffn_path: str = "auto", decode: str = "auto", timer=None, wait_limit_ns: int = 0,
-            withhold=None) -> Options:
+            withhold=None, w_down_f16=None, ws_down_f16=None) -> Options:
     """Build a moe_options: ffn_path in FFN_PATHS, decode in DECODE, timer =
     (kernel name, start event, stop event) or None, withhold in WITHHOLD (a
-    test aid that makes one device wait run out)."""
-    o = Options(FFN_PATHS[ffn_path], DECODE[decode], int(wait_limit_ns), -1, None, None, WITHHOLD[withhold])
+    test aid that makes one device wait run out), and w_down_f16 /
+    ws_down_f16: fp16 copies of the down weights (convert_bf16_to_f16) for the
+    tensor-core down pass. The struct keeps the tensors alive."""
+    o = Options(FFN_PATHS[ffn_path], DECODE[decode], int(wait_limit_ns), -1, None, None, WITHHOLD[withhold],
+                None, None)
     if timer is not None:
         name, ev0, ev1 = timer
         o.timer_kernel = KERNELS[name]
         o.timer_start = ev0.cuda_event
         o.timer_stop = ev1.cuda_event
+    o.f16_tensors = (w_down_f16, ws_down_f16)
+    if w_down_f16 is not None:
+        o.w_down_f16 = w_down_f16.data_ptr()
+    if ws_down_f16 is not None:
+        o.ws_down_f16 = ws_down_f16.data_ptr()
     return o
+
+
+def _check_down_f16(opts, dev, n_routed: int, n_shared: int):
+    """Size, dtype and device of the fp16 down-weight copies an Options holds."""
+    if opts is None:
+        return
+    wd, wsd = getattr(opts, "f16_tensors", (None, None))
+    _require(wd, "w_down_f16", n_routed, torch.float16)
+    _require(wsd, "ws_down_f16", n_shared, torch.float16)
+    _on_device(dev, w_down_f16=wd, ws_down_f16=wsd)
+
+
+def convert_bf16_to_f16(w, out=None, stream=None):
+    """fp16 copy of bf16 weights (moe_convert_bf16_to_f16), checked: raises if
+    a value is beyond fp16's range. Blocking (it reads the count)."""
+    if not isinstance(w, torch.Tensor) or w.dtype != torch.bfloat16 or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("w: expected a contiguous CUDA bf16 tensor")
+    if out is None:
+        out = torch.empty(w.shape, dtype=torch.float16, device=w.device)
+    _require(out, "out", w.numel(), torch.float16)
+    _on_device(w.device, out=out)
+    bad = torch.empty(1, dtype=torch.int32, device=w.device)
+    _check(lib.moe_convert_bf16_to_f16(_p(w), _p(out), w.numel(), _p(bad), _stream(stream)))
+    n_bad = int(bad.item())
+    if n_bad:
+        raise MoeError(7, f"{n_bad} values are beyond fp16's range")
+    return out
 
 
 def _opts(o):
@@ -140,6 +180,7 @@ def _load():
         "moe_dense_mlp": (st, [ctypes.c_int32, ctypes.c_int32, vp, i64, vp, vp, vp, vp, sz, vp, op]),
         "moe_forward_q8": (st, [cfgp, vp, i64, vp, vp, vp, ctypes.POINTER(Q8Weights), vp, vp, vp, vp, vp, vp, sz, vp,
                                 op]),
+        "moe_convert_bf16_to_f16": (st, [vp, vp, i64, vp, vp]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -348,6 +389,7 @@ def moe_expert_ffn(cfg, x, expert_offsets, tok_of, topk_w, w_gate_up, w_down, ws
     _on_device(dev, x=x, x_perm=x_perm, expert_offsets=expert_offsets, tok_of=tok_of, topk_w=topk_w,
                w_gate_up=w_gate_up, w_down=w_down, ws_gate_up=ws_gate_up, ws_down=ws_down, y_slots=y_slots,
                shared_out=shared_out)
+    _check_down_f16(opts, dev, E * H * I, H * Is)
     _check_ws(ws, dev)
     if y_slots is None:
         y_slots = torch.empty((T * k, H), dtype=torch.float32, device=dev)
@@ -379,6 +421,8 @@ def moe_forward(cfg, x, router_w, expert_bias, w_gate_up, w_down, ws_gate_up, ws
     T = _rows(x, "x")
     k = c.num_experts_per_tok
     _check_block_tensors(c, T, x, router_w, expert_bias, logits_override, w_gate_up, w_down, ws_gate_up, ws_down, y)
+    _check_down_f16(opts, x.device, c.num_experts * c.hidden_size * c.moe_intermediate_size,
+                    c.hidden_size * shared_width(c))
     _check_ws(ws, x.device)
     if y is None:
         y = torch.empty_like(x)
@@ -420,6 +464,7 @@ def moe_dense_mlp(x, w_gate_up, w_down, ws: Workspace, y=None, stream=None, opts
     _require(w_down, "w_down", H * Id, torch.bfloat16)
     _require(y, "y", T * H, torch.bfloat16)
     _on_device(dev, x=x, w_gate_up=w_gate_up, w_down=w_down, y=y)
+    _check_down_f16(opts, dev, H * Id, 0)
     _check_ws(ws, dev)
     if y is None:
         y = torch.empty_like(x)

@@ -85,7 +85,8 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
   MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE_CHECK = 5, /* a device-side index check failed (see moe_check_device) */
-  MOE_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out */
+  MOE_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out */
+  MOE_ERR_RANGE = 7         /* a value left the range of an fp16 intermediate (see moe_options.w_down_f16) */
 } moe_status;
 
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_function;
@@ -144,6 +145,18 @@ typedef struct {
                              end in MOE_ERR_TIMEOUT after wait_limit_ns and
                              leave the workspace usable once moe_check_device
                              has reported. Any other value is rejected. */
+  /* Optional fp16 copies of the call's down-projection weights (layouts of
+   * w_down [E,H,I] and ws_down [H,Is], e.g. from moe_convert_bf16_to_f16),
+   * read by the tensor-core expert path only; NULL: bf16 throughout. With
+   * them, the SwiGLU product h is rounded to fp16 (11 significant bits)
+   * rather than split into two bf16 planes (about 16), and the down pass
+   * runs one fp16 MMA per k-step instead of two bf16 ones, with half the h
+   * bytes. An h beyond fp16's range (|h| >= 65520, or not finite) is
+   * recorded as MOE_ERR_RANGE in the workspace error word. ws_down_f16 is
+   * required when the block has a shared MLP. The bf16 weights stay
+   * required: the streaming kernels read them. */
+  const uint16_t* w_down_f16;
+  const uint16_t* ws_down_f16;
 } moe_options;
 
 /* Workspace bytes moe_permute, moe_expert_ffn and moe_forward need for up to
@@ -200,8 +213,10 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T
 /* Routed SwiGLU experts and the shared MLP ([ARCH], [SHARED], [GGUF]):
  *   F_e(v) = down_e( silu(gate_e v) * up_e v ),   silu(z) = z / (1 + exp(-z)),
  * fp32 accumulation. The SwiGLU product stays fp32 on the streaming (decode)
- * path and is rounded to bf16 on the tensor-core path, whose MMA operands are
- * bf16. Only experts with rows in expert_offsets are read.
+ * path. The tensor-core path's MMA operands are 16-bit: it keeps h as two bf16
+ * planes (h_hi = bf16(h), h_lo = bf16(h - h_hi)) whose products the down pass
+ * adds, or, given opts->w_down_f16, as one fp16 plane. Only experts with rows
+ * in expert_offsets are read.
  *   y_slots[t*k + j] = topk_w[t*k + j] * F_{e}(x_t)  (fp32) for the expert e
  *                      holding that slot (topk_w NULL: weight 1);
  *   shared_out[t]    = F_shared(x_t)  (fp32; when ws_gate_up is not NULL).
@@ -288,9 +303,20 @@ moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, c
 
 /* Synchronises `stream`, reads and clears the workspace error word (after an
  * error the whole 256-byte header is cleared, barrier state included). Returns
- * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT (first error recorded), or
- * MOE_ERR_CUDA if the stream itself reports an error. Blocking. */
+ * MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT or MOE_ERR_RANGE (the first
+ * error recorded), or MOE_ERR_CUDA if the stream itself reports an error.
+ * Blocking. */
 moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
+
+/* dst[i] = fp16(src[i]) for n bf16 values, round to nearest even: a one-time
+ * conversion of down-projection weights for moe_options.w_down_f16. Every
+ * bf16 value of magnitude 2^-14 .. 65504 is exact in fp16; smaller ones keep
+ * fp16's subnormal spacing of 2^-24 (an absolute error of at most 2^-25).
+ * *out_of_range (device int32, zeroed by the call) counts the values that
+ * become infinite or are not finite (|v| >= 65520, inf, NaN); weights with a
+ * nonzero count cannot use the fp16 path. src and dst may not overlap. */
+moe_status moe_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, int32_t* out_of_range,
+                                   void* stream);
 
 /* Number of this library's kernel launches made by the calling thread since
  * the library was loaded (a host-side counter). */

@@ -179,6 +179,8 @@ OPTION_BAD = [
     ("timer_kernel", -2, "timer_kernel"),
     ("timer_kernel", 0, "timer events"),   # a kernel id without its events
     ("test_withhold", 3, "test_withhold"),
+    ("w_down_f16", (1 << 20) + 8, "w_down_f16"),      # misaligned
+    ("ws_down_f16", 1 << 20, "ws_down_f16"),          # the shared copy without the routed one
 ]
 
 
@@ -195,6 +197,44 @@ def test_options_rejected_before_launch(M, field, value, text):
     assert st == 1 and text in M.last_error(), (st, M.last_error())
     st = M.lib.moe_dense_mlp(4096, 9216, fake, 4, fake, fake, fake, fake, 1 << 40, None, ctypes.byref(o))
     assert st == 1 and text in M.last_error()
+    assert M.lib.moe_launch_count() == n0
+
+
+def test_fp16_down_options_need_the_shared_copy(M):
+    # A block with a shared MLP needs both fp16 copies; without a shared MLP
+    # (dense MLP) the routed copy alone is enough.
+    c = _cfg(M)
+    assert M.shared_width(c) > 0
+    fake = ctypes.c_void_p(1 << 20)
+    o = M.options()
+    o.w_down_f16 = 1 << 20
+    n0 = M.lib.moe_launch_count()
+    st = M.lib.moe_forward(ctypes.byref(c), fake, 4, fake, None, None, fake, fake, fake, fake, fake, None, None,
+                           fake, 1 << 40, None, ctypes.byref(o))
+    assert st == 1 and "ws_down_f16 is NULL" in M.last_error(), M.last_error()
+    st = M.lib.moe_expert_ffn(ctypes.byref(c), 4, fake, None, fake, fake, None, fake, fake, fake, fake, fake, fake,
+                              fake, 1 << 40, None, ctypes.byref(o))
+    assert st == 1 and "ws_down_f16 is NULL" in M.last_error(), M.last_error()
+    assert M.lib.moe_launch_count() == n0
+    w = _q8(M, shared=False)
+    st = M.lib.moe_forward_q8(ctypes.byref(c), fake, 4, fake, None, None, ctypes.byref(w), fake, fake, fake, None,
+                              None, fake, 1 << 40, None, ctypes.byref(o))
+    assert st == 1 and "moe_forward_q8" in M.last_error(), M.last_error()
+
+
+def test_convert_rejects_before_launch(M):
+    fake = 1 << 20
+    n0 = M.lib.moe_launch_count()
+    cnt = ctypes.c_void_p(fake)
+    assert M.lib.moe_convert_bf16_to_f16(ctypes.c_void_p(fake), ctypes.c_void_p(fake * 2), -1, cnt, None) == 1
+    assert "negative" in M.last_error()
+    # dst starts inside src's range
+    assert M.lib.moe_convert_bf16_to_f16(ctypes.c_void_p(fake), ctypes.c_void_p(fake + 64), 1000, cnt, None) == 1
+    assert "overlap" in M.last_error()
+    assert M.lib.moe_convert_bf16_to_f16(ctypes.c_void_p(fake), ctypes.c_void_p(fake + 8 * 1024), 16, None, None) == 1
+    assert "out_of_range" in M.last_error()
+    assert M.lib.moe_convert_bf16_to_f16(ctypes.c_void_p(fake + 2), ctypes.c_void_p(fake * 2), 16, cnt, None) == 1
+    assert "src" in M.last_error()
     assert M.lib.moe_launch_count() == n0
 
 

@@ -207,9 +207,21 @@ FFN_CASES = [
 ]
 
 
-@pytest.fixture(params=["streaming", "tensor_cores"])
+@pytest.fixture(params=["streaming", "tensor_cores", "tensor_cores_f16"])
 def path(request, M):
     return request.param
+
+
+def _path_opts(M, path, inp):
+    """moe_options for an expert path, and the inputs the oracle must see: on
+    the fp16 down path the down weights are the fp16 copies the kernels read
+    (equal to the bf16 ones except below 2^-14 in magnitude)."""
+    if path != "tensor_cores_f16":
+        return M.options(ffn_path=path), inp
+    wd = M.convert_bf16_to_f16(inp["w_down"])
+    wsd = None if inp["ws_down"] is None else M.convert_bf16_to_f16(inp["ws_down"])
+    return (M.options(ffn_path="tensor_cores", w_down_f16=wd, ws_down_f16=wsd),
+            dict(inp, w_down=wd, ws_down=wsd))
 
 
 @pytest.mark.parametrize("name,over", FFN_CASES, ids=[c[0] for c in FFN_CASES])
@@ -227,10 +239,11 @@ def test_expert_ffn(M, name, over, path):
     d_w = torch.from_numpy(w).to(DEV)
     off, _, tok_of, _ = M.moe_permute(wl, d_idx, ws)
     has_shared = inp["ws_gate_up"] is not None
+    opts, inp_o = _path_opts(M, path, inp)
     y_slots, shared = M.moe_expert_ffn(wl, inp["x"], off, tok_of, d_w.reshape(-1), inp["w_gate_up"], inp["w_down"],
-                                       ws, ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"],
-                                       opts=M.options(ffn_path=path))
+                                       ws, ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"], opts=opts)
     ws.check()
+    inp = inp_o
     X = O.as_f64(inp["x"])
     I = wl["moe_intermediate_size"]
     ref = np.zeros((T * k, H))
@@ -256,7 +269,7 @@ def _oracle_rows(M, inp, rows):
     return sub
 
 
-def _forward_and_compare(M, wl, inp, tokens=None, logits=None, opts=None, constructed_ties=0):
+def _forward_and_compare(M, wl, inp, tokens=None, logits=None, opts=None, constructed_ties=0, oracle_inp=None):
     """Run moe_forward on all tokens and compare the output of every token in
     `tokens` (default: all) with the oracle.
 
@@ -266,7 +279,9 @@ def _forward_and_compare(M, wl, inp, tokens=None, logits=None, opts=None, constr
     line of their own, to the same bars. Tokens whose routing flipped (only
     possible when each side computes its own router logits, and only inside a
     1e-5 gap) are compared with the oracle block evaluated on the GPU's
-    routing, again on a line of their own. The near-tie count is bounded."""
+    routing, again on a line of their own. The near-tie count is bounded.
+    oracle_inp: the weights the oracle uses, when they differ from the bf16
+    ones passed to moe_forward (the fp16 down-weight copies)."""
     T = inp["tokens"]
     ws = M.Workspace(wl, T)
     Ld = None if logits is None else torch.from_numpy(logits).to(DEV)
@@ -298,7 +313,7 @@ def _forward_and_compare(M, wl, inp, tokens=None, logits=None, opts=None, constr
     y_rows = O.as_f64(y[torch.from_numpy(rows).to(DEV)])
     same = ~differ
     if same.any():
-        ref = O.moe_block(_oracle_rows(M, inp, rows[same]), wl, logits=L[same])["y"]
+        ref = O.moe_block(_oracle_rows(M, oracle_inp or inp, rows[same]), wl, logits=L[same])["y"]
         got = y_rows[same]
         plain = ~near[same]
         if plain.any():
@@ -306,7 +321,8 @@ def _forward_and_compare(M, wl, inp, tokens=None, logits=None, opts=None, constr
         if (~plain).any():
             S.compare(got[~plain], ref[~plain], f"{name} T={T} near-tie: {int((~plain).sum())} tokens")
     if differ.any():
-        ref = O.moe_block(_oracle_rows(M, inp, rows[differ]), wl, idx=g_idx[differ], w=g_w[differ])["y"]
+        ref = O.moe_block(_oracle_rows(M, oracle_inp or inp, rows[differ]), wl, idx=g_idx[differ],
+                          w=g_w[differ])["y"]
         S.compare(y_rows[differ], ref, f"{name} T={T} routing flipped inside 1e-5: {int(differ.sum())} tokens, "
                                        "oracle on the GPU's routing")
     print(f"{name}: near-tie {int(near.sum())} (bound {bound}), flipped {int(differ.sum())}, compared {len(rows)}")
@@ -326,7 +342,8 @@ FORWARD_CASES = [
 def test_forward_matches_oracle(M, name, over, path):
     wl, inp = _inputs(name)
     wl = dict(wl, **over, name=f"{name}[{path}]")
-    _forward_and_compare(M, wl, inp, opts=M.options(ffn_path=path))
+    opts, inp_o = _path_opts(M, path, inp)
+    _forward_and_compare(M, wl, inp, opts=opts, oracle_inp=inp_o)
 
 
 @pytest.mark.parametrize("T", [1, 8, 32])
@@ -336,25 +353,34 @@ def test_forward_decode_batches(M, T):
     _forward_and_compare(M, dict(wl, name=f"decode_t{T}"), sub)
 
 
-@pytest.mark.parametrize("name", ["ling26_flash_prefill_t8192", "ling26_flash_prefill_t32768"])
-def test_forward_prefill_every_token(M, name):
+@pytest.mark.parametrize("name,path", [("ling26_flash_prefill_t8192", "auto"),
+                                       ("ling26_flash_prefill_t32768", "auto"),
+                                       ("ling26_flash_prefill_t8192", "tensor_cores_f16"),
+                                       ("ling26_flash_prefill_t32768", "tensor_cores_f16")])
+def test_forward_prefill_every_token(M, name, path):
     # Full size, every token compared: every (expert, token tile) of both
-    # expert passes, ragged last tiles included, holds compared rows.
+    # expert passes, ragged last tiles included, holds compared rows; on the
+    # bf16 (two h planes) and the fp16 down path.
     wl, inp = _inputs(name)
-    _forward_and_compare(M, dict(wl, name=name), inp)
+    opts, inp_o = _path_opts(M, path, inp)
+    _forward_and_compare(M, dict(wl, name=f"{name}[{path}]"), inp, opts=opts, oracle_inp=inp_o)
 
 
-@pytest.mark.parametrize("over", [{}, dict(norm_topk_prob=False, routed_scaling_factor=1.0)])
-def test_forward_skew_ties_every_token(M, over):
+@pytest.mark.parametrize("over,path", [({}, "auto"), (dict(norm_topk_prob=False, routed_scaling_factor=1.0), "auto"),
+                                       ({}, "tensor_cores_f16"),
+                                       (dict(norm_topk_prob=False, routed_scaling_factor=1.0), "tensor_cores_f16")])
+def test_forward_skew_ties_every_token(M, over, path):
     # Skewed routing with 1% exact ties (given logits): every token compared.
     wl, inp = _inputs("ling30_flash_skew_t16384")
     wl = dict(wl, **over)
+    opts, inp_o = _path_opts(M, path, inp)
     T, E, k = inp["tokens"], wl["num_experts"], wl["num_experts_per_tok"]
     bias = _np_bias(inp)
     L = G.random_logits(T, E, S.logit_std(wl), seed=2).numpy()
     toks, pairs = S.add_exact_ties(L, bias, k)
     S.check_ties_constructed(L, bias, wl, toks, pairs)
-    _forward_and_compare(M, dict(wl, name="skew"), inp, logits=L, constructed_ties=len(toks))
+    _forward_and_compare(M, dict(wl, name=f"skew[{path}]"), inp, logits=L, constructed_ties=len(toks), opts=opts,
+                         oracle_inp=inp_o)
 
 
 def test_forward_skew_router_projection(M):
