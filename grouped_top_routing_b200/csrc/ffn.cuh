@@ -30,6 +30,9 @@ struct FfnArgs {
   // h as one fp16 plane and multiplies fp16 operands in the down pass
   const uint16_t* w_down_f16;   // [E, H, I]
   const uint16_t* ws_down_f16;  // [H, Is]; set whenever ws_gate_up is
+  // with the fp16 down weights: write the routed slot rows as fp16 (y_slots
+  // then holds [T*k, H] uint16_t; shared_out stays fp32)
+  bool slots_f16;
   void* h_perm;               // [T*k, I]: fp32 (streaming path), two bf16 planes or one fp16 plane (tensor cores)
   void* h_shared;             // [T, Is]: same element type as h_perm
   float* y_slots;             // [T*k, H]
@@ -42,6 +45,9 @@ struct FfnArgs {
 };
 
 cudaError_t launch_gemv_ffn(const FfnArgs& a, cudaStream_t s);
+// y[t] = bf16( sum_j y16[t*k + j] + shared_out[t] ) for fp16 slot rows
+cudaError_t launch_combine16(const uint16_t* y16, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
+                             cudaStream_t s);
 int umma_pick_bn(int64_t T, int k, int E);
 cudaError_t launch_umma_ffn(const FfnArgs& a, const uint16_t* x_perm, int bn, cudaStream_t s);
 

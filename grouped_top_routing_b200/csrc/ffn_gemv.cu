@@ -19,6 +19,8 @@
 // shuffles. Tokens are taken MT at a time (MT follows the batch, up to 8); an
 // expert with more rows streams its weights again per group of MT (those
 // re-reads hit L2), which is why larger batches take the tensor-core path.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "ffn.cuh"
 
@@ -388,6 +390,48 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   }
 }
 
+// The same with fp16 slot rows (the tensor-core path on fp16 down weights):
+// y[t] = bf16( sum_j float(y16[t*k + j]) + shared_out[t] ); one thread per 8
+// outputs (16-byte slot loads).
+__global__ void __launch_bounds__(256) combine16_kernel(const uint16_t* __restrict__ y16,
+                                                        const float* __restrict__ shared_out, int64_t T, int k, int H,
+                                                        uint16_t* __restrict__ y) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int nv = H / 8;
+  const int64_t n = T * nv;
+  const uint4* ys = reinterpret_cast<const uint4*>(y16);
+  const float4* sh = reinterpret_cast<const float4*>(shared_out);
+  uint4* out = reinterpret_cast<uint4*>(y);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nv;
+    const int v = (int)(i - t * nv);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const uint4 f = __ldg(ys + (t * k + j) * nv + v);
+      const uint32_t w4[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += __half2float(__ushort_as_half((unsigned short)(w4[q] & 0xFFFFu)));
+        acc[2 * q + 1] += __half2float(__ushort_as_half((unsigned short)(w4[q] >> 16)));
+      }
+    }
+    if (sh != nullptr) {
+      const float4 a = __ldg(sh + 2 * i), b = __ldg(sh + 2 * i + 1);
+      acc[0] += a.x;
+      acc[1] += a.y;
+      acc[2] += a.z;
+      acc[3] += a.w;
+      acc[4] += b.x;
+      acc[5] += b.y;
+      acc[6] += b.z;
+      acc[7] += b.w;
+    }
+    out[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                        pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
 }  // namespace
 
 // One resident wave: as many 256-thread blocks as the kernel's register use
@@ -436,6 +480,19 @@ cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_
   if (blocks > cap) blocks = cap;
   before_launch(MOE_KERNEL_COMBINE, s);
   launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(256), 0, s, y_slots, shared_out, T, k, H, y);
+  after_launch(MOE_KERNEL_COMBINE, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine16(const uint16_t* y16, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
+                             cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t n = T * (H / 8);
+  int64_t blocks = (n + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  before_launch(MOE_KERNEL_COMBINE, s);
+  launch_pdl(combine16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, y16, shared_out, T, k, H, y);
   after_launch(MOE_KERNEL_COMBINE, s);
   return cudaGetLastError();
 }

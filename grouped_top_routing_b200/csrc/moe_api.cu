@@ -334,11 +334,14 @@ bool use_tensor_cores(const moe_config& c, int64_t T) {
 Q8Mat q8mat(const moe_q8_matrix& m) { return Q8Mat{m.q, m.scale, m.bias}; }
 
 // q8: 8-bit affine expert weights (dequantised by the streaming kernels), or
-// null for bf16 weights.
+// null for bf16 weights. slots16: when given, the caller takes fp16 slot rows
+// (y_slots as [T*k, H] uint16_t) where the fp16 down path runs, and learns
+// here whether it did.
 moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint16_t* x_perm,
                    const int32_t* offsets, const int32_t* tok_of, const float* topk_w, const uint16_t* wgu,
                    const uint16_t* wd, const uint16_t* swgu, const uint16_t* swd, float* y_slots, float* shared_out,
-                   void* ws, bool active_ready, cudaStream_t s, const moe_q8_weights* q8 = nullptr) {
+                   void* ws, bool active_ready, cudaStream_t s, const moe_q8_weights* q8 = nullptr,
+                   bool* slots16 = nullptr) {
   const Layout L = layout(c, T);
   WsHeader* hdr = at<WsHeader>(ws, L.hdr);
   int32_t* active = at<int32_t>(ws, L.active);
@@ -386,6 +389,8 @@ moe_status run_ffn(const moe_config& c, int64_t T, const uint16_t* x, const uint
     if (t_opts != nullptr && t_opts->w_down_f16 != nullptr) {
       a.w_down_f16 = t_opts->w_down_f16;
       a.ws_down_f16 = a.ws_gate_up != nullptr ? t_opts->ws_down_f16 : nullptr;
+      a.slots_f16 = slots16 != nullptr;
+      if (slots16 != nullptr) *slots16 = true;
     }
     if (x_perm == nullptr) {  // the tensor-core path reads expert rows contiguously
       uint16_t* xp = at<uint16_t>(ws, L.x_perm);
@@ -689,9 +694,14 @@ moe_status moe_forward(const moe_config* cfg, const uint16_t* x, int64_t T, cons
   if (e != cudaSuccess) return cuda_fail(e, "permute");
   float* y_slots = at<float>(ws, L.y_slots);
   float* shared_out = has_shared ? at<float>(ws, L.shared_out) : nullptr;
+  // on the fp16 down path the routed slot rows are fp16 (half the bytes
+  // written by the down pass and read by the combine)
+  bool slots16 = false;
   MOE_TRY(run_ffn(c, T, x, x_perm, offsets, tok_of, w, w_gate_up, w_down, has_shared ? ws_gate_up : nullptr,
-                  has_shared ? ws_down : nullptr, y_slots, shared_out, ws, true, s));
-  e = launch_combine(y_slots, shared_out, T, c.num_experts_per_tok, c.hidden_size, y, s);
+                  has_shared ? ws_down : nullptr, y_slots, shared_out, ws, true, s, nullptr, &slots16));
+  e = slots16 ? launch_combine16(reinterpret_cast<const uint16_t*>(y_slots), shared_out, T, c.num_experts_per_tok,
+                                 c.hidden_size, y, s)
+              : launch_combine(y_slots, shared_out, T, c.num_experts_per_tok, c.hidden_size, y, s);
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   return MOE_OK;
 }

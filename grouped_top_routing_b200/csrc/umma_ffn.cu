@@ -89,6 +89,7 @@ struct UmmaParams {
   int ksplit, kper, kbH;
   uint64_t wait_ns;  // bound on every mbarrier wait
   int withhold;      // test aid: 1 = never hand the first accumulator to the epilogue
+  int slots16;       // H16 DOWN: routed slot rows are fp16 (y_slots holds uint16_t), the shared rows fp32
 };
 
 // ----------------------------------------------------------------------------
@@ -665,7 +666,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           // stores touched 32 lines per instruction and left the pass
           // store-bound at twice its MMA time).
           constexpr int kCW = L::kCW, G = kCW / 4, RPI = 32 / G;  // lanes per row, rows per instruction
+          static_assert(!H16 || L::kStgRow >= 144, "fp16 slot rows stage 64 columns (128 bytes) per row");
           const int n0 = t.nb * 2 * BM;
+          if (H16 && p.slots16 && !t.shared) {
+            // fp16 slot rows: 64 columns (128 bytes) per row and chunk, 8 lanes per row
+            const long long dst16 = (tm_valid && tm_slot >= 0) ? tm_slot * (long long)p.H : -1ll;
+            uint16_t* o16 = reinterpret_cast<uint16_t*>(p.y_slots);
+            uint8_t* stg16 = staging + (size_t)q * 32 * L::kStgRow;
+            const int sub8 = lane >> 3, part8 = lane & 7;
+            bool fin = true;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 2 * BM; c0 += 64) {
+              float v[64];
+#pragma unroll
+              for (int j = 0; j < 64; j += 16) tmem_ld16(taddr + c0 + j, v + j);
+              const int n = n0 + c0;
+              if (n >= p.H) continue;  // warp-uniform
+              uint32_t h2[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const uint16_t lo = f32_to_f16(tm_w * v[2 * i]), hi = f32_to_f16(tm_w * v[2 * i + 1]);
+                fin = fin && f16_finite(lo) && f16_finite(hi);
+                h2[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+              }
+              if (n + 64 <= p.H) {
+                __syncwarp();  // the previous chunk's reads of the tile are done
+                uint4* d = reinterpret_cast<uint4*>(stg16 + lane * L::kStgRow);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d[i] = make_uint4(h2[4 * i], h2[4 * i + 1], h2[4 * i + 2], h2[4 * i + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int r0 = 0; r0 < 32; r0 += 4) {
+                  const int r = r0 + sub8;
+                  const long long dst = __shfl_sync(0xffffffffu, dst16, r);
+                  const uint4 val = *reinterpret_cast<const uint4*>(stg16 + r * L::kStgRow + part8 * 16);
+                  if (dst >= 0) *reinterpret_cast<uint4*>(o16 + dst + n + part8 * 8) = val;
+                }
+              } else if (dst16 >= 0) {  // ragged last chunk of the hidden size: per element
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                  if (n + i < p.H) o16[dst16 + n + i] = (uint16_t)(h2[i / 2] >> (16 * (i & 1)));
+              }
+            }
+            if (!fin && dst16 >= 0) record_error(p.hdr, MOE_ERR_RANGE, (int)(t.r0 + tm_tok));
+          } else {
           // the destination row offset of this lane's row, or -1 when the row is absent
           const long long my_dst = !(tm_valid && tm_slot >= 0)
                                        ? -1ll
@@ -699,6 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < kCW; ++i)
                 if (n + i < p.H) obase[my_dst + n + i] = tm_w * v[i];
             }
+          }
           }
         }
 #pragma unroll
@@ -753,7 +798,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const long long slot = __shfl_sync(0xffffffffu, col_slot[c / 32], c % 32);
                 const float w = __shfl_sync(0xffffffffu, col_w[c / 32], c % 32);
                 const float d = SH::kTwoPlanes ? v0[i] + v1[i] : v0[i];
-                if (slot >= 0 && nn < p.H) base[slot * p.H + nn] = w * d;
+                if (slot >= 0 && nn < p.H) {
+                  if (H16 && p.slots16 && !t.shared) {
+                    const uint16_t hv = f32_to_f16(w * d);
+                    if (!f16_finite(hv)) record_error(p.hdr, MOE_ERR_RANGE, (int)slot);
+                    reinterpret_cast<uint16_t*>(p.y_slots)[slot * p.H + nn] = hv;
+                  } else {
+                    base[slot * p.H + nn] = w * d;
+                  }
+                }
               }
             }
           }
@@ -857,6 +910,7 @@ cudaError_t run_bn(const FfnArgs& a, const uint16_t* x_perm, cudaStream_t s) {
   p.shared_out = a.shared_out;
   p.wait_ns = opt_wait_ns();
   p.withhold = opt_withhold() == 2 ? 1 : 0;
+  p.slots16 = (H16 && a.slots_f16) ? 1 : 0;
   // maps: A routed, B routed, B2 routed, A shared, B shared, B2 shared
   CUtensorMap m[6];
 

@@ -92,3 +92,26 @@ def test_swiglu_beyond_fp16_is_reported(M, tokens):
     M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
                   inp["ws_gate_up"], inp["ws_down"], ws, opts=opts)
     ws.check()
+
+
+@pytest.mark.parametrize("tokens,hidden", [(40, 200), (90, 64), (600, 200), (600, 136)])
+def test_forward_f16_ragged_shapes(M, tokens, hidden):
+    # The whole block on the fp16 down path, where the routed slot rows are
+    # fp16 too: weight-major tiles (40, 90 tokens) and token-major tiles (600),
+    # hidden sizes that leave a ragged last 64-column chunk, against the oracle
+    # on the fp16 weights.
+    import support as S
+    from oracle import moe_oracle as O
+    wl = G.tiny_workload(tokens=tokens, hidden_size=hidden, num_experts=6, num_experts_per_tok=2,
+                         moe_intermediate_size=136, shared_width=272, num_shared_experts=2, name="f16-forward")
+    inp = G.make_inputs(wl, seed=6, device=DEV)
+    wd = M.convert_bf16_to_f16(inp["w_down"])
+    wsd = M.convert_bf16_to_f16(inp["ws_down"])
+    L = G.random_logits(tokens, wl["num_experts"], 1.0, seed=7).numpy()
+    ws = M.Workspace(wl, tokens)
+    y = M.moe_forward(wl, inp["x"], inp["router_w"], inp["expert_bias"], inp["w_gate_up"], inp["w_down"],
+                      inp["ws_gate_up"], inp["ws_down"], ws, logits_override=torch.from_numpy(L).to(DEV),
+                      opts=M.options(ffn_path="tensor_cores", w_down_f16=wd, ws_down_f16=wsd))
+    ws.check()
+    ref = O.moe_block(dict(inp, w_down=wd, ws_down=wsd), wl, logits=L)["y"]
+    S.compare(O.as_f64(y), ref, f"f16 forward T={tokens} H={hidden}")
