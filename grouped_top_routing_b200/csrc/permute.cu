@@ -12,8 +12,9 @@
 //   count   : per tile, popcount of each expert's mask -> tile_cnt[tile][e]
 //   scan    : one block: expert totals, exclusive scan -> offsets, per-tile
 //             bases tile_base[tile][e], compacted list of experts with rows
-//   scatter : per tile, rebuild masks, row = base + rank; write row_of/tok_of;
-//             copy x rows into x_perm when asked
+//   scatter : per tile, rebuild masks, row = base + rank; write row_of/tok_of
+//   rows    : when asked, x rows into x_perm in token order (each row of x
+//             read once and written to the rows of its k slots)
 // A single tile (T <= 128) runs all three steps in one block.
 #include "common.cuh"
 
@@ -108,6 +109,29 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int32_t* __restr
     const int64_t slot = tok_of[r];
     if (slot < 0 || slot >= T * k) continue;
     dst[i] = __ldg(src + (slot / k) * nv + v);
+  }
+}
+
+// The same copy in token order, when row_of is known: each 16-byte chunk of
+// x[t] is read once and written to the k rows row_of[t*k + j] (x read once
+// instead of k times).
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const int32_t* __restrict__ row_of, int k, int64_t T,
+                                                           const uint16_t* __restrict__ x, int H,
+                                                           uint16_t* __restrict__ x_perm) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int nv = H / 8;
+  const int64_t n = T * nv, R = T * k;
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+  uint4* dst = reinterpret_cast<uint4*>(x_perm);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nv;
+    const int v = (int)(i - t * nv);
+    const uint4 val = __ldg(src + i);
+    for (int j = 0; j < k; ++j) {
+      const int64_t r = row_of[t * k + j];
+      if (r >= 0 && r < R) dst[r * nv + v] = val;
+    }
   }
 }
 
@@ -259,13 +283,13 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, int64_t T, c
     launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, tile_cnt, n_tiles, E, offsets, tile_base, active, hdr);
     launch_pdl(permute_scatter_kernel, dim3(n_tiles), dim3(kTile), mask_bytes, s, idx, T, k, E, tile_base, row_of, tok_of);
   }
-  if (x_perm != nullptr) {
-    const int64_t chunks = T * k * (H / 8);
+  if (x_perm != nullptr) {  // row_of is known here: copy in token order, each x row read once
+    const int64_t chunks = T * (H / 8);
     int64_t blocks = (chunks + 255) / 256;
     const int64_t cap = (int64_t)sm_count() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, offsets, E, tok_of, k, T, x, H, x_perm);
+    launch_pdl(scatter_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, row_of, k, T, x, H, x_perm);
     ++nk;
   }
   after_launch(MOE_KERNEL_PERMUTE, s, nk);

@@ -257,6 +257,29 @@ def test_expert_ffn(M, name, over, path):
         S.compare(O.as_f64(shared), O.swiglu_mlp(X, Wg, Wu, Wd), f"{name} [{path}] shared", bf16_out=False)
 
 
+@pytest.mark.parametrize("name", ["tiny_bn64", "tiny_token_major"])
+def test_expert_ffn_reads_given_x_perm(M, name):
+    # moe_expert_ffn with a caller's x_perm reads the permuted rows as tiles;
+    # without it the gate/up pass gathers the rows from x (the case above):
+    # both must give the same slot rows bit for bit.
+    over = dict(FFN_CASES)[name]
+    wl = G.tiny_workload(**over)
+    inp = S.inputs_to(G.make_inputs(wl, seed=3, device="cpu"), DEV)
+    T, E = inp["tokens"], wl["num_experts"]
+    L = G.random_logits(T, E, S.logit_std(wl), seed=8).numpy()
+    idx, w = O.route(L, _np_bias(inp), wl)
+    ws = M.Workspace(wl, T)
+    off, _, tok_of, x_perm = M.moe_permute(wl, torch.from_numpy(idx).to(DEV), ws, x=inp["x"], want_x_perm=True)
+    d_w = torch.from_numpy(w).to(DEV).reshape(-1)
+    args = (wl, inp["x"], off, tok_of, d_w, inp["w_gate_up"], inp["w_down"], ws)
+    kw = dict(ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"], opts=M.options(ffn_path="tensor_cores"))
+    a_slots, a_sh = M.moe_expert_ffn(*args, **kw)
+    a_slots, a_sh = a_slots.clone(), a_sh.clone()
+    b_slots, b_sh = M.moe_expert_ffn(*args, x_perm=x_perm, **kw)
+    ws.check()
+    assert torch.equal(a_slots, b_slots) and torch.equal(a_sh, b_sh)
+
+
 # ---------------------------------------------------------------------------
 # whole block
 # ---------------------------------------------------------------------------
