@@ -33,6 +33,12 @@ cudaError_t launch_active_from_offsets(const int32_t* offsets, int E, int32_t* a
 cudaError_t launch_identity_route(int64_t T, int32_t* offsets, int32_t* tok_of, float* w, cudaStream_t s);
 cudaError_t launch_combine(const float* y_slots, const float* shared_out, int64_t T, int k, int H, uint16_t* y,
                            cudaStream_t s);
+cudaError_t launch_ep_send(const int32_t* offsets, int E, const int32_t* tok_of, const float* topk_w, int64_t R_max,
+                           int64_t* counts, float* row_w, cudaStream_t s);
+cudaError_t launch_ep_recv(const int64_t* recv_counts, int nseg, int n_local, int64_t R, int32_t* local_expert,
+                           cudaStream_t s);
+cudaError_t launch_ep_scatter_back(const float* y_perm, const int32_t* tok_of, int64_t R, int64_t n_slots, int H,
+                                   float* y_slots, cudaStream_t s);
 cudaError_t launch_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, int32_t* bad_count,
                                        cudaStream_t s);
 cudaError_t launch_gather_rows(const int32_t* offsets, int E, const int32_t* tok_of, int k, int64_t T,
@@ -723,6 +729,48 @@ moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream) {
     return fail(MOE_ERR_RANGE, "a SwiGLU product left fp16's range (expert row %d); use the bf16 down weights",
                 word[1]);
   return fail(MOE_ERR_DEVICE_CHECK, "device index check failed (index %d)", word[1]);
+}
+
+moe_status moe_ep_send(const moe_config* cfg, int64_t T, const int32_t* expert_offsets, const int32_t* tok_of,
+                       const float* topk_w, int64_t* counts, float* row_w, void* stream) {
+  MOE_TRY(validate_config(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_ptr("expert_offsets", expert_offsets, 4, true));
+  MOE_TRY(check_ptr("counts", counts, 8, true));
+  MOE_TRY(check_ptr("tok_of", tok_of, 4, T > 0));
+  MOE_TRY(check_ptr("topk_w", topk_w, 4, T > 0));
+  MOE_TRY(check_ptr("row_w", row_w, 4, T > 0));
+  cudaError_t e = launch_ep_send(expert_offsets, cfg->num_experts, tok_of, topk_w, T * cfg->num_experts_per_tok,
+                                 counts, row_w, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel send lists");
+  return MOE_OK;
+}
+
+moe_status moe_ep_recv(const int64_t* recv_counts, int32_t P, int32_t n_local, int64_t R_recv, int32_t* local_expert,
+                       void* stream) {
+  if (P < 1 || n_local < 1 || (int64_t)P * n_local > 1024)
+    return fail(MOE_ERR_INVALID_ARG, "P = %d, n_local = %d: need P, n_local >= 1 and P * n_local <= 1024", P,
+                n_local);
+  if (R_recv < 0) return fail(MOE_ERR_INVALID_ARG, "R_recv = %lld is negative", (long long)R_recv);
+  MOE_TRY(check_ptr("recv_counts", recv_counts, 8, true));
+  MOE_TRY(check_ptr("local_expert", local_expert, 4, R_recv > 0));
+  cudaError_t e = launch_ep_recv(recv_counts, P * n_local, n_local, R_recv, local_expert, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel receive list");
+  return MOE_OK;
+}
+
+moe_status moe_ep_scatter_back(const float* y_perm, const int32_t* tok_of, int64_t R, int64_t n_slots, int32_t H,
+                               float* y_slots, void* stream) {
+  if (R < 0 || n_slots < 0) return fail(MOE_ERR_INVALID_ARG, "R = %lld, n_slots = %lld", (long long)R,
+                                        (long long)n_slots);
+  if (H < 4 || H % 4 != 0 || H > kMaxHidden)
+    return fail(MOE_ERR_INVALID_ARG, "H = %d is not a multiple of 4 in [4, %d]", H, kMaxHidden);
+  MOE_TRY(check_ptr("y_perm", y_perm, 16, R > 0));
+  MOE_TRY(check_ptr("tok_of", tok_of, 4, R > 0));
+  MOE_TRY(check_ptr("y_slots", y_slots, 16, R > 0));
+  cudaError_t e = launch_ep_scatter_back(y_perm, tok_of, R, n_slots, H, y_slots, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel scatter back");
+  return MOE_OK;
 }
 
 moe_status moe_convert_bf16_to_f16(const uint16_t* src, uint16_t* dst, int64_t n, int32_t* out_of_range,

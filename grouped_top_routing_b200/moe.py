@@ -26,7 +26,7 @@ KERNELS = {"router_logits": 0, "route": 1, "permute": 2, "expert_gate_up": 3, "e
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_router_logits", "moe_route", "moe_permute",
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_check_device", "moe_launch_count", "moe_last_error",
            "moe_permute_static", "moe_dense_mlp_workspace_size", "moe_dense_mlp", "moe_forward_q8",
-           "moe_convert_bf16_to_f16")
+           "moe_convert_bf16_to_f16", "moe_ep_send", "moe_ep_recv", "moe_ep_scatter_back")
 FFN_PATHS = {"auto": 0, "streaming": 1, "tensor_cores": 2}
 FUSED_DECODE_MAX_TOKENS = 2  # moe_forward runs the whole block as one launch up to this batch (shapes permitting)
 STREAM_MAX_TOKENS = 2  # ffn_path "auto": the streaming expert kernels up to this batch, the tensor cores above
@@ -181,6 +181,9 @@ def _load():
         "moe_forward_q8": (st, [cfgp, vp, i64, vp, vp, vp, ctypes.POINTER(Q8Weights), vp, vp, vp, vp, vp, vp, sz, vp,
                                 op]),
         "moe_convert_bf16_to_f16": (st, [vp, vp, i64, vp, vp]),
+        "moe_ep_send": (st, [cfgp, i64, vp, vp, vp, vp, vp, vp]),
+        "moe_ep_recv": (st, [vp, ctypes.c_int32, ctypes.c_int32, i64, vp, vp]),
+        "moe_ep_scatter_back": (st, [vp, vp, i64, i64, ctypes.c_int32, vp, vp]),
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -237,6 +240,7 @@ class Workspace:
 
     def __init__(self, cfg, max_tokens: int, device="cuda", nbytes: int | None = None):
         self.nbytes = moe_workspace_size(cfg, max_tokens) if nbytes is None else int(nbytes)
+        self.max_tokens = int(max_tokens)
         self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
         base = self.buf.data_ptr()
         self.ptr = (base + 255) & ~255
@@ -532,3 +536,62 @@ def moe_forward_q8(cfg, x, router_w, expert_bias, q8: dict, ws: Workspace, ws_ga
     if return_routing:
         return y, idx, w
     return y
+
+
+# ---------------------------------------------------------------------------
+# expert parallelism: the row lists around the all-to-alls (moe_ep_*)
+# ---------------------------------------------------------------------------
+
+def ep_send(cfg, T: int, offsets, tok_of, topk_w, counts=None, row_w=None, stream=None):
+    """Per-expert row counts (int64 [E]) and the routing weight of every
+    permuted row (fp32 [T*k]; rows past offsets[E] are not written)."""
+    c = _as_cfg(cfg)
+    E, k = c.num_experts, c.num_experts_per_tok
+    dev = offsets.device
+    _require(offsets, "expert_offsets", E + 1, torch.int32)
+    _require(tok_of, "tok_of", T * k, torch.int32)
+    _require(topk_w, "topk_w", T * k, torch.float32)
+    if counts is None:
+        counts = torch.empty(E, dtype=torch.int64, device=dev)
+    if row_w is None:
+        row_w = torch.empty(T * k, dtype=torch.float32, device=dev)
+    _require(counts, "counts", E, torch.int64)
+    _require(row_w, "row_w", T * k, torch.float32)
+    _on_device(dev, offsets=offsets, tok_of=tok_of, topk_w=topk_w, counts=counts, row_w=row_w)
+    _check(lib.moe_ep_send(ctypes.byref(c), T, _p(offsets), _p(tok_of), _p(topk_w), _p(counts), _p(row_w),
+                           _stream(stream)))
+    return counts, row_w
+
+
+def ep_recv(recv_counts, R_recv: int, out=None, stream=None):
+    """Local expert id (int32 [R_recv]) of every received row, from the
+    exchanged counts recv_counts [P, n_local] (int64)."""
+    if not isinstance(recv_counts, torch.Tensor) or recv_counts.dim() != 2:
+        raise ValueError("recv_counts: expected an int64 tensor [P, n_local]")
+    P, n_local = (int(v) for v in recv_counts.shape)
+    _require(recv_counts, "recv_counts", P * n_local, torch.int64)
+    dev = recv_counts.device
+    if out is None:
+        out = torch.empty(R_recv, dtype=torch.int32, device=dev)
+    _require(out, "local_expert", R_recv, torch.int32)
+    _on_device(dev, recv_counts=recv_counts, local_expert=out)
+    _check(lib.moe_ep_recv(_p(recv_counts), P, n_local, int(R_recv), _p(out), _stream(stream)))
+    return out
+
+
+def ep_scatter_back(y_perm, tok_of, n_slots: int, out=None, stream=None):
+    """y_slots[tok_of[r]] = y_perm[r] for the rows of y_perm (fp32 [R, H])."""
+    if not isinstance(y_perm, torch.Tensor) or y_perm.dim() != 2:
+        raise ValueError("y_perm: expected an fp32 tensor [R, H]")
+    R, H = (int(v) for v in y_perm.shape)
+    _require(y_perm, "y_perm", R * H, torch.float32)
+    if not isinstance(tok_of, torch.Tensor) or tok_of.dtype != torch.int32 or tok_of.numel() < R:
+        raise ValueError(f"tok_of: expected at least {R} int32 entries")
+    dev = y_perm.device
+    if out is None:
+        out = torch.empty((n_slots, H), dtype=torch.float32, device=dev)
+    _require(out, "y_slots", n_slots * H, torch.float32)
+    _on_device(dev, y_perm=y_perm, tok_of=tok_of, y_slots=out)
+    _check(lib.moe_ep_scatter_back(_p(y_perm), _p(tok_of), R, int(n_slots), H, _p(out), _stream(stream)))
+    return out
+

@@ -308,6 +308,33 @@ moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, c
  * Blocking. */
 moe_status moe_check_device(void* ws, size_t ws_bytes, void* stream);
 
+/* Expert parallelism ([ARCH]: a distributed entry; [SHARED]: the shared MLP
+ * is never routed, so every rank keeps it). The routed experts are placed
+ * contiguously, E/P per rank. A rank routes and permutes its own T tokens; its
+ * permuted rows are then grouped by expert, hence by owner. The caller moves
+ * rows with two variable-size all-to-alls; these three calls build what the
+ * exchange needs, on the device, in the call's stream:
+ *
+ * moe_ep_send: counts[e] = expert_offsets[e+1] - expert_offsets[e] (int64
+ *   [E], the payload of the count exchange, [P, E/P] by owner) and
+ *   row_w[r] = topk_w[tok_of[r]] (fp32 [T*k]) for the rows r < expert_offsets[E]
+ *   (the routing weight travels with its row). expert_offsets [E+1], tok_of
+ *   [T*k] from moe_permute; topk_w [T*k] fp32.
+ * moe_ep_recv: the local expert id (0 .. n_local-1, int32) of every received
+ *   row. recv_counts [P * n_local] int64 is what the count exchange delivered:
+ *   rows arrive source by source, each source's grouped by local expert in
+ *   ascending order. R_recv = sum(recv_counts); rows past it get -1.
+ *   n_local = E/P; P * n_local <= 1024.
+ * moe_ep_scatter_back: y_slots[tok_of[r]] = y_perm[r] for r < R (the rows
+ *   this rank sent, returned in the order sent), fp32 [., H], H a multiple of
+ *   4; a slot outside [0, n_slots) is skipped. */
+moe_status moe_ep_send(const moe_config* cfg, int64_t T, const int32_t* expert_offsets, const int32_t* tok_of,
+                       const float* topk_w, int64_t* counts, float* row_w, void* stream);
+moe_status moe_ep_recv(const int64_t* recv_counts, int32_t P, int32_t n_local, int64_t R_recv, int32_t* local_expert,
+                       void* stream);
+moe_status moe_ep_scatter_back(const float* y_perm, const int32_t* tok_of, int64_t R, int64_t n_slots,
+                               int32_t H, float* y_slots, void* stream);
+
 /* dst[i] = fp16(src[i]) for n bf16 values, round to nearest even: a one-time
  * conversion of down-projection weights for moe_options.w_down_f16. Every
  * bf16 value of magnitude 2^-14 .. 65504 is exact in fp16; smaller ones keep

@@ -411,3 +411,21 @@ def test_component_wrappers_check_sizes(M):
         M.moe_forward_q8(wl, torch.zeros(T, H, dtype=bf), torch.zeros(E, H), None, bad_q8, ws=None)
     with pytest.raises(ValueError, match="router_w"):
         M.moe_forward_q8(wl, torch.zeros(T, H, dtype=bf), torch.zeros(E, H + 8), None, q8, ws=None)
+
+
+def test_expert_parallel_lists_reject_before_launch(M):
+    fake = ctypes.c_void_p(1 << 20)
+    n0 = M.lib.moe_launch_count()
+    assert M.lib.moe_ep_recv(fake, 33, 32, 10, fake, None) == 1 and "1024" in M.last_error()
+    assert M.lib.moe_ep_recv(fake, 0, 8, 10, fake, None) == 1
+    assert M.lib.moe_ep_recv(fake, 2, 8, -1, fake, None) == 1 and "R_recv" in M.last_error()
+    assert M.lib.moe_ep_recv(None, 2, 8, 10, fake, None) == 1 and "recv_counts" in M.last_error()
+    assert M.lib.moe_ep_scatter_back(fake, fake, 4, 4, 6, fake, None) == 1 and "multiple of 4" in M.last_error()
+    assert M.lib.moe_ep_scatter_back(ctypes.c_void_p((1 << 20) + 4), fake, 4, 4, 64, fake, None) == 1
+    assert "y_perm" in M.last_error()
+    c = _cfg(M, num_experts_per_tok=0)
+    assert M.lib.moe_ep_send(ctypes.byref(c), 4, fake, fake, fake, fake, fake, None) == 1
+    c = _cfg(M)
+    assert M.lib.moe_ep_send(ctypes.byref(c), 4, fake, fake, fake, ctypes.c_void_p((1 << 20) + 4), fake, None) == 1
+    assert "counts" in M.last_error()
+    assert M.lib.moe_launch_count() == n0

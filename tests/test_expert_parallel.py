@@ -42,6 +42,21 @@ def test_placement_and_counts():
     assert EP.received_local_experts(recv).tolist() == [0, 0, 2, 0, 1, 1, 1]
 
 
+def test_host_lists():
+    # the host form of the device lists (moe_ep_send / recv / scatter_back)
+    p = EP.ExpertPlacement(4, 2)
+    offsets = torch.tensor([0, 2, 2, 5, 6], dtype=torch.int32)
+    tok_of = torch.tensor([3, 0, 5, 1, 2, 4], dtype=torch.int32)
+    topk_w = torch.tensor([0.5, 0.25, 0.125, 1.0, 2.0, 4.0])
+    L = EP.host_lists(2)
+    counts, row_w = L.send(offsets, tok_of, topk_w, p)
+    assert counts.tolist() == [[2, 0], [3, 1]] and counts.dtype == torch.int64
+    assert row_w.tolist() == [1.0, 0.5, 4.0, 0.25, 0.125, 2.0]
+    y_perm = torch.arange(12, dtype=torch.float32).reshape(6, 2)
+    y = L.scatter_back(y_perm, tok_of, 6)
+    assert y[3].tolist() == [0.0, 1.0] and y[0].tolist() == [2.0, 3.0] and y[4].tolist() == [10.0, 11.0]
+
+
 def _oracle_experts(inp, I, lo):
     """weight * expert(row) for the rank's experts lo + local id, from the oracle."""
     def run(rows, local_expert, weight):
@@ -78,7 +93,7 @@ def _worker(rank, world, port, out_dir, case):
         placement = EP.ExpertPlacement(E, world)
         lo, _ = placement.local_range(rank)
         y_slots = EP.routed_rows_ep(x_perm, torch.from_numpy(offsets), torch.from_numpy(tok_of.astype(np.int64)),
-                                    torch.from_numpy(w), placement, _oracle_experts(inp, I, lo))
+                                    torch.from_numpy(w), placement, _oracle_experts(inp, I, lo), EP.host_lists(k))
         # combine: slot rows in slot order, then the shared MLP (held by every rank)
         y = y_slots.reshape(T, k, -1).sum(1).numpy() if T else np.zeros((0, wl["hidden_size"]))
         if wl["shared_width"] > 0:

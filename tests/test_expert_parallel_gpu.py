@@ -43,11 +43,47 @@ def test_expert_parallel_library_experts_one_rank(T):
         ws = M.Workspace(wl, T)
         offsets, _, tok_of, x_perm = M.moe_permute(wl, idx, ws, x=inp["x"], want_x_perm=True)
         placement = EP.ExpertPlacement(E, 1)
-        experts = EP.library_experts(wl, placement, inp["w_gate_up"], inp["w_down"])
-        y_slots = EP.routed_rows_ep(x_perm, offsets, tok_of, w, placement, experts)
+        ews = EP.experts_workspace(wl, placement, T * k)   # allocated once, reused by every step
+        experts = EP.library_experts(wl, placement, inp["w_gate_up"], inp["w_down"], ews)
+        lists = EP.library_lists(wl)
+        for _ in range(2):  # the same workspace twice
+            y_slots = EP.routed_rows_ep(x_perm, offsets, tok_of, w, placement, experts, lists)
+        ews.check()
         torch.cuda.synchronize()
         routed = y_slots.reshape(T, k, -1).sum(1).double().cpu().numpy()
         ref = O.moe_block(inp, dict(wl, num_shared_experts=0), logits=L)["y"]
         S.compare(routed, ref, f"expert-parallel routed sum T={T}")
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("P,n_local,T,k", [(1, 32, 40, 4), (4, 8, 300, 6), (8, 64, 1000, 8)])
+def test_device_lists_match_host_lists(P, n_local, T, k):
+    # moe_ep_send / moe_ep_recv / moe_ep_scatter_back against the host form,
+    # bit for bit, on a real permutation (rows grouped by expert)
+    B.build()
+    from grouped_top_routing_b200 import moe as M
+    E = P * n_local
+    wl = G.tiny_workload(tokens=T, hidden_size=64, num_experts=E, num_experts_per_tok=k, moe_intermediate_size=32,
+                         shared_width=0, num_shared_experts=0)
+    rng = np.random.default_rng(P * 1000 + T)
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    topk_w = torch.from_numpy(rng.random((T, k)).astype(np.float32)).cuda()
+    ws = M.Workspace(wl, T)
+    offsets, _, tok_of, _ = M.moe_permute(wl, torch.from_numpy(idx).cuda(), ws)
+    placement = EP.ExpertPlacement(E, P)
+    dev, host = EP.library_lists(wl), EP.host_lists(k)
+    c_d, w_d = dev.send(offsets, tok_of, topk_w, placement)
+    c_h, w_h = host.send(offsets.cpu(), tok_of.cpu(), topk_w.cpu(), placement)
+    assert torch.equal(c_d.cpu(), c_h) and torch.equal(w_d.cpu(), w_h)
+    # receive side: skewed counts from P sources, zeros included
+    recv_counts = torch.from_numpy(rng.integers(0, 5, size=(P, n_local)) * rng.integers(0, 2, size=(P, n_local)))
+    R = int(recv_counts.sum())
+    le_d = dev.recv(recv_counts.cuda(), R)
+    assert torch.equal(le_d.cpu(), EP.received_local_experts(recv_counts))
+    y_perm = torch.randn(T * k, 64, device="cuda")
+    y_d = dev.scatter_back(y_perm, tok_of, T * k)
+    y_h = host.scatter_back(y_perm.cpu(), tok_of.cpu(), T * k)
+    torch.cuda.synchronize()
+    assert torch.equal(y_d.cpu(), y_h)
+
