@@ -74,9 +74,9 @@ KERNEL_SOURCES = {
     "decode_fused": ["decode_fused.cu", "decode_fused.cuh", "fused_common.cuh", "route_block.cuh", "route.cuh",
                      "mbarrier.cuh", "common.cuh"],
 }
-MEASURED_TRAFFIC = {
-    ("expert_gate_up", "ling26_flash_t512"): (2884745856, "a5d1e9a9b5d9b50a"),
-    ("expert_down", "ling26_flash_t512"): (1491174528, "a5d1e9a9b5d9b50a"),
+MEASURED_TRAFFIC = {  # profiles/dram_traffic_ling26_prefill_t32768.md (fp16 down path, the default)
+    ("expert_gate_up", "ling26_flash_prefill_t32768"): (9712724224, "0f613fafdc6d1fd7"),
+    ("expert_down", "ling26_flash_prefill_t32768"): (5767136000, "0f613fafdc6d1fd7"),
 }
 
 
@@ -91,22 +91,24 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decode: str = "auto"):
+def measured_traffic(kernel: str, workload: str, overrides, ffn_path: str, decode: str = "auto",
+                     down_weights: str = "f16"):
     """Bytes per launch from the capture, or None when it no longer applies."""
     entry = MEASURED_TRAFFIC.get((kernel, workload))
-    if entry is None or overrides or ffn_path != "auto" or decode != "auto":
+    if entry is None or overrides or ffn_path != "auto" or decode != "auto" or down_weights != "f16":
         return None
     return entry[0] if kernel_source_hash(kernel) == entry[1] else None
 
 
-def algorithmic(wl, T, n_unique, weight_bytes=2.0, h_bytes=4):
+def algorithmic(wl, T, n_unique, weight_bytes=2.0, h_bytes=4, slot_bytes=4):
     """Bytes each expert pass must move, and the block's flops, given the
     number of distinct routed experts the batch touched. Expert weights count
     weight_bytes per element (2 for bf16 or fp16; 1 + 4 / group for 8-bit
     affine codes with a bf16 scale and bias per group). Activations count at
     the width this design stores them: token rows bf16 (2 B), the SwiGLU
     product h_bytes (two bf16 planes or fp32: 4 B; one fp16 plane: 2 B),
-    expert slot rows and the shared MLP output fp32 (4 B)."""
+    routed slot rows slot_bytes (fp32 4 B, fp16 2 B) and the shared MLP output
+    fp32 (4 B)."""
     H, E, k, I, Is = (wl["hidden_size"], wl["num_experts"], wl["num_experts_per_tok"],
                       wl["moe_intermediate_size"], wl["shared_width"])
     R = T * k
@@ -114,7 +116,7 @@ def algorithmic(wl, T, n_unique, weight_bytes=2.0, h_bytes=4):
     w_down = int((n_unique * I + Is) * H * weight_bytes)
     h_elems = R * I + T * Is
     gate_up_bytes = w_gate_up + (R + T) * H * 2 + h_elems * h_bytes   # weights + token rows in + h out
-    down_bytes = w_down + h_elems * h_bytes + (R + T) * H * 4          # weights + h in + fp32 rows out
+    down_bytes = w_down + h_elems * h_bytes + R * H * slot_bytes + T * H * 4  # weights + h in + rows out
     step_bytes = (w_gate_up + w_down + E * H * 4 + 2 * T * H * 2)  # weights + router + x in + y out
     gate_up_flops = 2 * H * 2 * h_elems          # gate and up projections of every routed and shared row
     down_flops = 2 * H * h_elems
@@ -341,8 +343,9 @@ def run_ours(args):
                               opts=M.options(**base_opts))
     n_unique = int(torch.unique(idx).numel())
     tc_path = not fused and (args.ffn_path == "tensor_cores" or (args.ffn_path == "auto" and T > M.STREAM_MAX_TOKENS))
+    f16_tc = f16 and tc_path  # h as one fp16 plane, routed slot rows fp16
     work = algorithmic(wl, T, n_unique, 1.0 + 4.0 / args.q8 if q8 is not None else 2.0,
-                       h_bytes=2 if (f16 and tc_path) else 4)
+                       h_bytes=2 if f16_tc else 4, slot_bytes=2 if f16_tc else 4)
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -451,7 +454,8 @@ def run_ours(args):
     else:
         kbytes = work["gate_up_bytes"] if kernel == "expert_gate_up" else work["down_bytes"]
         kflops = work["gate_up_flops"] if kernel == "expert_gate_up" else work["down_flops"]
-    traffic = None if q8 is not None else measured_traffic(kernel, args.workload, args.set, args.ffn_path, args.decode)
+    traffic = None if q8 is not None else measured_traffic(kernel, args.workload, args.set, args.ffn_path, args.decode,
+                                                           args.down_weights)
     others = {n: statistics.mean(v) for n, v in kern_ms.items() if n != kernel}
     # the bound is the resource the kernel's arithmetic intensity saturates first
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
