@@ -54,7 +54,13 @@
  *     passed in; an out-of-range id is skipped and recorded in the workspace
  *     error word, which moe_check_device() reports as MOE_ERR_DEVICE_CHECK.
  *   - Device-side waits are bounded; a wait that runs out records
- *     MOE_ERR_TIMEOUT in the same word and the kernel returns.
+ *     MOE_ERR_TIMEOUT in the same word and the kernel returns. After a
+ *     timeout, call moe_check_device (which reports it and zeroes the
+ *     header) or moe_workspace_init before the workspace's next use: the
+ *     fused decode kernel's grid barrier counts arrivals in the header, and
+ *     an interrupted count would make every later barrier wait out its limit.
+ *     For the same reason a workspace belongs to one device (the barrier's
+ *     generation size is that device's SM count).
  *
  * Shapes (T tokens, H hidden_size, E num_experts, k num_experts_per_tok,
  * I moe_intermediate_size, Is the shared MLP width):
