@@ -637,7 +637,7 @@ def main():
     ap.add_argument("--kernel", default="auto", choices=["auto", "expert_gate_up", "expert_down", "decode_fused"],
                     help="kernel whose live timing gives the roofline (auto: the fused decode kernel when the "
                          "library runs the block as one launch, else whichever expert pass takes longer)")
-    ap.add_argument("--cpu-sample", type=int, default=64)
+    ap.add_argument("--cpu-sample", type=int, default=256)
     ap.add_argument("--ref-sample", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "streaming", "tensor_cores"],
