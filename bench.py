@@ -75,8 +75,8 @@ KERNEL_SOURCES = {
                      "mbarrier.cuh", "common.cuh"],
 }
 MEASURED_TRAFFIC = {  # profiles/dram_traffic_ling26_prefill_t32768.md (fp16 down path, the default)
-    ("expert_gate_up", "ling26_flash_prefill_t32768"): (9712724224, "0f613fafdc6d1fd7"),
-    ("expert_down", "ling26_flash_prefill_t32768"): (5767136000, "0f613fafdc6d1fd7"),
+    ("expert_gate_up", "ling26_flash_prefill_t32768"): (6817733632, "465f18060116542f"),
+    ("expert_down", "ling26_flash_prefill_t32768"): (5130166528, "465f18060116542f"),
 }
 
 
