@@ -252,7 +252,10 @@ moe_status moe_combine(const moe_config* cfg, int64_t T, const float* y_slots, c
  * multiplies on the CUDA cores (fp32 sums throughout).
  * Its routing (indices and weights) is bit-identical to moe_route on the same
  * logits; its logits and output equal those of the separate kernels up to the
- * fp32 summation order of the dot products.
+ * fp32 summation order of the dot products. Larger batches run the separate
+ * kernels; on the tensor-core path with opts->w_down_f16, h and the routed
+ * slot rows handed from the down pass to the combine are fp16 (the shared
+ * MLP's rows stay fp32), half the bytes of the fp32 rows of moe_expert_ffn.
  *   logits_override [T,E] fp32 or NULL: when given, replaces the router
  *   projection (router_w may then be NULL).
  *   topk_idx_out [T,k] int32 / topk_w_out [T,k] fp32: optional copies of the
