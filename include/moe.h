@@ -372,9 +372,11 @@ uint64_t moe_launch_count(void);
  *   the process: it does not survive cudaDeviceReset (or the destruction of
  *   the device's primary context), after which this function must not be
  *   called on that device again.
- *   Calls share the array: two calls whose work overlaps on the GPU (other
- *   streams, other threads, other devices' calls are fine) race and corrupt
- *   each other's results. Each call clears what must start at zero.
+ *   Calls on one device share that device's array: two of them whose work
+ *   overlaps on the GPU (issued on different streams, or from different
+ *   threads) race and corrupt each other's results; calls in one stream, and
+ *   calls on different devices, are safe. Each call clears what must start
+ *   at zero.
  *   Invalid or repeated ids are skipped as in moe_permute; with no workspace
  *   error word to read, a caller detects them by expert_offsets[E] < T*k.
  * Arguments, layouts and ownership otherwise as moe_permute. Allocates nothing. */
