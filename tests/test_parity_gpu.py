@@ -204,6 +204,10 @@ FFN_CASES = [
                         moe_intermediate_size=64, shared_width=64)),
     ("tiny_token_major", dict(tokens=600, hidden_size=200, num_experts=6, num_experts_per_tok=2,
                               moe_intermediate_size=136, shared_width=272, num_shared_experts=2)),
+    # more permuted rows (2400) than the streaming kernels stage per block, so
+    # they read each row's slot id from global memory
+    ("tiny_many_slots", dict(tokens=300, hidden_size=64, num_experts=16, num_experts_per_tok=8,
+                             moe_intermediate_size=64, shared_width=64)),
 ]
 
 
@@ -602,6 +606,10 @@ Q8_CASES = [
     ("ling26_flash_t512", 17, 128, True),    # grouped routing; 17 tokens: several token passes
     ("ling_lite_t64", 5, 64, True),          # softmax, Is = 2I
     ("tiny_q8", 37, 32, True),
+    # 2250 permuted rows, more than the streaming kernels stage per block; the
+    # shared MLP in many 4-token blocks, 8-bit and bf16
+    ("tiny_q8", 450, 32, True),
+    ("tiny_q8", 450, 32, False),
 ]
 
 
