@@ -303,7 +303,11 @@ typedef struct {
  * shared MLP is 8-bit when w->shared_gate_up.q is set, else bf16 from
  * ws_gate_up / ws_down (the XL recipe keeps it bf16). Routing, permutation and
  * combine are those of moe_forward. H, I and Is must be multiples of 16 (one
- * 16-byte chunk of codes per lane step). ws / ws_bytes >= moe_workspace_size. */
+ * 16-byte chunk of codes per lane step). ws / ws_bytes >= moe_workspace_size.
+ * Arithmetic: per 16 inputs of one group, scale * sum(q * v) + bias * sum(v)
+ * in fp32, the products q * v formed exactly on activations scaled by 2^33;
+ * activations x and the fp32 SwiGLU products h must stay below 2^95 in
+ * magnitude (larger ones give non-finite outputs). */
 moe_status moe_forward_q8(const moe_config* cfg, const uint16_t* x, int64_t T, const float* router_w,
                           const float* expert_bias, const float* logits_override, const moe_q8_weights* w,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down, uint16_t* y,
