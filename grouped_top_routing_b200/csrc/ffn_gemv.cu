@@ -333,6 +333,9 @@ __device__ __forceinline__ void prefetch_down_item(const FfnArgs& a, const Stage
 // gate row and up row (bf16, or 8-bit affine when Q8) against up to MT tokens
 // per pass. The shared MLP, which sees every token, has one item per (j,
 // block of MT tokens), so its passes spread over warps like the experts'.
+// Launch bounds: the 8-bit kernels ask for two resident 256-thread blocks per
+// SM (at most 128 registers a thread); a minimum of 0 leaves the bf16
+// kernels' register use to the compiler, as with no minimum at all.
 template <int MT, bool Q8>
 __global__ void __launch_bounds__(256, Q8 ? 2 : 0) gemv_gate_up_kernel(FfnArgs a) {
   pdl_launch_dependents();
